@@ -1,0 +1,385 @@
+"""Pins for the oracle: each check ties it to something other than itself.
+
+Sources: the OSC page ("W4A4量化技术：OSC框架如何实现高效LLM部署", coreui.cn/article/2607942.html)
+for the method (§2.2 density, §2.3 tiers, §3.1 Algorithm 1, §3.2 extraction, microscaling and the
+dual-path equation), the OCP MX v1.0 element formats that the path names (E2M1, E4M3, E8M0), and
+mathematics: brute-force nearest-value rounding, closed-form thresholds, library matmul on
+dequantized values, exact-representability identities.
+"""
+import os
+
+import numpy as np
+import pytest
+
+from w4a4_outlier_separated_b200 import inputs as I
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_table(name):
+    rows = []
+    for line in open(os.path.join(GOLD, name)):
+        line = line.strip()
+        if line and not line.startswith("#"):
+            rows.append(line.split())
+    return rows
+
+
+def _all_finite_bf16():
+    b = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    return b[(b & 0x7F80) != 0x7F80]
+
+
+# ---- element formats ------------------------------------------------------------------
+
+def test_e2m1_code_table_and_counts(oracle):
+    rows = _read_table("e2m1_code_table.txt")
+    assert len(rows) == 16 == 2 ** 4                      # 4-bit code: 16 values
+    for code_s, val_s in rows:
+        v = oracle.decode_e2m1(int(code_s, 16))
+        assert v == float(val_s) and np.signbit(v) == val_s.startswith("-")
+    mags = sorted({abs(oracle.decode_e2m1(c)) for c in range(16)})
+    assert len(mags) == 8 == 2 ** 3                       # 3 magnitude bits: 8 levels
+    assert len({oracle.decode_e2m1(c) for c in range(16)}) == 15   # +0 == -0
+
+
+def _nearest_even(a, table_vals, table_codes, mant_mask):
+    """Brute force: the nearest representable magnitude; on a tie, the code with an even mantissa
+    (adjacent codes always differ in their lowest mantissa bit)."""
+    d = np.abs(a[:, None] - table_vals[None, :])
+    cand = d == d.min(axis=1, keepdims=True)
+    even = (table_codes & mant_mask) == 0
+    score = cand.astype(np.int64) * 2 + (cand & even[None, :])
+    return table_codes[np.argmax(score, axis=1)]
+
+
+def _bruteforce_e2m1(v):
+    mags = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], dtype=np.float64)
+    codes = np.arange(8)
+    a = np.minimum(np.abs(v), 6.0)                # saturation beyond the largest element
+    mag = _nearest_even(a, mags, codes, 1)
+    return np.where(np.signbit(v), 8, 0) | mag
+
+
+def _blocks_with_anchor(anchor_bits, vals_bits, per=31):
+    n = len(vals_bits)
+    nb = (n + per - 1) // per
+    pad = np.zeros(nb * per, dtype=np.uint16)
+    pad[:n] = vals_bits
+    X = np.concatenate([np.full((nb, 1), anchor_bits, np.uint16), pad.reshape(nb, per)], axis=1)
+    return X, n
+
+
+@pytest.mark.parametrize("shift", [0, 10, -60, 100])
+def test_e2m1_rounding_matches_bruteforce(oracle, shift):
+    """Every finite bf16 value within the anchor's block range, at several scales: the oracle's
+    binade-quantum rounding must equal a brute-force nearest search with ties to even."""
+    anchor = I.bf16_bits(np.array([7.5 * 2.0 ** shift]))[0]       # floor(log2 7.5) - 2 = 0
+    b = _all_finite_bf16()
+    f = I.bf16_to_f32(b).astype(np.float64)
+    keep = np.abs(f) <= 7.5 * 2.0 ** shift
+    vals = b[keep]
+    X, n = _blocks_with_anchor(anchor, vals)
+    codes, exps = oracle.mx_quantize(X, 32)
+    assert np.all(exps == shift)
+    got = codes[:, 1:].reshape(-1)[:n]
+    v = I.bf16_to_f32(vals).astype(np.float64) / 2.0 ** shift
+    want = _bruteforce_e2m1(v)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, (v[bad[:5]], got[bad[:5]], want[bad[:5]])
+
+
+def test_e2m1_known_ties(oracle):
+    # ties: 0.25->0, 0.75->1, 1.25->1, 1.75->2, 2.5->2, 3.5->4, 5->4; saturation 7->6
+    v = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0, -0.1, -0.25])
+    X = I.bf16_bits(np.concatenate([[7.5], v, np.zeros(32 - 1 - len(v))]))[None, :]
+    codes, exps = oracle.mx_quantize(X, 32)
+    assert exps[0, 0] == 0
+    dec = [oracle.decode_e2m1(int(c)) for c in codes[0, 1:1 + len(v)]]
+    assert dec[:8] == [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0, 6.0]
+    assert codes[0, 9] == 0x8 and codes[0, 10] == 0x8     # negative values rounding to 0 keep the sign
+
+
+def _e4m3_table():
+    codes = np.arange(128)
+    E, m = codes >> 3, codes & 7
+    vals = np.where(E == 0, m * 2.0 ** -9, (1 + m / 8.0) * 2.0 ** (E - 7.0))
+    ok = codes != 0x7F                                     # 0x7F is NaN
+    return vals[ok], codes[ok]
+
+
+def test_e4m3_decode_definition(oracle):
+    vals, codes = _e4m3_table()
+    for v, c in zip(vals, codes):
+        assert oracle.decode_e4m3(int(c)) == v
+        assert oracle.decode_e4m3(int(c) | 0x80) == -v
+    assert vals.max() == 448.0 and np.isnan(oracle.decode_e4m3(0x7F))
+
+
+@pytest.mark.parametrize("shift", [0, 7, -50])
+def test_e4m3_rounding_matches_bruteforce(oracle, shift):
+    anchor = I.bf16_bits(np.array([480.0 * 2.0 ** shift]))[0]      # floor(log2 480) - 8 = 0
+    b = _all_finite_bf16()
+    f = I.bf16_to_f32(b).astype(np.float64)
+    vals = b[np.abs(f) <= 480.0 * 2.0 ** shift]
+    X, n = _blocks_with_anchor(anchor, vals)
+    codes, exps = oracle.mx_quantize(X, 32, oracle.FMT_E4M3)
+    assert np.all(exps == shift)
+    got = codes[:, 1:].reshape(-1)[:n]
+    v = I.bf16_to_f32(vals).astype(np.float64) / 2.0 ** shift
+    tv, tc = _e4m3_table()
+    mag = _nearest_even(np.minimum(np.abs(v), 448.0), tv, tc, 1)
+    want = np.where(np.signbit(v), 0x80, 0) | mag
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, (v[bad[:5]], got[bad[:5]], want[bad[:5]])
+
+
+def test_shared_exponent_invariant(oracle):
+    rng = np.random.default_rng(5)
+    X = I.bf16_bits(rng.standard_normal((64, 256)) * np.exp2(rng.integers(-40, 40, (64, 1))))
+    X[3, :32] = 0                                          # all-zero block
+    codes, exps = oracle.mx_quantize(X, 32)
+    f = I.bf16_to_f32(X).astype(np.float64).reshape(64, 8, 32)
+    amax = np.abs(f).max(axis=2)
+    e = exps.astype(np.float64)
+    nz = amax > 0
+    r = amax[nz] * 2.0 ** -e[nz]
+    assert np.all((r >= 4) & (r < 8))                      # 4 <= amax * 2^-e < 8
+    assert exps[3, 0] == -127
+    # fp8: 256 <= amax * 2^-e < 512
+    _, e8 = oracle.mx_quantize(X, 32, oracle.FMT_E4M3)
+    r8 = amax[nz] * 2.0 ** -e8.astype(np.float64)[nz]
+    assert np.all((r8 >= 256) & (r8 < 512))
+
+
+def test_shared_exponent_clamps_low(oracle):
+    tiny = np.array([2.0 ** -130, 2.0 ** -126, 2.0 ** -125], dtype=np.float64)
+    X = I.bf16_bits(np.repeat(tiny, 32).reshape(3, 32))
+    codes, exps = oracle.mx_quantize(X, 32)
+    assert list(exps[:, 0]) == [-127, -127, -127]
+    # 2^-125 * 2^127 = 4 -> code 6; 2^-126 -> 2 -> code 4; 2^-130 -> 0.125 -> 0
+    assert list(codes[:, 0]) == [0, 4, 6]
+
+
+def test_group_sizes_share_scales(oracle):
+    rng = np.random.default_rng(6)
+    X = I.bf16_bits(rng.standard_normal((4, 256)) * np.array([[1], [100], [0.01], [3]]))
+    c64, e64 = oracle.mx_quantize(X, 64)
+    assert e64.shape == (4, 8) and np.all(e64[:, 0::2] == e64[:, 1::2])
+    c32, e32 = oracle.mx_quantize(X, 32)
+    assert np.all(e64[:, 0::2] == np.maximum(e32[:, 0::2], e32[:, 1::2]))
+    c16, e16 = oracle.mx_quantize(X, 16)
+    assert e16.shape == (4, 16)
+    assert np.all(e32 == np.maximum(e16[:, 0::2], e16[:, 1::2]))
+
+
+def test_bf16_rounding_of_doubles(oracle):
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal(2000) * np.exp2(rng.integers(-30, 30, 2000))).astype(np.float32)
+    want = I.bf16_bits(x)                                   # fp32 -> bf16 by the bit trick
+    got = np.array([oracle.double_to_bf16(float(v)) for v in x], dtype=np.uint16)
+    assert np.array_equal(got, want)
+    assert oracle.double_to_bf16(1.0 + 2.0 ** -8) == 0x3F80   # tie -> even
+    assert oracle.double_to_bf16(1.0 + 3 * 2.0 ** -8) == 0x3F82
+
+
+# ---- Algorithm 1 and the density --------------------------------------------------------
+
+def _group_rows(vals_list, G=32):
+    return I.bf16_bits(np.array(vals_list, dtype=np.float64))
+
+
+def test_table_picks_consistent_channel(oracle):
+    rng = np.random.default_rng(8)
+    S, G = 40, 32
+    X = rng.standard_normal((S, 3 * G)) * 0.5
+    X[:, 0 * G + 3] = 100.0                  # group 0: channel 3 on every token
+    X[:12, 1 * G + 0] = -90.0                # group 1: channel 0, 12 tokens (j* = 0 is valid)
+    X[:3, 2 * G + 7] = 90.0                  # group 2: only 3 events < min_hits
+    L = oracle.build_table(I.bf16_bits(X), G, alpha=5.0, min_hits=5)
+    assert list(L) == [3, 0, -1]
+
+
+def test_table_tie_goes_to_lowest_channel(oracle):
+    S, G = 20, 32
+    X = np.full((S, G), 0.25)
+    X[:10, 9] = 50.0
+    X[10:, 5] = 50.0
+    L = oracle.build_table(I.bf16_bits(X), G, alpha=5.0, min_hits=5)
+    assert list(L) == [5]
+    X = np.zeros((S, G))                     # all-zero group: no events
+    assert list(oracle.build_table(I.bf16_bits(X), G, 5.0, 1)) == [-1]
+
+
+def test_event_threshold_closed_form(oracle):
+    """Group [a, 1 x 31]: an event iff 32 a >= alpha (a + 31), i.e. a >= 31 alpha / (32 - alpha)."""
+    alpha, G = 5.0, 32
+    thr = 31 * alpha / (G - alpha)           # 5.7407...
+    for a, expect in [(5.5, 0), (5.75, 1), (6.0, 1), (5.625, 0)]:
+        X = np.ones((6, G))
+        X[:, 4] = a
+        nh, nt = oracle.density(I.bf16_bits(X), G, np.array([4], np.int8), alpha)
+        assert nt[0] == 6 * expect and nh[0] == nt[0], (a, thr)
+    # alpha + 1 raises the threshold: a = 6 stops being an event at alpha = 6 (thr = 7.15)
+    X = np.ones((6, G)); X[:, 4] = 6.0
+    assert oracle.density(I.bf16_bits(X), G, np.array([4], np.int8), 6.0)[1][0] == 0
+
+
+def test_table_recovers_planted_qkv(oracle):
+    c = I.qkv_case(1)
+    L = oracle.build_table(c.calib, 32, alpha=5.0, min_hits=5)
+    assert np.array_equal(L, c.planted)
+    assert (L >= 0).sum() == round(0.7 * 128)
+
+
+def test_density_on_planted_tiny(oracle):
+    c = I.tiny_case()
+    nh, nt = oracle.density(c.X, 32, c.planted, 5.0)
+    planted = c.planted >= 0
+    assert np.all(nh[planted] == nt[planted]) and np.all(nt[planted] > 0)   # C_k = 1
+    assert nt[planted].sum() >= 0.8 * 16 * 6                                  # ~90% of tokens
+
+
+def test_density_tiers_follow_table1(oracle):
+    bands = {r[0]: tuple(map(float, r[1:])) for r in _read_table("table1_density_bands.txt")}
+    q = I.qkv_case(1024)
+    L = oracle.build_table(q.calib, 32)
+    nh, nt = oracle.density(q.X, 32, L)
+    cq = (nh[nt > 0] / nt[nt > 0]).mean()
+    assert cq > bands["tier_high"][0]                       # attention input: static protection
+    w = I.w2_case(M=512, calib_tokens=1536)
+    Lw = oracle.build_table(w.calib, 32)
+    nh, nt = oracle.density(w.X, 32, Lw)
+    cw = (nh[nt > 0] / nt[nt > 0]).mean()
+    lo, hi = bands["w2"]
+    assert lo <= cw <= hi and cw < bands["tier_fp8"][0]     # W2: FP8 fallback tier
+
+
+# ---- extraction, reconstruction and the dual-path product -----------------------------
+
+def test_extract_moves_table_values(oracle):
+    c = I.tiny_case()
+    K_L = 16
+    Xz, B = oracle.extract(c.X, 32, c.planted, K_L)
+    cols = [k * 32 + int(j) for k, j in enumerate(c.planted) if j >= 0]
+    assert np.array_equal(B[:, :len(cols)], c.X[:, cols])
+    assert np.all(B[:, len(cols):] == 0)
+    assert np.all(Xz[:, cols] == 0)
+    mask = np.ones(256, bool); mask[cols] = False
+    assert np.array_equal(Xz[:, mask], c.X[:, mask])
+    with pytest.raises(ValueError):
+        oracle.extract(c.X, 32, c.planted, len(cols) - 1)
+
+
+def test_reconstruction_bound(oracle):
+    c = I.qkv_case(64)
+    L = c.planted
+    K_L = I.pad16(oracle.table_count(L))
+    Xz, B = oracle.extract(c.X, 32, L, K_L)
+    codes, exps = oracle.mx_quantize(Xz, 32)
+    deq = oracle.mx_dequantize(codes, exps)
+    cols = [k * 32 + int(j) for k, j in enumerate(L) if j >= 0]
+    rec = deq.copy()
+    rec[:, cols] = I.bf16_to_f32(B[:, :len(cols)])
+    x = I.bf16_to_f32(c.X).astype(np.float64)
+    err = np.abs(rec - x)
+    assert np.all(err[:, cols] == 0)                        # table slots are exact
+    scale = np.repeat(2.0 ** exps.astype(np.float64), 32, axis=1)
+    v = np.abs(I.bf16_to_f32(Xz).astype(np.float64)) / scale
+    half = np.where(v <= 2, 0.25, np.where(v <= 4, 0.5, 1.0)) * scale
+    inside = v <= 6
+    assert np.all(err[inside] <= half[inside])
+    sat = ~inside
+    assert np.all(np.isclose(err[sat], (v[sat] - 6) * scale[sat], rtol=0, atol=0))
+    assert np.all(err[sat] < 2 * scale[sat])
+
+
+def test_linear_equals_matmul_of_dequantized(oracle):
+    """The dual-path product is a matmul of dequantized operands plus B W_L^T (library matmul)."""
+    c = I.tiny_case()
+    L, K_L = c.planted, 16
+    cw, ew, WL = oracle.osc_prepare_weight(c.W, 32, L, K_L)
+    r = oracle.osc_forward(c.X, 32, L, K_L, cw, ew, WL)
+    want = oracle.mx_dequantize(r["cx"], r["ex"]) @ oracle.mx_dequantize(cw, ew).T
+    want += I.bf16_to_f32(r["B"]).astype(np.float64) @ I.bf16_to_f32(WL).astype(np.float64).T
+    assert np.allclose(r["Y"], want, rtol=1e-12, atol=1e-12)
+    rows = np.array([3, 0, 15], np.int32)
+    r2 = oracle.osc_forward(c.X, 32, L, K_L, cw, ew, WL, rows=rows)
+    assert np.array_equal(r2["Y"], r["Y"][rows])
+
+
+def _representable(rng, rows, K, V=32, e_range=(-8, 3)):
+    """Rows whose every V-block is exactly an E2M1 grid times 2^e, with the block max at 4 or 6."""
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    q = rng.choice(grid, size=(rows, K)) * rng.choice([-1, 1], size=(rows, K))
+    q[:, ::V] = rng.choice([4.0, 6.0], size=(rows, K // V)) * rng.choice([-1, 1], size=(rows, K // V))
+    e = rng.integers(e_range[0], e_range[1], size=(rows, K // V))
+    return q * np.repeat(2.0 ** e, V, axis=1)
+
+
+def test_osc_is_exact_on_representable_inputs(oracle):
+    """If the non-table values of X and all of W are exactly MXFP4-representable, the dual-path
+    output equals X W^T exactly: any dropped term, wrong column or transposed W_L breaks it."""
+    rng = np.random.default_rng(11)
+    M, K, N, G = 24, 256, 40, 32
+    x = _representable(rng, M, K)
+    w = _representable(rng, N, K)
+    L = np.array([5, -1, 0, 31, -1, 12, 7, -1], np.int8)
+    for k, j in enumerate(L):
+        if j >= 0:
+            x[:, k * G + int(j)] = rng.choice([-1, 1], size=M) * rng.uniform(200, 900, size=M)
+    X, W = I.bf16_bits(x), I.bf16_bits(w)
+    xf, wf = I.bf16_to_f32(X).astype(np.float64), I.bf16_to_f32(W).astype(np.float64)
+    K_L = 16
+    cw, ew, WL = oracle.osc_prepare_weight(W, G, L, K_L)
+    r = oracle.osc_forward(X, G, L, K_L, cw, ew, WL)
+    assert np.allclose(r["Y"], xf @ wf.T, rtol=1e-13, atol=1e-9)
+    # and without the table the outliers wreck the same product (MXFP4 direct)
+    L0 = np.full(8, -1, np.int8)
+    cw0, ew0, _ = oracle.osc_prepare_weight(W, G, L0, 0)
+    r0 = oracle.osc_forward(X, G, L0, 0, cw0, ew0, None)
+    assert np.abs(r0["Y"] - xf @ wf.T).max() > 1.0
+
+
+def test_all_minus_one_table_is_mxfp4_direct(oracle):
+    c = I.tiny_case()
+    L0 = np.full(8, -1, np.int8)
+    assert oracle.table_count(L0) == 0
+    cw, ew, WL = oracle.osc_prepare_weight(c.W, 32, L0, 0)
+    r = oracle.osc_forward(c.X, 32, L0, 0, cw, ew, WL)
+    assert r["B"].shape == (16, 0) and np.array_equal(r["Xz"], c.X)
+    cx, ex = oracle.mx_quantize(c.X, 32)
+    direct = oracle.mx_dequantize(cx, ex) @ oracle.mx_dequantize(cw, ew).T
+    assert np.allclose(r["Y"], direct, rtol=1e-12, atol=1e-12)
+
+
+def test_fp8_fallback_exact_on_representable(oracle):
+    rng = np.random.default_rng(12)
+    M, K, N = 8, 128, 16
+    g = np.array([0, 2 ** -9, 0.5, 1.125, 3.5, 15, 104, 256, 448])
+    def rep(rows):
+        q = rng.choice(g, size=(rows, K)) * rng.choice([-1, 1], size=(rows, K))
+        q[:, ::32] = 448.0
+        return q * np.repeat(2.0 ** rng.integers(-12, -4, size=(rows, K // 32)), 32, axis=1)
+    x, w = rep(M), rep(N)
+    X, W = I.bf16_bits(x), I.bf16_bits(w)
+    r = oracle.fp8_forward(X, W)
+    xf, wf = I.bf16_to_f32(X).astype(np.float64), I.bf16_to_f32(W).astype(np.float64)
+    assert np.allclose(r["Y"], xf @ wf.T, rtol=1e-13, atol=1e-12)
+
+
+def test_group_size_sweep_roundtrip(oracle):
+    """G = 16 / 32 / 64 all reduce the error of the same layer relative to MXFP4 direct."""
+    c = I.ffn_case(32, M=32, calib_tokens=256)
+    Wsmall = c.W[:64]
+    xf = I.bf16_to_f32(c.X).astype(np.float64)
+    ref = xf @ I.bf16_to_f32(Wsmall).astype(np.float64).T
+    for G in (16, 32, 64):
+        L = I.planted_table(I.make_structure(4096, 0.65, seed=1003), G)
+        K_L = I.pad16(oracle.table_count(L))
+        cw, ew, WL = oracle.osc_prepare_weight(Wsmall, G, L, K_L)
+        r = oracle.osc_forward(c.X, G, L, K_L, cw, ew, WL)
+        L0 = np.full(4096 // G, -1, np.int8)
+        cw0, ew0, _ = oracle.osc_prepare_weight(Wsmall, G, L0, 0)
+        r0 = oracle.osc_forward(c.X, G, L0, 0, cw0, ew0, None)
+        assert np.abs(r["Y"] - ref).mean() < 0.8 * np.abs(r0["Y"] - ref).mean()
