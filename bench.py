@@ -1,0 +1,346 @@
+"""Benchmark of the OSC W4A4 linear layer (quantize + dual-path product) on B200.
+
+Workload (default): the Qwen3-8B-shaped fused QKV projection, M=2048 tokens, K=4096,
+N=6144, G=32, table from Algorithm 1 (alpha=5) on 3x512 calibration tokens; synthetic seeded
+inputs with the outlier structure of the OSC page (its Qwen3 activations are not available).
+One step = osc_quantize(X) + osc_linear over one batch with the weights prepared offline.
+The metric counts the useful 2*M*N*K flops per step (the compensation flops are reported
+apart). Between timed steps L2 is flushed (a 512 MiB write) outside the timed events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl osc|reference]
+
+Prints one JSON line (rank 0). Under torchrun each rank runs its own batch (weak scaling; the
+token rows shard with no data-path collective); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "OSC W4A4 linear TFLOP/s (M=2048, K=4096, N=6144) and % of B200 FP4 roofline"
+M_, K_, N_, G_ = 2048, 4096, 6144, 32
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["osc", "reference"], default="osc")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, dev_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(dev_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                for k, v in self.REASONS.items():
+                    if r & v:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv is not None:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def src_hash(paths):
+    h = hashlib.sha1()
+    for p in paths:
+        h.update(open(os.path.join(ROOT, p), "rb").read())
+    return h.hexdigest()[:16]
+
+
+LINEAR_SRC = ["w4a4_outlier_separated_b200/csrc/osc_linear.cu", "w4a4_outlier_separated_b200/csrc/osc_device.cuh"]
+
+
+def committed_traffic():
+    """DRAM bytes per osc_linear launch from the committed ncu summary, if the kernel source
+    is the one the counters were taken on."""
+    p = os.path.join(ROOT, "profiles", "osc_linear_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("source_sha1") != src_hash(LINEAR_SRC):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+def make_workload(rank: int):
+    """QKV M=2048 inputs (per-rank token seed), table by Algorithm 1 on the GPU."""
+    import torch
+    from w4a4_outlier_separated_b200 import inputs as I
+    from w4a4_outlier_separated_b200 import osc
+    st = I.make_structure(K_, 0.70, seed=1002)
+    X = I.gen_tokens(st, M_, seed=1002 + M_ + 7919 * rank, spike_frac=0.05)
+    calib = I.gen_tokens(st, 1536, seed=1102, spike_frac=0.05)
+    W = I.gen_weights(N_, K_, seed=2002)
+    dev = torch.device("cuda")
+    Xd = torch.from_numpy(X.view(np.int16)).to(dev)
+    Wd = torch.from_numpy(W.view(np.int16)).to(dev)
+    Cd = torch.from_numpy(calib.view(np.int16)).to(dev)
+    Ld = torch.empty(K_ // G_, dtype=torch.int8, device=dev)
+    osc.osc_build_table(Cd, G_, 5.0, 5, Ld)
+    K_L = osc.osc_table_kl(Ld.cpu().numpy())
+    QW, SW, WL = osc.prepare_weight(Wd, G_, Ld, K_L)
+    QX, SX, B = osc.alloc_quantize_outputs(M_, K_, G_, K_L, dev)
+    Y = torch.empty((M_, N_), dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize()
+    return dict(X=X, Xd=Xd, Ld=Ld, K_L=K_L, QW=QW, SW=SW, WL=WL, QX=QX, SX=SX, B=B, Y=Y, calib=calib, W=W)
+
+
+def run_osc(args):
+    import torch
+    import torch.distributed as dist
+    from w4a4_outlier_separated_b200 import osc
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev_index = torch.cuda.current_device()
+    wl = make_workload(rank)
+    K_L = wl["K_L"]
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+
+    def step():
+        osc.osc_quantize(wl["Xd"], G_, wl["Ld"], K_L, wl["QX"], wl["SX"], wl["B"])
+        osc.osc_linear(wl["QX"], wl["SX"], wl["B"], wl["QW"], wl["SW"], wl["WL"], M_, N_, K_, G_, K_L, wl["Y"])
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev_index) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            osc.osc_quantize(wl["Xd"], G_, wl["Ld"], K_L, wl["QX"], wl["SX"], wl["B"])
+            ev[i][1].record(stream)
+            osc.osc_linear(wl["QX"], wl["SX"], wl["B"], wl["QW"], wl["SW"], wl["WL"], M_, N_, K_, G_, K_L, wl["Y"])
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    code, raw = osc.osc_status()
+    if code != 0:
+        raise RuntimeError(f"device status {code} ({raw}) after the timed steps")
+    tq = np.array([e[0].elapsed_time(e[1]) for e in ev])
+    tl = np.array([e[1].elapsed_time(e[2]) for e in ev])
+    step_ms = float((tq + tl).mean())
+    q_ms, l_ms = float(tq.mean()), float(tl.mean())
+    if ws > 1:
+        t = torch.tensor([step_ms, q_ms, l_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms, q_ms, l_ms = (float(v) for v in t.tolist())
+
+    # end to end through the public API with host buffers: pinned X in, pinned Y out
+    Xh = torch.from_numpy(wl["X"].view(np.int16)).pin_memory()
+    Yh = torch.empty((M_, N_), dtype=torch.bfloat16).pin_memory()
+    Xd2 = torch.empty_like(wl["Xd"])
+    e2e_steps = max(10, min(args.steps, 50))
+    for _ in range(3):
+        Xd2.copy_(Xh, non_blocking=True)
+        step()
+        Yh.copy_(wl["Y"], non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        Xd2.copy_(Xh, non_blocking=True)
+        osc.osc_quantize(Xd2, G_, wl["Ld"], K_L, wl["QX"], wl["SX"], wl["B"])
+        osc.osc_linear(wl["QX"], wl["SX"], wl["B"], wl["QW"], wl["SW"], wl["WL"], M_, N_, K_, G_, K_L, wl["Y"])
+        Yh.copy_(wl["Y"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if ws > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    flops = 2.0 * M_ * N_ * K_
+    comp_flops = 2.0 * M_ * N_ * K_L
+    peaks, src = measured_peaks()
+    fp4_peak = 4.0 * peaks["bf16_tflops"]
+    achieved = flops / (l_ms * 1e-3) / 1e12
+    quant_bytes = M_ * K_ * 2 + M_ * K_ // 2 + M_ * K_ // 32 + M_ * K_L * 2
+    res = None
+    if rank == 0:
+        res = {
+            "metric": METRIC, "value": round(ws * flops / (step_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(step_ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e2m1",
+            "data": "synthetic (seeded; Qwen3-8B QKV shapes, outlier structure of the OSC page)",
+            "config": {"workload": "qkv_proj M=2048 K=4096 N=6144 G=32 (Qwen3-8B fused QKV)",
+                       "global_batch": ws * M_, "K": K_, "N": N_, "G": G_, "K_L": K_L,
+                       "table": "Algorithm 1, alpha=5, min_hits=5, 1536 calibration tokens",
+                       "parallelism": f"dp{ws} (token rows, no collective)",
+                       "l2": "flushed between steps (512 MiB write, outside the timed events)",
+                       "compute": "MXFP4 E2M1 x E2M1 block-scaled + BF16 compensation, fp32 accumulate, bf16 out"},
+            "kernels": {"osc_quantize_ms": round(q_ms, 5), "osc_linear_ms": round(l_ms, 5),
+                        "osc_quantize_GBps": round(quant_bytes / (q_ms * 1e-3) / 1e9, 1),
+                        "osc_quantize_hbm_frac": round(quant_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+                        "compensation_tflop_per_step": comp_flops / 1e12},
+            "roofline": {"bound": "tensor", "kernel": "osc_linear", "achieved": round(achieved, 1),
+                         "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
+                         "peak_source": f"{src} bf16 burst x 4 (nominal FP4/BF16 ratio)",
+                         "traffic": committed_traffic()},
+            "e2e": {"value": round(ws * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": M_ * K_ * 2, "d2h_bytes_per_step": M_ * N_ * 2,
+                    "ms_per_step": round(e2e_ms, 4)},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk.summary(),
+        }
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return res, wl
+
+
+def oracle_rows_timing(X, W, calib, rows_per_call: int, calls: int):
+    """Time the oracle (single-threaded C, fp64) on row samples of the same layer: extraction,
+    quantization and the dual-path product for `rows_per_call` rows, `calls` times. The table
+    (Algorithm 1) and the weight preparation are offline and outside the timing."""
+    from oracle import oracle as O
+    from w4a4_outlier_separated_b200 import inputs as I
+    L = O.build_table(calib, G_)
+    K_L = I.pad16(O.table_count(L))
+    cw, ew, WL = O.osc_prepare_weight(W, G_, L, K_L)
+    rng = np.random.default_rng(0)
+    times = []
+    for _ in range(calls):
+        r0 = int(rng.integers(0, M_ - rows_per_call + 1))
+        Xs = np.ascontiguousarray(X[r0:r0 + rows_per_call])
+        t0 = time.perf_counter()
+        O.osc_forward(Xs, G_, L, K_L, cw, ew, WL)
+        times.append(time.perf_counter() - t0)
+    return np.array(times)
+
+
+def cpu_baseline(X, W, calib, target_s: float):
+    probe = oracle_rows_timing(X, W, calib, 2, 1)[0] / 2
+    rows = int(max(2, min(M_, target_s / max(probe, 1e-6))))
+    t = oracle_rows_timing(X, W, calib, rows, 1)[0]
+    flops = 2.0 * rows * N_ * K_
+    return {"value": round(flops / t / 1e12, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} of the {M_} token rows of the same QKV layer (extract + quantize + dual-path "
+                      f"product in fp64, single thread); {t:.1f} s; table and weight prep offline"}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    from w4a4_outlier_separated_b200 import inputs as I
+    st = I.make_structure(K_, 0.70, seed=1002)
+    X = I.gen_tokens(st, M_, seed=1002 + M_, spike_frac=0.05)
+    calib = I.gen_tokens(st, 1536, seed=1102, spike_frac=0.05)
+    W = I.gen_weights(N_, K_, seed=2002)
+    probe = oracle_rows_timing(X, W, calib, 2, 1)[0] / 2
+    budget = 120.0
+    rows = int(max(1, min(64, budget / ((args.steps + max(args.warmup, 3)) * max(probe, 1e-6)))))
+    oracle_rows_timing(X, W, calib, rows, max(args.warmup, 3))
+    t = oracle_rows_timing(X, W, calib, rows, args.steps)
+    flops = 2.0 * rows * N_ * K_
+    ms = float(t.mean() * 1e3)
+    val = round(flops / t.mean() / 1e12, 6)
+    return {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeds as the GPU arm)",
+        "config": {"workload": "qkv_proj M=2048 K=4096 N=6144 G=32 (Qwen3-8B fused QKV)",
+                   "sample_rows_per_step": rows, "parallelism": "rank 0 only"},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{rows} token rows per step of the same layer, fp64 single thread"},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        res = run_reference(args)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    res, wl = run_osc(args)
+    if res is not None:
+        if not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(wl["X"], wl["W"], wl["calib"], args.cpu_seconds)
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,176 @@
+/*
+ * libosc: B200 (sm_100a) OSC W4A4 linear layer behind a plain C ABI.
+ *
+ * The method is the one of the OSC page, "W4A4量化技术：OSC框架如何实现高效LLM部署"
+ * (coreui.cn/article/2607942.html): a static, offline suppression table names one outlier
+ * channel per G-wide channel group (§3.1, Algorithm 1); at run time that value is moved into
+ * a high-precision buffer B and zeroed, the zeroed tensor is microscaled to 4 bits (§3.2,
+ * Figure 2), and the layer output is the dual-path product
+ *     Y = (Q_X (x) Q_W) * S + B * W_L                         (§3.2)
+ * with W_L the bf16 weight rows of the table's channels (§3.3). Low-clustering inputs (W2)
+ * fall back to an FP8 microscaled product (§2.3, §4); MoE expert layers use a grouped form
+ * (§1, §5.2). Element formats are OCP MX: E2M1 (or E4M3) elements with one E8M0
+ * power-of-two scale per block.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are caller-allocated DEVICE memory (e.g. from PyTorch); the library never
+ *     allocates or frees memory and never synchronizes the stream, except osc_status.
+ *   - Every call is asynchronous on the given stream (a cudaStream_t; NULL = legacy stream).
+ *   - bf16 values are passed as uint16_t bit patterns; 4-bit and 8-bit codes as uint8_t.
+ *   - All pointers must be 16-byte aligned (cudaMalloc / PyTorch allocations are).
+ *   - Inputs must be finite (no NaN / Inf).
+ *   - Return value: OSC_OK (0) or a negative OSC_ERR_* code; nothing is launched on error.
+ *     Errors found by a kernel while it runs (a table entry >= G, more entries than K_L,
+ *     a bounded wait that ran out) are recorded in a per-device status word that
+ *     osc_status() reads and clears.
+ *
+ * Shapes: X is M x K bf16 row-major (tokens x input channels); W is N x K bf16 row-major
+ * (output x input channels, the layout of a PyTorch Linear weight); Y is M x N bf16.
+ * K must be a multiple of 256. N must be a multiple of 16. G is 16, 32 or 64.
+ *
+ * Layouts the calls exchange (all row-major):
+ *   QX / QW  (MXFP4) rows x K/2 bytes: element k of a row in byte k/2, even k in the low nibble.
+ *            (MXFP8) rows x K bytes, one E4M3 code per element.
+ *            Codes keep the sign of the input even when the magnitude rounds to zero.
+ *   SX / SW  E8M0 scale bytes (e + 127) in the tensor-core scale layout: 512-byte atoms of
+ *            128 rows x 4 slots; slot s of row r lives at byte
+ *              ((r/128) * (K/V/4) + s/4) * 512 + (r%32)*16 + ((r%128)/32)*4 + s%4
+ *            with V = 16 for G = 16 and V = 32 otherwise (G = 64 stores its one exponent in
+ *            both 32-slots of the group). Rows are padded to a multiple of 128; the pad
+ *            rows hold 0. Size: osc_scale_bytes().
+ *            Shared exponent e = floor(log2(amax)) - 2 (E2M1) or - 8 (E4M3), clamped to
+ *            [-127, 127]; an all-zero block gets e = -127.
+ *   L        int8, K/G entries: local channel 0..G-1 of the group's outlier, or -1.
+ *   B        M x K_L bf16: column i holds the i-th table channel (groups with L >= 0 in
+ *            ascending order); columns past the entry count are 0.
+ *   W_L      N x K_L bf16: W_L[n][i] = W[n][channel of table entry i]; pad columns 0.
+ *   K_L      the compensation width: the number of table entries rounded up to a multiple
+ *            of 16 (osc_table_kl), or any larger multiple of 16.
+ */
+#ifndef OSC_H_
+#define OSC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define OSC_API __attribute__((visibility("default")))
+#else
+#define OSC_API
+#endif
+
+typedef struct CUstream_st* osc_stream_t; /* same type as cudaStream_t */
+
+enum {
+  OSC_OK = 0,
+  OSC_ERR_ARG = -1,      /* null pointer, negative or unsupported size */
+  OSC_ERR_ALIGN = -2,    /* pointer not 16-byte aligned, K % 256 != 0, N % 16 != 0, K_L % 16 != 0 */
+  OSC_ERR_G = -3,        /* G not in {16, 32, 64} */
+  OSC_ERR_CUDA = -4,     /* a CUDA runtime/driver call failed; see osc_last_cuda_error() */
+  OSC_ERR_TIMEOUT = -5,  /* (from osc_status) a kernel's bounded wait ran out */
+  OSC_ERR_TABLE = -6,    /* (from osc_status) a table entry >= G or more entries than K_L */
+  OSC_ERR_DEVICE = -7    /* the current device is not an sm_100 GPU */
+};
+
+/* Library version string. */
+OSC_API const char* osc_version(void);
+/* Human-readable text for an OSC_* code. */
+OSC_API const char* osc_error_string(int code);
+/* The cudaError_t value behind the last OSC_ERR_CUDA returned on this thread. */
+OSC_API int osc_last_cuda_error(void);
+
+/* Bytes of a scale buffer for `rows` rows of K channels with group size G (G = 16, 32, 64),
+ * or for the MXFP8 path when G == 0. Returns 0 on invalid arguments. */
+OSC_API size_t osc_scale_bytes(int rows, int K, int G);
+
+/* K_L for a table held in HOST memory: count of entries >= 0, rounded up to 16. */
+OSC_API int osc_table_kl(const int8_t* L_host, int Kg);
+
+/* §3.1 Algorithm 1 (offline), one (position, layer): S x K calibration activations Xcal
+ * -> L (K/G entries, device). alpha is the page's threshold (default 5); min_hits is the
+ * fewest events a channel needs to be protected (default 5). An event of group k on token t
+ * is the channel j_t of largest |x| (lowest j on ties) when G*|x_max| >= alpha * sum|x_j|
+ * (sum in fp32 over ascending j, comparison in fp64); L[k] is the channel with the most
+ * events (lowest on ties) if it has >= min_hits, else -1. */
+OSC_API int osc_build_table(const uint16_t* Xcal, int S, int K, int G, float alpha, int min_hits,
+                    int8_t* L, osc_stream_t stream);
+
+/* §3.2, Figure 2 (online): extraction + zeroing through the table, then MXFP4 quantization
+ * of the zeroed tensor. X (M x K bf16) -> QX (M x K/2), SX (osc_scale_bytes(M, K, G)),
+ * B (M x K_L bf16). L may be NULL (no table: plain MXFP4; then K_L must be 0 and B may be
+ * NULL). X is not modified. */
+OSC_API int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int K_L,
+                 uint8_t* QX, uint8_t* SX, uint16_t* B, osc_stream_t stream);
+
+/* §3.3 weight side (offline): W (N x K bf16) -> QW (N x K/2), SW (osc_scale_bytes(N, K, G))
+ * quantized with no table (its outlier columns meet zeroed activations), and
+ * W_L (N x K_L bf16) gathered through L (device; may be NULL when K_L == 0). */
+OSC_API int osc_prepare_weight(const uint16_t* W, int N, int K, int G, const int8_t* L, int K_L,
+                       uint8_t* QW, uint8_t* SW, uint16_t* WL, osc_stream_t stream);
+
+/* §3.2 equation for Y: Y (M x N bf16, round to nearest even from the fp32 accumulator)
+ *   = sum_b 2^(eX+eW) sum_{i in b} qX qW  +  B * W_L^T.
+ * Yf32 (M x N fp32) may be NULL; when given it receives the fp32 accumulator as well
+ * (a checking aid; it slows the call down). B and WL may be NULL when K_L == 0. */
+OSC_API int osc_linear(const uint8_t* QX, const uint8_t* SX, const uint16_t* B,
+               const uint8_t* QW, const uint8_t* SW, const uint16_t* WL,
+               int M, int N, int K, int G, int K_L, uint16_t* Y, float* Yf32,
+               osc_stream_t stream);
+
+/* §4 FP8 fallback, quantize side: X (M x K bf16) -> QX8 (M x K E4M3 codes),
+ * SX (osc_scale_bytes(M, K, 0)); per-32 E8M0 scales, no separation. Also used for the
+ * weights of the fallback. */
+OSC_API int osc_quantize_fp8(const uint16_t* X, int M, int K, uint8_t* QX8, uint8_t* SX,
+                     osc_stream_t stream);
+
+/* §4 FP8 fallback product: Y = sum_b 2^(eX+eW) sum_{i in b} qX qW over E4M3 codes. */
+OSC_API int osc_linear_fp8_fallback(const uint8_t* QX8, const uint8_t* SX, const uint8_t* QW8,
+                            const uint8_t* SW, int M, int N, int K, uint16_t* Y, float* Yf32,
+                            osc_stream_t stream);
+
+/* ---- grouped (MoE) form, §1 and §5.2 (Qwen3-30B-A3B expert layers) -------------------
+ * Tokens arrive sorted by expert: expert e owns rows off[e] .. off[e+1] of X. The grouped
+ * calls work on a PADDED row space in which expert e's rows start at poff[e], a multiple of
+ * 128, so that every 128-row block belongs to one expert (mblock_expert[b] = e).
+ * osc_grouped_plan fills the three host arrays from per-expert counts. */
+
+/* counts (E entries, host) -> off (E+1), poff (E+1), mblock_expert (poff[E]/128 entries),
+ * all host arrays; returns the padded row count poff[E], or a negative code. mblock_expert
+ * may be NULL to query the size first. */
+OSC_API int osc_grouped_plan(const int* counts, int E, int* off, int* poff, int* mblock_expert,
+                     int mblock_capacity);
+
+/* Per-expert extraction + MXFP4 quantization. X: off[E] x K bf16 (device). off, poff,
+ * mblock_expert: device copies of the plan. L: E x K/G (device), expert e's table at e*K/G.
+ * Outputs over the padded rows: QX (Mp x K/2), SX (osc_scale_bytes(Mp, K, G)),
+ * B (Mp x K_L bf16, K_L a common width >= every expert's entry count); pad rows are 0. */
+OSC_API int osc_quantize_grouped(const uint16_t* X, int E, const int* off, const int* poff,
+                         const int* mblock_expert, int Mp, int K, int G, const int8_t* L,
+                         int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B, osc_stream_t stream);
+
+/* Per-expert dual-path product over the padded rows. QW: E x N x K/2, SW: E blocks of
+ * osc_scale_bytes(N, K, G), WL: E x N x K_L (each expert's W_L padded to the common K_L),
+ * kl: E compensation widths (device, multiples of 16, <= K_L; NULL = K_L for all).
+ * Y: Mp x N bf16 (pad rows receive 0). */
+OSC_API int osc_linear_grouped(const uint8_t* QX, const uint8_t* SX, const uint16_t* B,
+                       const uint8_t* QW, const uint8_t* SW, const uint16_t* WL,
+                       const int* mblock_expert, const int* kl, int E, int Mp, int N, int K,
+                       int G, int K_L, uint16_t* Y, float* Yf32, osc_stream_t stream);
+
+/* Reads and clears the current device's status word (synchronizes `stream`). Returns
+ * OSC_OK, OSC_ERR_TIMEOUT or OSC_ERR_TABLE; *raw (may be NULL) gets the raw device code. */
+OSC_API int osc_status(int* raw, osc_stream_t stream);
+
+/* Tile width of the tensor-core kernels: 0 = automatic (default), 128 or 256. Applies to
+ * calls made afterwards from any thread. Returns the previous value, or OSC_ERR_ARG. */
+OSC_API int osc_set_tile_n(int bn);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OSC_H_ */

@@ -384,7 +384,10 @@ int orc_linear(const uint8_t* cx, const int16_t* ex, const uint8_t* cw,
     if (K_L < 0 || (K_L > 0 && (!B || !WL))) return -1;
     int nslot = K / V;
     int nr = rows ? nrows : M;
-    double* qx = (double*)malloc((size_t)K * sizeof(double));
+    /* decode the selected rows of X once, then each row of W once; every (t, n) sum runs in
+     * the same order as the formula: slots ascending, elements ascending within a slot, then
+     * the K_L compensation terms ascending */
+    double* qx = (double*)malloc((size_t)nr * (size_t)K * sizeof(double));
     double* qw = (double*)malloc((size_t)K * sizeof(double));
     if (!qx || !qw) { free(qx); free(qw); return -1; }
     for (int r = 0; r < nr; ++r) {
@@ -392,17 +395,21 @@ int orc_linear(const uint8_t* cx, const int16_t* ex, const uint8_t* cw,
         if (t < 0 || t >= M) { free(qx); free(qw); return -1; }
         for (int k = 0; k < K; ++k) {
             uint8_t c = cx[(int64_t)t * K + k];
-            qx[k] = (fmt == ORC_FMT_E2M1) ? orc_decode_e2m1(c) : orc_decode_e4m3(c);
+            qx[(int64_t)r * K + k] = (fmt == ORC_FMT_E2M1) ? orc_decode_e2m1(c) : orc_decode_e4m3(c);
         }
-        for (int n = 0; n < N; ++n) {
-            for (int k = 0; k < K; ++k) {
-                uint8_t c = cw[(int64_t)n * K + k];
-                qw[k] = (fmt == ORC_FMT_E2M1) ? orc_decode_e2m1(c) : orc_decode_e4m3(c);
-            }
+    }
+    for (int n = 0; n < N; ++n) {
+        for (int k = 0; k < K; ++k) {
+            uint8_t c = cw[(int64_t)n * K + k];
+            qw[k] = (fmt == ORC_FMT_E2M1) ? orc_decode_e2m1(c) : orc_decode_e4m3(c);
+        }
+        for (int r = 0; r < nr; ++r) {
+            int t = rows ? rows[r] : r;
+            const double* xr = qx + (int64_t)r * K;
             double acc = 0.0;
             for (int b = 0; b < nslot; ++b) {
                 double part = 0.0;
-                for (int i = b * V; i < (b + 1) * V; ++i) part += qx[i] * qw[i];
+                for (int i = b * V; i < (b + 1) * V; ++i) part += xr[i] * qw[i];
                 acc += ldexp(part, ex[(int64_t)t * nslot + b] + ew[(int64_t)n * nslot + b]);
             }
             for (int i = 0; i < K_L; ++i)

@@ -1,0 +1,187 @@
+"""GPU parity of the dual-path product (osc_linear, osc_linear_fp8_fallback, osc_linear_grouped)
+against the oracle's fp64 Y.
+
+Tolerance: the fp32 accumulator (the Yf32 output of the same launch) must satisfy
+max|dY| <= 1e-3 * max|Y_ref| over the compared rows. The bf16 output must equal the fp32
+accumulator rounded to bf16, and lie within 1e-3 * max|Y_ref| + 1 bf16 ulp of Y_ref."""
+import numpy as np
+import pytest
+import torch
+
+from tests._layout import bf16_ulp
+from tests.conftest import to_dev, to_np
+from w4a4_outlier_separated_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+REL = 1e-3
+
+
+def _compare(Y_bf16, Y_f32, Yref):
+    ymax = np.abs(Yref).max()
+    d32 = np.abs(Y_f32.astype(np.float64) - Yref).max()
+    assert d32 <= REL * ymax, (d32, ymax)
+    yb = I.bf16_to_f32(Y_bf16).astype(np.float64)
+    assert np.array_equal(Y_bf16, I.bf16_bits(Y_f32))            # bf16 = RNE(fp32 accumulator)
+    assert np.all(np.abs(yb - Yref) <= REL * ymax + bf16_ulp(Yref))
+
+
+def _run_osc(oracle, osc, X, W, G, L, rows=None, bn=0):
+    M, K = X.shape
+    N = W.shape[0]
+    K_L = I.pad16(oracle.table_count(L)) if L is not None else 0
+    Ld = to_dev(L) if L is not None else None
+    prev = osc.osc_set_tile_n(bn)
+    try:
+        QW, SW, WL = osc.prepare_weight(to_dev(W), G, Ld, K_L)
+        QX, SX, B = osc.quantize(to_dev(X), G, Ld, K_L)
+        Y, Yf = osc.linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, want_f32=True)
+        torch.cuda.synchronize()
+    finally:
+        osc.osc_set_tile_n(prev)
+    assert osc.osc_status() == (0, 0)
+    Lo = L if L is not None else np.full(K // G, -1, np.int8)
+    cw, ew, WLr = oracle.osc_prepare_weight(W, G, Lo, K_L)
+    sel = np.arange(M) if rows is None else np.asarray(rows)
+    ref = oracle.osc_forward(X, G, Lo, K_L, cw, ew, WLr, rows=sel)["Y"]
+    _compare(to_np(Y)[sel], to_np(Yf)[sel], ref)
+    return ref
+
+
+@pytest.mark.parametrize("bn", [128, 256])
+def test_tiny(oracle, osc, bn):
+    c = I.tiny_case()
+    _run_osc(oracle, osc, c.X, c.W, 32, c.planted, bn=bn)
+
+
+@pytest.mark.parametrize("M", [1, 16, 128, 2048])
+def test_qkv(oracle, osc, M):
+    c = I.qkv_case(M)
+    L = oracle.build_table(c.calib, 32)
+    rows = None if M <= 16 else I.sample_rows(M, 24, seed=M)
+    _run_osc(oracle, osc, c.X, c.W, 32, L, rows=rows)
+
+
+def test_qkv_both_tile_widths(oracle, osc):
+    c = I.qkv_case(2048)
+    L = oracle.build_table(c.calib, 32)
+    rows = I.sample_rows(2048, 12, seed=5)
+    for bn in (128, 256):
+        _run_osc(oracle, osc, c.X, c.W, 32, L, rows=rows, bn=bn)
+
+
+@pytest.mark.parametrize("G", [16, 32, 64])
+def test_ffn_full_size(oracle, osc, G):
+    c = I.ffn_case(G, M=4096, calib_tokens=1536)
+    L = oracle.build_table(c.calib, G)
+    _run_osc(oracle, osc, c.X, c.W, G, L, rows=I.sample_rows(4096, 8, seed=G))
+
+
+def test_w2_osc_full_size(oracle, osc):
+    c = I.w2_case(M=4096)
+    L = oracle.build_table(c.calib, 32)
+    _run_osc(oracle, osc, c.X, c.W, 32, L, rows=I.sample_rows(4096, 12, seed=7))
+
+
+@pytest.mark.parametrize("shape", [(4096, 12288, 4096), (130, 512, 144), (1, 256, 16)])
+def test_fp8_fallback(oracle, osc, shape):
+    M, K, N = shape
+    if M == 4096:
+        c = I.w2_case(M=4096)
+        X, W = c.X, c.W
+        rows = I.sample_rows(M, 12, seed=8)
+    else:
+        rng = np.random.default_rng(M)
+        X = I.bf16_bits(rng.standard_normal((M, K)) * np.exp2(rng.integers(-6, 6, (M, 1))))
+        W = I.gen_weights(N, K, seed=N)
+        rows = None
+    Xd, Wd = to_dev(X), to_dev(W)
+    QX, SX, _ = osc.alloc_quantize_outputs(M, K, 32, 0, fp8=True)
+    QW, SW, _ = osc.alloc_quantize_outputs(N, K, 32, 0, fp8=True)
+    osc.osc_quantize_fp8(Xd, QX, SX)
+    osc.osc_quantize_fp8(Wd, QW, SW)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    Yf = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    osc.osc_linear_fp8_fallback(QX, SX, QW, SW, M, N, K, Y, Yf)
+    torch.cuda.synchronize()
+    sel = np.arange(M) if rows is None else rows
+    ref = oracle.fp8_forward(X[sel], W)["Y"]
+    _compare(to_np(Y)[sel], to_np(Yf)[sel], ref)
+
+
+@pytest.mark.parametrize("bn", [128, 256])
+def test_ragged_shapes_and_compensation_width(oracle, osc, bn):
+    """M not a multiple of 128, N not a multiple of the tile, two compensation stages with a
+    partial second one (K_L = 80), entries at channel 0 and G-1."""
+    rng = np.random.default_rng(21)
+    M, K, N, G = 130, 1024, 400, 32
+    x = rng.standard_normal((M, K))
+    L = np.full(K // G, -1, np.int8)
+    idx = rng.permutation(K // G)[:70]
+    L[idx] = rng.integers(0, G, size=70)
+    L[idx[0]], L[idx[1]] = 0, G - 1
+    for k, j in enumerate(L):
+        if j >= 0:
+            x[:, k * G + int(j)] = rng.choice([-1, 1], M) * rng.uniform(20, 80, M)
+    X = I.bf16_bits(x)
+    W = I.gen_weights(N, K, seed=3)
+    _run_osc(oracle, osc, X, W, G, L, bn=bn)
+
+
+def test_all_minus_one_table_is_mxfp4_direct(oracle, osc):
+    c = I.qkv_case(128)
+    L = np.full(128, -1, np.int8)
+    _run_osc(oracle, osc, c.X, c.W[:512], 32, L)
+    _run_osc(oracle, osc, c.X, c.W[:512], 32, None)
+
+
+def _moe(oracle, osc, counts, which="gateup", rows_per_expert=None):
+    case = I.moe_case(which, E=len(counts), counts_override=counts) if counts is not None else I.moe_case(which)
+    K, N, G = case.K, case.N, 32
+    counts, E = case.counts, case.E
+    tables = np.stack([oracle.build_table(case.calib[e], G) if case.calib[e].shape[0] else
+                       np.full(K // G, -1, np.int8) for e in range(E)])
+    kls = np.array([I.pad16(oracle.table_count(tables[e])) for e in range(E)], np.int32)
+    K_L = max(16, int(kls.max()))
+    off, poff, mbe = osc.osc_grouped_plan(counts)
+    Mp = int(poff[-1])
+    offd, poffd, mbed = off.cuda(), poff.cuda(), mbe.cuda()
+    Ld = to_dev(tables)
+    QX = torch.empty((Mp, K // 2), dtype=torch.uint8, device="cuda")
+    SX = torch.empty(osc.osc_scale_bytes(Mp, K, G), dtype=torch.uint8, device="cuda")
+    B = torch.empty((Mp, K_L), dtype=torch.int16, device="cuda")
+    osc.osc_quantize_grouped(to_dev(case.X), E, offd, poffd, mbed, Mp, G, Ld, K_L, QX, SX, B)
+    sw = osc.osc_scale_bytes(N, K, G)
+    QW = torch.empty((E, N, K // 2), dtype=torch.uint8, device="cuda")
+    SW = torch.empty((E, sw), dtype=torch.uint8, device="cuda")
+    WL = torch.empty((E, N, K_L), dtype=torch.int16, device="cuda")
+    Wd = to_dev(case.W)
+    for e in range(E):
+        osc.osc_prepare_weight(Wd[e], G, Ld[e], K_L, QW[e], SW[e], WL[e])
+    Y = torch.empty((Mp, N), dtype=torch.bfloat16, device="cuda")
+    Yf = torch.empty((Mp, N), dtype=torch.float32, device="cuda")
+    osc.osc_linear_grouped(QX, SX, B, QW, SW, WL, mbed, to_dev(kls), E, Mp, N, K, G, K_L, Y, Yf)
+    torch.cuda.synchronize()
+    assert osc.osc_status() == (0, 0)
+    Yn, Yfn = to_np(Y), to_np(Yf)
+    off_n, poff_n = off.numpy(), poff.numpy()
+    for e in range(E):
+        cnt = int(counts[e])
+        # padding rows of the expert's last block come out as zeros
+        pad = slice(poff_n[e] + cnt, poff_n[e + 1])
+        assert np.all(Yfn[pad] == 0)
+        if cnt == 0:
+            continue
+        Xe = case.X[off_n[e]:off_n[e + 1]]
+        sel = np.arange(cnt) if rows_per_expert is None else np.unique(
+            np.r_[0, cnt - 1, np.random.default_rng(e).integers(0, cnt, rows_per_expert)])
+        cw, ew, WLr = oracle.osc_prepare_weight(case.W[e], G, tables[e], K_L)
+        ref = oracle.osc_forward(Xe, G, tables[e], K_L, cw, ew, WLr, rows=sel)["Y"]
+        _compare(Yn[poff_n[e] + sel], Yfn[poff_n[e] + sel], ref)
+
+
+def test_moe_grouped_small(oracle, osc):
+    _moe(oracle, osc, [130, 0, 1, 257, 64, 3, 128, 40])
+
+
+def test_moe_grouped_full_size_gateup(oracle, osc):
+    _moe(oracle, osc, None, "gateup", rows_per_expert=2)

@@ -1,0 +1,199 @@
+"""GPU parity of the quantize side (osc_quantize, osc_quantize_fp8, osc_prepare_weight,
+osc_build_table) against the oracle: codes, scales, B, W_L and table entries bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+from tests._layout import pad_rows_zero, unpack_e2m1, unswizzle_scales
+from tests.conftest import to_dev, to_np
+from w4a4_outlier_separated_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_quant(osc, X, G, L, K_L):
+    M, K = X.shape
+    Ld = to_dev(L) if L is not None else None
+    QX, SX, B = osc.quantize(to_dev(X), G, Ld, K_L)
+    torch.cuda.synchronize()
+    assert osc.osc_status() == (0, 0)
+    return to_np(QX), to_np(SX), (to_np(B) if B is not None else None)
+
+
+def _check_quant(oracle, osc, X, G, L, K_L, rows=None):
+    M, K = X.shape
+    QX, SX, B = _gpu_quant(osc, X, G, L, K_L)
+    V = 16 if G == 16 else 32
+    codes = unpack_e2m1(QX, K)
+    exps = unswizzle_scales(SX, M, K, V)
+    assert pad_rows_zero(SX, M, K, V)
+    sel = np.arange(M) if rows is None else np.asarray(rows)
+    Xs = X[sel]
+    if L is not None:
+        Xz, Bref = oracle.extract(Xs, G, L, K_L)
+        assert np.array_equal(B[sel], Bref)
+    else:
+        Xz = Xs
+    cref, eref = oracle.mx_quantize(Xz, G)
+    bad = np.argwhere(codes[sel] != cref)
+    assert bad.size == 0, f"{len(bad)} code mismatches, first {bad[:4]}"
+    assert np.array_equal(exps[sel], eref)
+
+
+def _anchor_rows(anchor, vals, K=256):
+    per = 31
+    n = len(vals)
+    nb = (n + per - 1) // per
+    nb = (nb + K // 32 - 1) // (K // 32) * (K // 32)
+    pad = np.zeros(nb * per, dtype=np.uint16)
+    pad[:n] = vals
+    blocks = np.concatenate([np.full((nb, 1), anchor, np.uint16), pad.reshape(nb, per)], axis=1)
+    return blocks.reshape(-1, K)
+
+
+def _finite_bf16():
+    b = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    return b[(b & 0x7F80) != 0x7F80]
+
+
+@pytest.mark.parametrize("shift", [0, 10, -60, -126, 100])
+def test_every_bf16_value_e2m1(oracle, osc, shift):
+    """All finite bf16 values under a block anchor: the hardware conversion, the exponent
+    from the bf16 bits and the zero-sign rule agree with the oracle bit for bit."""
+    anchor = I.bf16_bits(np.array([7.5 * 2.0 ** shift]))[0]
+    b = _finite_bf16()
+    f = I.bf16_to_f32(b).astype(np.float64)
+    X = _anchor_rows(anchor, b[np.abs(f) <= 7.5 * 2.0 ** shift])
+    _check_quant(oracle, osc, X, 32, None, 0)
+
+
+@pytest.mark.parametrize("G", [16, 64])
+def test_every_bf16_value_other_groups(oracle, osc, G):
+    b = _finite_bf16()
+    rng = np.random.default_rng(G)
+    X = rng.permutation(b)[: (len(b) // 256) * 256].reshape(-1, 256)
+    _check_quant(oracle, osc, X, G, None, 0)
+
+
+@pytest.mark.parametrize("shift", [0, 7, -50, -120])
+def test_every_bf16_value_e4m3(oracle, osc, shift):
+    anchor = I.bf16_bits(np.array([480.0 * 2.0 ** shift]))[0]
+    b = _finite_bf16()
+    f = I.bf16_to_f32(b).astype(np.float64)
+    X = _anchor_rows(anchor, b[np.abs(f) <= 480.0 * 2.0 ** shift])
+    M, K = X.shape
+    QX8, SX, _ = osc.alloc_quantize_outputs(M, K, 32, 0, fp8=True)
+    osc.osc_quantize_fp8(to_dev(X), QX8, SX)
+    torch.cuda.synchronize()
+    cref, eref = oracle.mx_quantize(X, 32, oracle.FMT_E4M3)
+    assert np.array_equal(to_np(QX8), cref)
+    assert np.array_equal(unswizzle_scales(to_np(SX), M, K, 32), eref)
+
+
+def test_tiny_planted(oracle, osc):
+    c = I.tiny_case()
+    _check_quant(oracle, osc, c.X, 32, c.planted, 16)
+
+
+@pytest.mark.parametrize("M", [1, 16, 128, 2048])
+def test_qkv_table_from_algorithm1(oracle, osc, M):
+    c = I.qkv_case(M)
+    L = oracle.build_table(c.calib, 32)
+    K_L = I.pad16(oracle.table_count(L))
+    assert K_L == 96
+    _check_quant(oracle, osc, c.X, 32, L, K_L)
+
+
+@pytest.mark.parametrize("G", [16, 32, 64])
+def test_ffn_group_sizes_full_size(oracle, osc, G):
+    c = I.ffn_case(G, M=4096, calib_tokens=1536)
+    L = oracle.build_table(c.calib, G)
+    K_L = I.pad16(oracle.table_count(L))
+    _check_quant(oracle, osc, c.X, G, L, K_L, rows=I.sample_rows(4096, 256, seed=G))
+
+
+def test_w2_osc_and_fp8_full_size(oracle, osc):
+    c = I.w2_case(M=4096)
+    L = oracle.build_table(c.calib, 32)
+    K_L = I.pad16(oracle.table_count(L))
+    rows = I.sample_rows(4096, 128, seed=4)
+    _check_quant(oracle, osc, c.X, 32, L, K_L, rows=rows)
+    QX8, SX, _ = osc.alloc_quantize_outputs(4096, 12288, 32, 0, fp8=True)
+    osc.osc_quantize_fp8(to_dev(c.X), QX8, SX)
+    torch.cuda.synchronize()
+    cref, eref = oracle.mx_quantize(c.X[rows], 32, oracle.FMT_E4M3)
+    assert np.array_equal(to_np(QX8)[rows], cref)
+    assert np.array_equal(unswizzle_scales(to_np(SX), 4096, 12288, 32)[rows], eref)
+
+
+def test_edge_cases(oracle, osc):
+    rng = np.random.default_rng(3)
+    # ragged M, all-zero rows, negative zeros, K_L larger than the entry count, j* = 0 and G-1
+    M, K, G = 130, 512, 32
+    x = rng.standard_normal((M, K)) * 3
+    x[5] = 0.0
+    x[6] = -0.0
+    X = I.bf16_bits(x)
+    L = np.full(K // G, -1, np.int8)
+    L[[0, 3, 15]] = [0, 31, 7]
+    _check_quant(oracle, osc, X, G, L, 48)
+    # all -1 table with K_L = 0, and no table at all
+    _check_quant(oracle, osc, X, G, np.full(K // G, -1, np.int8), 0)
+    _check_quant(oracle, osc, X, G, None, 0)
+    # M = 0 is a no-op
+    QX, SX, B = osc.alloc_quantize_outputs(0, K, G, 16)
+    osc.osc_quantize(torch.zeros((0, K), dtype=torch.int16, device="cuda"), G, to_dev(L), 16, QX, SX, B)
+
+
+def test_bad_table_is_reported_not_faulted(osc):
+    X = to_dev(I.bf16_bits(np.ones((4, 256))))
+    L = np.full(8, -1, np.int8)
+    L[2] = 40                                   # >= G
+    QX, SX, B = osc.quantize(X, 32, to_dev(L), 16)
+    torch.cuda.synchronize()
+    code, raw = osc.osc_status()
+    assert code == -6 and raw == 2
+    assert osc.osc_status() == (0, 0)           # cleared
+
+
+def test_argument_errors(osc):
+    X = torch.zeros((4, 256), dtype=torch.int16, device="cuda")
+    QX, SX, B = osc.alloc_quantize_outputs(4, 256, 32, 16)
+    with pytest.raises(osc.OSCError) as e:
+        osc.osc_quantize(X, 24, None, 0, QX, SX, None)
+    assert e.value.code == -3
+    Xb = torch.zeros((4, 200), dtype=torch.int16, device="cuda")
+    with pytest.raises(osc.OSCError) as e:
+        osc.osc_quantize(Xb, 32, None, 0, QX, SX, None)
+    assert e.value.code == -2
+
+
+def test_prepare_weight(oracle, osc):
+    c = I.qkv_case(1)
+    L = c.planted
+    K_L = I.pad16(oracle.table_count(L))
+    QW, SW, WL = osc.prepare_weight(to_dev(c.W), 32, to_dev(L), K_L)
+    torch.cuda.synchronize()
+    cw, ew, WLr = oracle.osc_prepare_weight(c.W, 32, L, K_L)
+    assert np.array_equal(unpack_e2m1(to_np(QW), 4096), cw)
+    assert np.array_equal(unswizzle_scales(to_np(SW), 6144, 4096, 32), ew)
+    assert np.array_equal(to_np(WL), WLr)
+
+
+@pytest.mark.parametrize("case,G,alpha,min_hits", [
+    ("qkv", 32, 5.0, 5), ("w2", 32, 5.0, 5), ("ffn", 16, 5.0, 5), ("ffn", 64, 5.0, 5),
+    ("qkv", 32, 3.0, 2), ("random", 32, 2.5, 3)])
+def test_build_table(oracle, osc, case, G, alpha, min_hits):
+    if case == "qkv":
+        X = I.qkv_case(1).calib
+    elif case == "w2":
+        X = I.w2_case(M=1).calib
+    elif case == "ffn":
+        X = I.ffn_case(G, M=1).calib
+    else:
+        X = I.bf16_bits(np.random.default_rng(9).standard_t(3, size=(700, 1024)))
+    S, K = X.shape
+    L = torch.empty(K // G, dtype=torch.int8, device="cuda")
+    osc.osc_build_table(to_dev(X), G, alpha, min_hits, L)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(L), oracle.build_table(X, G, alpha, min_hits))

@@ -1,0 +1,363 @@
+// The C ABI of libosc.so (declared in include/osc.h): argument checks, per-device state,
+// TMA descriptor encoding and kernel launches. No entry point allocates or frees memory.
+#include "osc.h"
+#include "osc_device.cuh"
+#include "osc_internal.h"
+
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+namespace {
+
+thread_local int t_last_cuda = 0;
+std::atomic<int> g_tile_n{0};
+
+__device__ int g_status_word;   // per-device error word written by the kernels
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  bool sm100 = false;
+  int sms = 0;
+  int* status = nullptr;
+};
+
+int fail_cuda(cudaError_t e) {
+  t_last_cuda = (int)e;
+  return OSC_ERR_CUDA;
+}
+
+// Per-device facts, looked up once per device with that device current.
+int device_state(DeviceState** out) {
+  static std::mutex mu;
+  static DeviceState states[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (dev < 0 || dev >= kMaxDevices) return OSC_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  DeviceState& s = states[dev];
+  if (!s.ready) {
+    int major = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return fail_cuda(e);
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return fail_cuda(e);
+    void* addr = nullptr;
+    if ((e = cudaGetSymbolAddress(&addr, g_status_word)) != cudaSuccess) return fail_cuda(e);
+    s.sm100 = (major == 10);
+    s.sms = sms;
+    s.status = static_cast<int*>(addr);
+    s.ready = true;
+  }
+  if (!s.sm100) return OSC_ERR_DEVICE;
+  *out = &s;
+  return OSC_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Tiled TMA descriptor over a row-major tensor; dims[0] is the contiguous dimension.
+int make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+             const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return fail_cuda(cudaErrorNotSupported);
+  uint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void*>(base), reinterpret_cast<const cuuint64_t*>(dims),
+                  reinterpret_cast<const cuuint64_t*>(strides), reinterpret_cast<const cuuint32_t*>(box),
+                  reinterpret_cast<const cuuint32_t*>(es), CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail_cuda(cudaErrorInvalidValue);
+  return OSC_OK;
+}
+
+inline bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool valid_g(int G) { return G == 16 || G == 32 || G == 64; }
+
+int launch_result(cudaError_t e) { return e == cudaSuccess ? OSC_OK : fail_cuda(e); }
+
+}  // namespace
+
+namespace {
+
+// Shared launch path of the dense, fallback and grouped products.
+int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const uint8_t* QW,
+             const uint8_t* SW, const uint16_t* WL, int M, int N, int K, int K_L, int E,
+             const int* mblock_expert, const int* kl, uint16_t* Y, float* Yf32, cudaStream_t stream) {
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != OSC_OK) return rc;
+  const bool fp8 = kind == osc::KIND_MXF8_B32;
+  const int V = kind == osc::KIND_MXF4_B16 ? 16 : 32;
+  const int m_tiles = (M + 127) / 128;
+  int bn = g_tile_n.load();
+  if (bn == 0) bn = (N >= 256 && (long long)m_tiles * ((N + 255) / 256) >= ds->sms) ? 256 : 128;
+
+  osc::GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const uint64_t kb = fp8 ? (uint64_t)K : (uint64_t)K / 2;       // operand bytes per row
+  {
+    uint64_t d[2] = {kb, (uint64_t)M}, st[1] = {kb};
+    uint32_t box[2] = {128, 128};
+    if ((rc = make_map(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, QX, d, st, box, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+  }
+  {
+    uint64_t d[3] = {kb, (uint64_t)N, (uint64_t)E}, st[2] = {kb, kb * (uint64_t)N};
+    uint32_t box[3] = {128, (uint32_t)bn, 1};
+    if ((rc = make_map(&maps.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, QW, d, st, box, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+  }
+  if (K_L > 0) {
+    uint64_t d[2] = {(uint64_t)K_L, (uint64_t)M}, st[1] = {(uint64_t)K_L * 2};
+    uint32_t box[2] = {64, 128};
+    if ((rc = make_map(&maps.ca, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, d, st, box, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+    uint64_t d3[3] = {(uint64_t)K_L, (uint64_t)N, (uint64_t)E}, st3[2] = {(uint64_t)K_L * 2, (uint64_t)K_L * 2 * N};
+    uint32_t box3[3] = {64, (uint32_t)bn, 1};
+    if ((rc = make_map(&maps.cb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, WL, d3, st3, box3, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+  }
+  {
+    uint64_t d[2] = {(uint64_t)N, (uint64_t)M}, st[1] = {(uint64_t)N * 2};
+    uint32_t box[2] = {64, 32};
+    if ((rc = make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, d, st, box, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+  }
+  osc::GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = M; p.N = N; p.K = K; p.K_L = K_L;
+  p.SFA = SX; p.SFB = SW;
+  p.nslot4 = K / V / 4;
+  p.m_tiles = m_tiles;
+  p.n_tiles = (N + bn - 1) / bn;
+  p.Yf32 = Yf32;
+  p.status = ds->status;
+  p.num_groups = mblock_expert ? E : 0;
+  p.mblock_expert = mblock_expert;
+  p.group_kl = kl;
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int grid = tiles < ds->sms ? tiles : ds->sms;
+  return launch_result(osc::launch_gemm(kind, bn, maps, p, grid, stream));
+}
+
+int check_linear_common(const void* QX, const void* SX, const void* QW, const void* SW, int M, int N, int K,
+                        uint16_t* Y, float* Yf32) {
+  if (!QX || !SX || !QW || !SW || !Y || M < 0 || N <= 0 || K <= 0) return OSC_ERR_ARG;
+  if (!a16(QX) || !a16(SX) || !a16(QW) || !a16(SW) || !a16(Y) || (Yf32 && !a16(Yf32))) return OSC_ERR_ALIGN;
+  if (K % 256 != 0 || N % 16 != 0) return OSC_ERR_ALIGN;
+  return OSC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* osc_version(void) { return "osc-b200 0.1 (sm_100a)"; }
+
+const char* osc_error_string(int code) {
+  switch (code) {
+    case OSC_OK: return "ok";
+    case OSC_ERR_ARG: return "invalid argument (null pointer or unsupported size)";
+    case OSC_ERR_ALIGN: return "alignment or divisibility requirement not met";
+    case OSC_ERR_G: return "group size must be 16, 32 or 64";
+    case OSC_ERR_CUDA: return "CUDA call failed (see osc_last_cuda_error)";
+    case OSC_ERR_TIMEOUT: return "a kernel wait ran out of time";
+    case OSC_ERR_TABLE: return "table entry out of range or more entries than K_L";
+    case OSC_ERR_DEVICE: return "current device is not an sm_100 GPU";
+    default: return "unknown error";
+  }
+}
+
+int osc_last_cuda_error(void) { return t_last_cuda; }
+
+size_t osc_scale_bytes(int rows, int K, int G) {
+  if (rows < 0 || K <= 0) return 0;
+  int V;
+  if (G == 0) V = 32;
+  else if (valid_g(G)) V = (G == 16) ? 16 : 32;
+  else return 0;
+  if (K % (4 * V) != 0) return 0;
+  return (size_t)((rows + 127) / 128) * (size_t)(K / V / 4) * 512u;
+}
+
+int osc_table_kl(const int8_t* L_host, int Kg) {
+  if (!L_host || Kg < 0) return OSC_ERR_ARG;
+  int c = 0;
+  for (int k = 0; k < Kg; ++k) c += (L_host[k] >= 0);
+  return (c + 15) / 16 * 16;
+}
+
+int osc_set_tile_n(int bn) {
+  if (bn != 0 && bn != 128 && bn != 256) return OSC_ERR_ARG;
+  return g_tile_n.exchange(bn);
+}
+
+int osc_build_table(const uint16_t* Xcal, int S, int K, int G, float alpha, int min_hits, int8_t* L,
+                    osc_stream_t stream) {
+  if (!valid_g(G)) return OSC_ERR_G;
+  if (!Xcal || !L || S < 0 || K <= 0 || K % G != 0) return OSC_ERR_ARG;
+  if (!a16(Xcal)) return OSC_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != OSC_OK) return rc;
+  osc::TableParams p{Xcal, S, K, G, alpha, min_hits, L};
+  return launch_result(osc::launch_build_table(p, ds->sms, (cudaStream_t)stream));
+}
+
+int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int K_L, uint8_t* QX, uint8_t* SX,
+                 uint16_t* B, osc_stream_t stream) {
+  if (!valid_g(G)) return OSC_ERR_G;
+  if (!X || !QX || !SX || M < 0 || K <= 0 || K_L < 0) return OSC_ERR_ARG;
+  if (L == nullptr && K_L != 0) return OSC_ERR_ARG;
+  if (L != nullptr && K_L > 0 && !B) return OSC_ERR_ARG;
+  if (K_L > 32767) return OSC_ERR_ARG;
+  if (!a16(X) || !a16(QX) || !a16(SX) || (B && !a16(B))) return OSC_ERR_ALIGN;
+  if (K % 256 != 0 || K_L % 16 != 0) return OSC_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != OSC_OK) return rc;
+  if (M == 0) return OSC_OK;
+  osc::QuantParams p{X, M, K, G, K / G, L, K_L, QX, SX, B, ds->status};
+  return launch_result(osc::launch_quantize(p, false, ds->sms, (cudaStream_t)stream));
+}
+
+int osc_prepare_weight(const uint16_t* W, int N, int K, int G, const int8_t* L, int K_L, uint8_t* QW, uint8_t* SW,
+                       uint16_t* WL, osc_stream_t stream) {
+  if (!valid_g(G)) return OSC_ERR_G;
+  if (!W || !QW || !SW || N < 0 || K <= 0 || K_L < 0) return OSC_ERR_ARG;
+  if (K_L > 0 && (!L || !WL)) return OSC_ERR_ARG;
+  if (!a16(W) || !a16(QW) || !a16(SW) || (WL && !a16(WL))) return OSC_ERR_ALIGN;
+  if (K % 256 != 0 || K_L % 16 != 0) return OSC_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != OSC_OK) return rc;
+  if (N == 0) return OSC_OK;
+  osc::QuantParams p{W, N, K, G, K / G, nullptr, 0, QW, SW, nullptr, ds->status};
+  cudaError_t e = osc::launch_quantize(p, false, ds->sms, (cudaStream_t)stream);
+  if (e != cudaSuccess) return fail_cuda(e);
+  return launch_result(osc::launch_gather_wl(W, N, K, G, L, K_L, WL, ds->status, ds->sms, (cudaStream_t)stream));
+}
+
+int osc_linear(const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const uint8_t* QW, const uint8_t* SW,
+               const uint16_t* WL, int M, int N, int K, int G, int K_L, uint16_t* Y, float* Yf32,
+               osc_stream_t stream) {
+  if (!valid_g(G)) return OSC_ERR_G;
+  int rc = check_linear_common(QX, SX, QW, SW, M, N, K, Y, Yf32);
+  if (rc != OSC_OK) return rc;
+  if (K_L < 0 || K_L % 16 != 0) return K_L < 0 ? OSC_ERR_ARG : OSC_ERR_ALIGN;
+  if (K_L > 0 && (!B || !WL)) return OSC_ERR_ARG;
+  if (K_L > 0 && (!a16(B) || !a16(WL))) return OSC_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(&ds)) != OSC_OK) return rc;
+  if (M == 0) return OSC_OK;
+  const int kind = G == 16 ? osc::KIND_MXF4_B16 : osc::KIND_MXF4_B32;
+  return run_gemm(kind, QX, SX, B, QW, SW, WL, M, N, K, K_L, 1, nullptr, nullptr, Y, Yf32, (cudaStream_t)stream);
+}
+
+int osc_quantize_fp8(const uint16_t* X, int M, int K, uint8_t* QX8, uint8_t* SX, osc_stream_t stream) {
+  if (!X || !QX8 || !SX || M < 0 || K <= 0) return OSC_ERR_ARG;
+  if (!a16(X) || !a16(QX8) || !a16(SX)) return OSC_ERR_ALIGN;
+  if (K % 256 != 0) return OSC_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != OSC_OK) return rc;
+  if (M == 0) return OSC_OK;
+  osc::QuantParams p{X, M, K, 32, K / 32, nullptr, 0, QX8, SX, nullptr, ds->status};
+  return launch_result(osc::launch_quantize(p, true, ds->sms, (cudaStream_t)stream));
+}
+
+int osc_linear_fp8_fallback(const uint8_t* QX8, const uint8_t* SX, const uint8_t* QW8, const uint8_t* SW, int M,
+                            int N, int K, uint16_t* Y, float* Yf32, osc_stream_t stream) {
+  int rc = check_linear_common(QX8, SX, QW8, SW, M, N, K, Y, Yf32);
+  if (rc != OSC_OK) return rc;
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(&ds)) != OSC_OK) return rc;
+  if (M == 0) return OSC_OK;
+  return run_gemm(osc::KIND_MXF8_B32, QX8, SX, nullptr, QW8, SW, nullptr, M, N, K, 0, 1, nullptr, nullptr, Y, Yf32,
+                  (cudaStream_t)stream);
+}
+
+int osc_grouped_plan(const int* counts, int E, int* off, int* poff, int* mblock_expert, int mblock_capacity) {
+  if (!counts || !off || !poff || E <= 0 || mblock_capacity < 0) return OSC_ERR_ARG;
+  long long o = 0, po = 0;
+  for (int e = 0; e < E; ++e) {
+    if (counts[e] < 0) return OSC_ERR_ARG;
+    off[e] = (int)o;
+    poff[e] = (int)po;
+    o += counts[e];
+    po += (counts[e] + 127) / 128 * 128;
+    if (po > 0x7FFFFF80LL) return OSC_ERR_ARG;
+  }
+  off[E] = (int)o;
+  poff[E] = (int)po;
+  if (mblock_expert) {
+    if (po / 128 > mblock_capacity) return OSC_ERR_ARG;
+    for (int e = 0; e < E; ++e)
+      for (int b = poff[e] / 128; b < poff[e + 1] / 128; ++b) mblock_expert[b] = e;
+  }
+  return (int)po;
+}
+
+int osc_quantize_grouped(const uint16_t* X, int E, const int* off, const int* poff, const int* mblock_expert, int Mp,
+                         int K, int G, const int8_t* L, int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B,
+                         osc_stream_t stream) {
+  if (!valid_g(G)) return OSC_ERR_G;
+  if (!X || !off || !poff || !mblock_expert || !L || !QX || !SX || E <= 0 || Mp < 0 || K <= 0 || K_L < 0)
+    return OSC_ERR_ARG;
+  if (K_L > 0 && !B) return OSC_ERR_ARG;
+  if (K_L > 32767) return OSC_ERR_ARG;
+  if (!a16(X) || !a16(QX) || !a16(SX) || (B && !a16(B))) return OSC_ERR_ALIGN;
+  if (K % 256 != 0 || K_L % 16 != 0 || Mp % 128 != 0) return OSC_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != OSC_OK) return rc;
+  if (Mp == 0) return OSC_OK;
+  osc::GroupedQuantParams p{X, off, poff, mblock_expert, E, Mp, K, G, K / G, L, K_L, QX, SX, B, ds->status};
+  return launch_result(osc::launch_quantize_grouped(p, ds->sms, (cudaStream_t)stream));
+}
+
+int osc_linear_grouped(const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const uint8_t* QW, const uint8_t* SW,
+                       const uint16_t* WL, const int* mblock_expert, const int* kl, int E, int Mp, int N, int K,
+                       int G, int K_L, uint16_t* Y, float* Yf32, osc_stream_t stream) {
+  if (!valid_g(G)) return OSC_ERR_G;
+  int rc = check_linear_common(QX, SX, QW, SW, Mp, N, K, Y, Yf32);
+  if (rc != OSC_OK) return rc;
+  if (!mblock_expert || E <= 0) return OSC_ERR_ARG;
+  if (Mp % 128 != 0) return OSC_ERR_ALIGN;
+  if (K_L < 0 || K_L % 16 != 0) return K_L < 0 ? OSC_ERR_ARG : OSC_ERR_ALIGN;
+  if (K_L > 0 && (!B || !WL)) return OSC_ERR_ARG;
+  if (K_L > 0 && (!a16(B) || !a16(WL))) return OSC_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(&ds)) != OSC_OK) return rc;
+  if (Mp == 0) return OSC_OK;
+  const int kind = G == 16 ? osc::KIND_MXF4_B16 : osc::KIND_MXF4_B32;
+  return run_gemm(kind, QX, SX, B, QW, SW, WL, Mp, N, K, K_L, E, mblock_expert, K_L > 0 ? kl : nullptr, Y, Yf32,
+                  (cudaStream_t)stream);
+}
+
+int osc_status(int* raw, osc_stream_t stream) {
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != OSC_OK) return rc;
+  int v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ds->status, sizeof(int), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ds->status, 0, sizeof(int), (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (raw) *raw = v;
+  if (v == osc::DEV_TIMEOUT) return OSC_ERR_TIMEOUT;
+  if (v == osc::DEV_BAD_TABLE) return OSC_ERR_TABLE;
+  return OSC_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,73 @@
+// Internal declarations shared by the .cu files of libosc.so (not part of the C ABI).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <algorithm>
+
+namespace osc {
+
+struct QuantParams {
+  const uint16_t* X;   // M x K bf16
+  int M, K, G, Kg;
+  const int8_t* L;     // Kg entries (device) or nullptr for no table
+  int K_L;
+  uint8_t* Q;          // packed codes
+  uint8_t* S;          // scales in the MMA layout
+  uint16_t* B;         // M x K_L bf16 (table only)
+  int* status;
+};
+
+cudaError_t launch_quantize(const QuantParams& p, bool fp8, int num_sms, cudaStream_t s);
+
+struct GroupedQuantParams {
+  const uint16_t* X;          // off[E] x K bf16, expert-sorted
+  const int* off;             // E+1 (device)
+  const int* poff;            // E+1 (device)
+  const int* mblock_expert;   // Mp/128 (device)
+  int E, Mp, K, G, Kg;
+  const int8_t* L;            // E x Kg (device)
+  int K_L;
+  uint8_t* Q;
+  uint8_t* S;
+  uint16_t* B;
+  int* status;
+};
+cudaError_t launch_quantize_grouped(const GroupedQuantParams& p, int num_sms, cudaStream_t s);
+cudaError_t launch_gather_wl(const uint16_t* W, int N, int K, int G, const int8_t* L, int K_L, uint16_t* WL,
+                             int* status, int num_sms, cudaStream_t s);
+
+// GEMM operand kinds
+enum GemmKind : int { KIND_MXF4_B32 = 0, KIND_MXF4_B16 = 1, KIND_MXF8_B32 = 2 };
+
+struct GemmParams {
+  int M, N, K, K_L;
+  const uint8_t* SFA;    // activation scales (MMA layout)
+  const uint8_t* SFB;    // weight scales (MMA layout)
+  int nslot4;            // 512-byte scale atoms per 128-row block = K / V / 4
+  int m_tiles, n_tiles;
+  float* Yf32;           // optional fp32 copy of the output (tests)
+  int* status;
+  // grouped (MoE) mode when num_groups > 0: each 128-row block of the (padded) row space
+  // belongs to one expert, whose weights are slice e of the 3-D weight maps
+  int num_groups;
+  const int* mblock_expert;      // m_tiles entries (device)
+  const int* group_kl;           // per-expert compensation width (device) or nullptr = K_L
+};
+
+struct GemmMaps {
+  CUtensorMap a, b, ca, cb, y;
+};
+
+cudaError_t launch_gemm(int kind, int bn, const GemmMaps& maps, const GemmParams& p, int grid, cudaStream_t s);
+
+struct TableParams {
+  const uint16_t* X;   // S x K bf16
+  int S, K, G;
+  float alpha;
+  int min_hits;
+  int8_t* L;
+};
+cudaError_t launch_build_table(const TableParams& p, int num_sms, cudaStream_t s);
+
+}  // namespace osc

@@ -1,0 +1,66 @@
+// Offline suppression-table build on the GPU: Algorithm 1 of the OSC page
+// ("W4A4量化技术：OSC框架如何实现高效LLM部署", coreui.cn/article/2607942.html, §3.1), for one
+// (position, layer) given its S x K calibration activations.
+//
+// find_consistent_outlier is left undefined by the page; the rule used here: for each
+// calibration token the group's outlier event is the channel with the largest |x| (lowest
+// channel on ties), counted only when G * |x_max| >= alpha * sum_j |x_j| and |x_max| > 0; the
+// sum runs in fp32 in ascending channel order and the comparison in fp64, so the decision is
+// reproducible bit for bit. The channel with the most events wins (lowest on ties) when it
+// has at least min_hits events; otherwise the entry is -1. Counting is integer, so the table
+// does not depend on the order in which tokens are visited.
+//
+// One CTA per channel group; threads stride over tokens; a shared histogram of G counters.
+#include "osc_device.cuh"
+#include "osc_internal.h"
+
+namespace osc {
+
+template <int G>
+__global__ void __launch_bounds__(256) build_table_kernel(TableParams p) {
+  __shared__ int hist[G];
+  const int k = blockIdx.x;
+  for (int j = threadIdx.x; j < G; j += blockDim.x) hist[j] = 0;
+  __syncthreads();
+  for (int t = threadIdx.x; t < p.S; t += blockDim.x) {
+    const uint4* src = reinterpret_cast<const uint4*>(p.X + (size_t)t * p.K + (size_t)k * G);
+    float s = 0.0f;
+    uint32_t best = 0;
+    int jb = 0;
+#pragma unroll
+    for (int v = 0; v < G / 8; ++v) {
+      const uint4 r = __ldg(src + v);
+      const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        const uint32_t mag = (h & 1) ? (w[h >> 1] >> 16) & 0x7FFFu : w[h >> 1] & 0x7FFFu;
+        s += __uint_as_float(mag << 16);
+        if (mag > best) { best = mag; jb = v * 8 + h; }
+      }
+    }
+    const double amax = (double)__uint_as_float(best << 16);
+    if (best != 0u && (double)G * amax >= (double)p.alpha * (double)s) atomicAdd(&hist[jb], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int js = 0;
+    for (int j = 1; j < G; ++j)
+      if (hist[j] > hist[js]) js = j;
+    p.L[k] = (hist[js] > 0 && hist[js] >= p.min_hits) ? (int8_t)js : (int8_t)-1;
+  }
+}
+
+cudaError_t launch_build_table(const TableParams& p, int num_sms, cudaStream_t s) {
+  (void)num_sms;
+  const int Kg = p.K / p.G;
+  if (Kg == 0) return cudaSuccess;
+  switch (p.G) {
+    case 16: build_table_kernel<16><<<Kg, 256, 0, s>>>(p); break;
+    case 32: build_table_kernel<32><<<Kg, 256, 0, s>>>(p); break;
+    case 64: build_table_kernel<64><<<Kg, 256, 0, s>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace osc

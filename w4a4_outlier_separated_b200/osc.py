@@ -1,0 +1,212 @@
+"""Thin Python binding of libosc.so (the C ABI declared in include/osc.h).
+
+Argument marshalling only: every step of the OSC path runs in the library's sm_100a kernels.
+Tensors are PyTorch CUDA tensors; the current torch stream is used unless one is given.
+The library must exist (``python -m w4a4_outlier_separated_b200.build``); there is no fallback.
+
+Names follow the C ABI; ``alloc_*`` helpers allocate the output tensors of a call with torch.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libosc.so")
+
+OSC_OK = 0
+ERRORS = {-1: "OSC_ERR_ARG", -2: "OSC_ERR_ALIGN", -3: "OSC_ERR_G", -4: "OSC_ERR_CUDA",
+          -5: "OSC_ERR_TIMEOUT", -6: "OSC_ERR_TABLE", -7: "OSC_ERR_DEVICE"}
+
+
+class OSCError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str, cuda_err: int = 0):
+        super().__init__(f"{fn}: {ERRORS.get(code, code)} ({msg})" + (f", cudaError {cuda_err}" if cuda_err else ""))
+        self.code = code
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libosc.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"libosc.so not found at {_LIB_PATH}: build it with "
+                              "`python -m w4a4_outlier_separated_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        sig = {
+            "osc_version": ([], ctypes.c_char_p),
+            "osc_error_string": ([i32], ctypes.c_char_p),
+            "osc_last_cuda_error": ([], i32),
+            "osc_scale_bytes": ([i32, i32, i32], ctypes.c_size_t),
+            "osc_table_kl": ([P, i32], i32),
+            "osc_build_table": ([P, i32, i32, i32, f32, i32, P, P], i32),
+            "osc_quantize": ([P, i32, i32, i32, P, i32, P, P, P, P], i32),
+            "osc_prepare_weight": ([P, i32, i32, i32, P, i32, P, P, P, P], i32),
+            "osc_linear": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P], i32),
+            "osc_quantize_fp8": ([P, i32, i32, P, P, P], i32),
+            "osc_linear_fp8_fallback": ([P, P, P, P, i32, i32, i32, P, P, P], i32),
+            "osc_grouped_plan": ([P, i32, P, P, P, i32], i32),
+            "osc_quantize_grouped": ([P, i32, P, P, P, i32, i32, i32, P, i32, P, P, P, P], i32),
+            "osc_linear_grouped": ([P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P], i32),
+            "osc_status": ([P, P], i32),
+            "osc_set_tile_n": ([i32], i32),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(name: str, rc: int):
+    if rc != OSC_OK:
+        L = lib()
+        raise OSCError(name, rc, L.osc_error_string(rc).decode(), L.osc_last_cuda_error())
+
+
+# ---- sizes --------------------------------------------------------------------------------
+
+def osc_scale_bytes(rows: int, K: int, G: int) -> int:
+    return int(lib().osc_scale_bytes(rows, K, G))
+
+
+def osc_table_kl(L) -> int:
+    """K_L for a table (numpy int8 array or CPU tensor)."""
+    t = torch.as_tensor(L, dtype=torch.int8).contiguous().cpu()
+    rc = lib().osc_table_kl(ctypes.c_void_p(t.data_ptr()), t.numel())
+    if rc < 0:
+        _check("osc_table_kl", rc)
+    return int(rc)
+
+
+def osc_set_tile_n(bn: int) -> int:
+    return int(lib().osc_set_tile_n(bn))
+
+
+# ---- raw calls (outputs given) -----------------------------------------------------------------
+
+def osc_build_table(Xcal, G: int, alpha: float, min_hits: int, L, stream=None):
+    S, K = Xcal.shape
+    _check("osc_build_table", lib().osc_build_table(_ptr(Xcal), S, K, G, alpha, min_hits, _ptr(L), _stream(stream)))
+
+
+def osc_quantize(X, G: int, L, K_L: int, QX, SX, B, stream=None):
+    M, K = X.shape
+    _check("osc_quantize", lib().osc_quantize(_ptr(X), M, K, G, _ptr(L), K_L, _ptr(QX), _ptr(SX),
+                                              _ptr(B) if K_L else None, _stream(stream)))
+
+
+def osc_prepare_weight(W, G: int, L, K_L: int, QW, SW, WL, stream=None):
+    N, K = W.shape
+    _check("osc_prepare_weight", lib().osc_prepare_weight(_ptr(W), N, K, G, _ptr(L), K_L, _ptr(QW), _ptr(SW),
+                                                          _ptr(WL) if K_L else None, _stream(stream)))
+
+
+def osc_linear(QX, SX, B, QW, SW, WL, M: int, N: int, K: int, G: int, K_L: int, Y, Yf32=None, stream=None):
+    _check("osc_linear", lib().osc_linear(_ptr(QX), _ptr(SX), _ptr(B) if K_L else None, _ptr(QW), _ptr(SW),
+                                          _ptr(WL) if K_L else None, M, N, K, G, K_L, _ptr(Y), _ptr(Yf32),
+                                          _stream(stream)))
+
+
+def osc_quantize_fp8(X, QX8, SX, stream=None):
+    M, K = X.shape
+    _check("osc_quantize_fp8", lib().osc_quantize_fp8(_ptr(X), M, K, _ptr(QX8), _ptr(SX), _stream(stream)))
+
+
+def osc_linear_fp8_fallback(QX8, SX, QW8, SW, M: int, N: int, K: int, Y, Yf32=None, stream=None):
+    _check("osc_linear_fp8_fallback", lib().osc_linear_fp8_fallback(_ptr(QX8), _ptr(SX), _ptr(QW8), _ptr(SW), M, N, K,
+                                                                    _ptr(Y), _ptr(Yf32), _stream(stream)))
+
+
+def osc_grouped_plan(counts):
+    """Per-expert token counts -> (off, poff, mblock_expert) as int32 CPU tensors."""
+    c = torch.as_tensor(counts, dtype=torch.int32).contiguous().cpu()
+    E = c.numel()
+    off = torch.empty(E + 1, dtype=torch.int32)
+    poff = torch.empty(E + 1, dtype=torch.int32)
+    mp = lib().osc_grouped_plan(ctypes.c_void_p(c.data_ptr()), E, ctypes.c_void_p(off.data_ptr()),
+                                ctypes.c_void_p(poff.data_ptr()), None, 0)
+    if mp < 0:
+        _check("osc_grouped_plan", mp)
+    mbe = torch.empty(max(mp // 128, 1), dtype=torch.int32)
+    rc = lib().osc_grouped_plan(ctypes.c_void_p(c.data_ptr()), E, ctypes.c_void_p(off.data_ptr()),
+                                ctypes.c_void_p(poff.data_ptr()), ctypes.c_void_p(mbe.data_ptr()), mbe.numel())
+    if rc < 0:
+        _check("osc_grouped_plan", rc)
+    return off, poff, mbe[: mp // 128]
+
+
+def osc_quantize_grouped(X, E: int, off, poff, mblock_expert, Mp: int, G: int, L, K_L: int, QX, SX, B, stream=None):
+    K = X.shape[1]
+    _check("osc_quantize_grouped", lib().osc_quantize_grouped(_ptr(X), E, _ptr(off), _ptr(poff), _ptr(mblock_expert),
+                                                              Mp, K, G, _ptr(L), K_L, _ptr(QX), _ptr(SX),
+                                                              _ptr(B) if K_L else None, _stream(stream)))
+
+
+def osc_linear_grouped(QX, SX, B, QW, SW, WL, mblock_expert, kl, E: int, Mp: int, N: int, K: int, G: int, K_L: int,
+                       Y, Yf32=None, stream=None):
+    _check("osc_linear_grouped", lib().osc_linear_grouped(_ptr(QX), _ptr(SX), _ptr(B) if K_L else None, _ptr(QW),
+                                                          _ptr(SW), _ptr(WL) if K_L else None, _ptr(mblock_expert),
+                                                          _ptr(kl), E, Mp, N, K, G, K_L, _ptr(Y), _ptr(Yf32),
+                                                          _stream(stream)))
+
+
+def osc_status(stream=None):
+    """(code, raw device word); reads and clears the device status word (synchronizes)."""
+    raw = ctypes.c_int(0)
+    rc = lib().osc_status(ctypes.byref(raw), _stream(stream))
+    return int(rc), int(raw.value)
+
+
+# ---- allocation helpers ------------------------------------------------------------------------
+
+def alloc_quantize_outputs(M: int, K: int, G: int, K_L: int, device="cuda", fp8: bool = False):
+    dev = torch.device(device)
+    QX = torch.empty((M, K if fp8 else K // 2), dtype=torch.uint8, device=dev)
+    SX = torch.empty(osc_scale_bytes(M, K, 0 if fp8 else G), dtype=torch.uint8, device=dev)
+    B = torch.empty((M, K_L), dtype=torch.int16, device=dev) if K_L else None
+    return QX, SX, B
+
+
+def quantize(X, G: int, L=None, K_L: int = 0, stream=None):
+    """X (bf16 or int16 bits, M x K) -> (QX, SX, B)."""
+    M, K = X.shape
+    QX, SX, B = alloc_quantize_outputs(M, K, G, K_L, X.device)
+    osc_quantize(X, G, L, K_L, QX, SX, B, stream)
+    return QX, SX, B
+
+
+def prepare_weight(W, G: int, L=None, K_L: int = 0, stream=None):
+    N, K = W.shape
+    QW, SW, _ = alloc_quantize_outputs(N, K, G, 0, W.device)
+    WL = torch.empty((N, K_L), dtype=torch.int16, device=W.device) if K_L else None
+    osc_prepare_weight(W, G, L, K_L, QW, SW, WL, stream)
+    return QW, SW, WL
+
+
+def linear(QX, SX, B, QW, SW, WL, M: int, N: int, K: int, G: int, K_L: int, want_f32: bool = False, stream=None):
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=QX.device)
+    Yf = torch.empty((M, N), dtype=torch.float32, device=QX.device) if want_f32 else None
+    osc_linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y, Yf, stream)
+    return Y, Yf
