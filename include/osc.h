@@ -20,6 +20,7 @@
  *   - All pointers must be 16-byte aligned (cudaMalloc / PyTorch allocations are).
  *   - Inputs must be finite (no NaN / Inf).
  *   - Return value: OSC_OK (0) or a negative OSC_ERR_* code; nothing is launched on error.
+ *     A call with zero rows (M = 0) does nothing and returns OSC_OK; its pointers may be NULL.
  *     Errors found by a kernel while it runs (a table entry >= G, more entries than K_L,
  *     a bounded wait that ran out) are recorded in a per-device status word that
  *     osc_status() reads and clears.

@@ -44,6 +44,9 @@ def to_dev(a, dtype=None):
 
 def to_np(t, dtype=None):
     import numpy as np
+    import torch
+    if t.dtype == torch.bfloat16:
+        t = t.view(torch.int16)
     a = t.detach().cpu().numpy()
     if a.dtype == np.int16:
         a = a.view(np.uint16)

@@ -113,7 +113,7 @@ def test_ragged_shapes_and_compensation_width(oracle, osc, bn):
     """M not a multiple of 128, N not a multiple of the tile, two compensation stages with a
     partial second one (K_L = 80), entries at channel 0 and G-1."""
     rng = np.random.default_rng(21)
-    M, K, N, G = 130, 1024, 400, 32
+    M, K, N, G = 130, 2304, 400, 32
     x = rng.standard_normal((M, K))
     L = np.full(K // G, -1, np.int8)
     idx = rng.permutation(K // G)[:70]

@@ -216,6 +216,7 @@ int osc_build_table(const uint16_t* Xcal, int S, int K, int G, float alpha, int 
 int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int K_L, uint8_t* QX, uint8_t* SX,
                  uint16_t* B, osc_stream_t stream) {
   if (!valid_g(G)) return OSC_ERR_G;
+  if (M == 0 && K > 0 && K_L >= 0) return OSC_OK;          // nothing to read or write
   if (!X || !QX || !SX || M < 0 || K <= 0 || K_L < 0) return OSC_ERR_ARG;
   if (L == nullptr && K_L != 0) return OSC_ERR_ARG;
   if (L != nullptr && K_L > 0 && !B) return OSC_ERR_ARG;
@@ -251,6 +252,7 @@ int osc_linear(const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const ui
                const uint16_t* WL, int M, int N, int K, int G, int K_L, uint16_t* Y, float* Yf32,
                osc_stream_t stream) {
   if (!valid_g(G)) return OSC_ERR_G;
+  if (M == 0 && N > 0 && K > 0 && K_L >= 0) return OSC_OK;  // nothing to read or write
   int rc = check_linear_common(QX, SX, QW, SW, M, N, K, Y, Yf32);
   if (rc != OSC_OK) return rc;
   if (K_L < 0 || K_L % 16 != 0) return K_L < 0 ? OSC_ERR_ARG : OSC_ERR_ALIGN;
@@ -258,12 +260,12 @@ int osc_linear(const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const ui
   if (K_L > 0 && (!a16(B) || !a16(WL))) return OSC_ERR_ALIGN;
   DeviceState* ds = nullptr;
   if ((rc = device_state(&ds)) != OSC_OK) return rc;
-  if (M == 0) return OSC_OK;
   const int kind = G == 16 ? osc::KIND_MXF4_B16 : osc::KIND_MXF4_B32;
   return run_gemm(kind, QX, SX, B, QW, SW, WL, M, N, K, K_L, 1, nullptr, nullptr, Y, Yf32, (cudaStream_t)stream);
 }
 
 int osc_quantize_fp8(const uint16_t* X, int M, int K, uint8_t* QX8, uint8_t* SX, osc_stream_t stream) {
+  if (M == 0 && K > 0) return OSC_OK;                       // nothing to read or write
   if (!X || !QX8 || !SX || M < 0 || K <= 0) return OSC_ERR_ARG;
   if (!a16(X) || !a16(QX8) || !a16(SX)) return OSC_ERR_ALIGN;
   if (K % 256 != 0) return OSC_ERR_ALIGN;
@@ -277,6 +279,7 @@ int osc_quantize_fp8(const uint16_t* X, int M, int K, uint8_t* QX8, uint8_t* SX,
 
 int osc_linear_fp8_fallback(const uint8_t* QX8, const uint8_t* SX, const uint8_t* QW8, const uint8_t* SW, int M,
                             int N, int K, uint16_t* Y, float* Yf32, osc_stream_t stream) {
+  if (M == 0 && N > 0 && K > 0) return OSC_OK;              // nothing to read or write
   int rc = check_linear_common(QX8, SX, QW8, SW, M, N, K, Y, Yf32);
   if (rc != OSC_OK) return rc;
   DeviceState* ds = nullptr;
