@@ -170,6 +170,11 @@ OSC_API int osc_status(int* raw, osc_stream_t stream);
  * calls made afterwards from any thread. Returns the previous value, or OSC_ERR_ARG. */
 OSC_API int osc_set_tile_n(int bn);
 
+/* CTA grouping of the tensor-core kernels: -1 = automatic (default), 1 = one CTA per
+ * 128-row tile, 2 = a 2-CTA cluster per 256-row tile (tile width 256; dense calls only).
+ * Returns the previous value, or OSC_ERR_ARG. */
+OSC_API int osc_set_cta_pair(int mode);
+
 #ifdef __cplusplus
 }
 #endif

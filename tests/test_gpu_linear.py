@@ -25,12 +25,12 @@ def _compare(Y_bf16, Y_f32, Yref):
     assert np.all(np.abs(yb - Yref) <= REL * ymax + bf16_ulp(Yref))
 
 
-def _run_osc(oracle, osc, X, W, G, L, rows=None, bn=0):
+def _run_osc(oracle, osc, X, W, G, L, rows=None, bn=0, pair=-1):
     M, K = X.shape
     N = W.shape[0]
     K_L = I.pad16(oracle.table_count(L)) if L is not None else 0
     Ld = to_dev(L) if L is not None else None
-    prev = osc.osc_set_tile_n(bn)
+    prev, prev_pair = osc.osc_set_tile_n(bn), osc.osc_set_cta_pair(pair)
     try:
         QW, SW, WL = osc.prepare_weight(to_dev(W), G, Ld, K_L)
         QX, SX, B = osc.quantize(to_dev(X), G, Ld, K_L)
@@ -38,6 +38,7 @@ def _run_osc(oracle, osc, X, W, G, L, rows=None, bn=0):
         torch.cuda.synchronize()
     finally:
         osc.osc_set_tile_n(prev)
+        osc.osc_set_cta_pair(prev_pair)
     assert osc.osc_status() == (0, 0)
     Lo = L if L is not None else np.full(K // G, -1, np.int8)
     cw, ew, WLr = oracle.osc_prepare_weight(W, G, Lo, K_L)
@@ -61,12 +62,20 @@ def test_qkv(oracle, osc, M):
     _run_osc(oracle, osc, c.X, c.W, 32, L, rows=rows)
 
 
-def test_qkv_both_tile_widths(oracle, osc):
+def test_qkv_tile_shapes(oracle, osc):
+    """128- and 256-wide single-CTA tiles and the 2-CTA 256 x 256 pair tile."""
     c = I.qkv_case(2048)
     L = oracle.build_table(c.calib, 32)
     rows = I.sample_rows(2048, 12, seed=5)
-    for bn in (128, 256):
-        _run_osc(oracle, osc, c.X, c.W, 32, L, rows=rows, bn=bn)
+    for bn, pair in ((128, 1), (256, 1), (256, 2)):
+        _run_osc(oracle, osc, c.X, c.W, 32, L, rows=rows, bn=bn, pair=pair)
+
+
+@pytest.mark.parametrize("G", [16, 64])
+def test_cta_pair_group_sizes(oracle, osc, G):
+    c = I.ffn_case(G, M=512, calib_tokens=512)
+    L = oracle.build_table(c.calib, G)
+    _run_osc(oracle, osc, c.X, c.W[:1024], G, L, rows=I.sample_rows(512, 16, seed=G), bn=256, pair=2)
 
 
 @pytest.mark.parametrize("G", [16, 32, 64])
@@ -82,8 +91,9 @@ def test_w2_osc_full_size(oracle, osc):
     _run_osc(oracle, osc, c.X, c.W, 32, L, rows=I.sample_rows(4096, 12, seed=7))
 
 
-@pytest.mark.parametrize("shape", [(4096, 12288, 4096), (130, 512, 144), (1, 256, 16)])
-def test_fp8_fallback(oracle, osc, shape):
+@pytest.mark.parametrize("shape,pair", [((4096, 12288, 4096), -1), ((4096, 12288, 4096), 1), ((130, 512, 144), 1),
+                                        ((130, 512, 256), 2), ((1, 256, 16), -1)])
+def test_fp8_fallback(oracle, osc, shape, pair):
     M, K, N = shape
     if M == 4096:
         c = I.w2_case(M=4096)
@@ -101,15 +111,20 @@ def test_fp8_fallback(oracle, osc, shape):
     osc.osc_quantize_fp8(Wd, QW, SW)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     Yf = torch.empty((M, N), dtype=torch.float32, device="cuda")
-    osc.osc_linear_fp8_fallback(QX, SX, QW, SW, M, N, K, Y, Yf)
-    torch.cuda.synchronize()
+    prev, prev_bn = osc.osc_set_cta_pair(pair), osc.osc_set_tile_n(256 if pair == 2 else 0)
+    try:
+        osc.osc_linear_fp8_fallback(QX, SX, QW, SW, M, N, K, Y, Yf)
+        torch.cuda.synchronize()
+    finally:
+        osc.osc_set_cta_pair(prev)
+        osc.osc_set_tile_n(prev_bn)
     sel = np.arange(M) if rows is None else rows
     ref = oracle.fp8_forward(X[sel], W)["Y"]
     _compare(to_np(Y)[sel], to_np(Yf)[sel], ref)
 
 
-@pytest.mark.parametrize("bn", [128, 256])
-def test_ragged_shapes_and_compensation_width(oracle, osc, bn):
+@pytest.mark.parametrize("bn,pair", [(128, 1), (256, 1), (256, 2)])
+def test_ragged_shapes_and_compensation_width(oracle, osc, bn, pair):
     """M not a multiple of 128, N not a multiple of the tile, two compensation stages with a
     partial second one (K_L = 80), entries at channel 0 and G-1."""
     rng = np.random.default_rng(21)
@@ -124,7 +139,7 @@ def test_ragged_shapes_and_compensation_width(oracle, osc, bn):
             x[:, k * G + int(j)] = rng.choice([-1, 1], M) * rng.uniform(20, 80, M)
     X = I.bf16_bits(x)
     W = I.gen_weights(N, K, seed=3)
-    _run_osc(oracle, osc, X, W, G, L, bn=bn)
+    _run_osc(oracle, osc, X, W, G, L, bn=bn, pair=pair)
 
 
 def test_all_minus_one_table_is_mxfp4_direct(oracle, osc):

@@ -14,6 +14,7 @@ namespace {
 
 thread_local int t_last_cuda = 0;
 std::atomic<int> g_tile_n{0};
+std::atomic<int> g_pair{-1};   // -1 automatic, 1 single CTAs, 2 CTA pairs
 
 __device__ int g_status_word;   // per-device error word written by the kernels
 
@@ -102,13 +103,21 @@ int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
   if (rc != OSC_OK) return rc;
   const bool fp8 = kind == osc::KIND_MXF8_B32;
   const int V = kind == osc::KIND_MXF4_B16 ? 16 : 32;
-  const int m_tiles = (M + 127) / 128;
   int bn = g_tile_n.load();
-  if (bn == 0) bn = (N >= 256 && (long long)m_tiles * ((N + 255) / 256) >= ds->sms) ? 256 : 128;
+  int cg = g_pair.load();
+  const bool grouped = mblock_expert != nullptr;
+  if (bn == 0) bn = (N >= 256 && (long long)((M + 127) / 128) * ((N + 255) / 256) >= ds->sms) ? 256 : 128;
+  // the CTA pair needs 256-wide tiles, whole 256-row tiles of work and a per-128-row expert map
+  // it cannot honour, so grouped calls stay on single CTAs
+  if (cg < 0) cg = (bn == 256 && !grouped && (long long)((M + 255) / 256) * ((N + 255) / 256) >= ds->sms / 2) ? 2 : 1;
+  if (cg == 2 && (bn != 256 || grouped)) cg = 1;
+  const int m_tiles = (M + 128 * cg - 1) / (128 * cg);
 
   osc::GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   const uint64_t kb = fp8 ? (uint64_t)K : (uint64_t)K / 2;       // operand bytes per row
+  const int nslot4 = K / V / 4;
+  const int brows = bn / cg;
   {
     uint64_t d[2] = {kb, (uint64_t)M}, st[1] = {kb};
     uint32_t box[2] = {128, 128};
@@ -116,15 +125,26 @@ int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
   }
   {
     uint64_t d[3] = {kb, (uint64_t)N, (uint64_t)E}, st[2] = {kb, kb * (uint64_t)N};
-    uint32_t box[3] = {128, (uint32_t)bn, 1};
+    uint32_t box[3] = {128, (uint32_t)brows, 1};
     if ((rc = make_map(&maps.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, QW, d, st, box, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+  }
+  {
+    // scale buffers as (128 words of an atom) x (atoms along K) x (128-row blocks)
+    const uint64_t mblk = (uint64_t)((M + 127) / 128);
+    uint64_t d[3] = {128, (uint64_t)nslot4, mblk}, st[2] = {512, (uint64_t)nslot4 * 512};
+    uint32_t box[3] = {128, (uint32_t)(fp8 ? 1 : (V == 16 ? 4 : 2)), 1};
+    if ((rc = make_map(&maps.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, SX, d, st, box, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
+    const uint64_t nblk = (uint64_t)((N + 127) / 128) * (uint64_t)E;
+    uint64_t d2[3] = {128, (uint64_t)nslot4, nblk};
+    uint32_t box2[3] = {128, box[1], (uint32_t)(bn / 128)};
+    if ((rc = make_map(&maps.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, SW, d2, st, box2, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
   }
   if (K_L > 0) {
     uint64_t d[2] = {(uint64_t)K_L, (uint64_t)M}, st[1] = {(uint64_t)K_L * 2};
     uint32_t box[2] = {64, 128};
     if ((rc = make_map(&maps.ca, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, d, st, box, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
     uint64_t d3[3] = {(uint64_t)K_L, (uint64_t)N, (uint64_t)E}, st3[2] = {(uint64_t)K_L * 2, (uint64_t)K_L * 2 * N};
-    uint32_t box3[3] = {64, (uint32_t)bn, 1};
+    uint32_t box3[3] = {64, (uint32_t)brows, 1};
     if ((rc = make_map(&maps.cb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, WL, d3, st3, box3, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
   }
   {
@@ -136,7 +156,7 @@ int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
   std::memset(&p, 0, sizeof(p));
   p.M = M; p.N = N; p.K = K; p.K_L = K_L;
   p.SFA = SX; p.SFB = SW;
-  p.nslot4 = K / V / 4;
+  p.nslot4 = nslot4;
   p.m_tiles = m_tiles;
   p.n_tiles = (N + bn - 1) / bn;
   p.Yf32 = Yf32;
@@ -145,8 +165,9 @@ int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
   p.mblock_expert = mblock_expert;
   p.group_kl = kl;
   const int tiles = p.m_tiles * p.n_tiles;
-  const int grid = tiles < ds->sms ? tiles : ds->sms;
-  return launch_result(osc::launch_gemm(kind, bn, maps, p, grid, stream));
+  const int units = ds->sms / cg;
+  const int grid = (tiles < units ? tiles : units) * cg;
+  return launch_result(osc::launch_gemm(kind, bn, cg, maps, p, grid, stream));
 }
 
 int check_linear_common(const void* QX, const void* SX, const void* QW, const void* SW, int M, int N, int K,
@@ -199,6 +220,11 @@ int osc_table_kl(const int8_t* L_host, int Kg) {
 int osc_set_tile_n(int bn) {
   if (bn != 0 && bn != 128 && bn != 256) return OSC_ERR_ARG;
   return g_tile_n.exchange(bn);
+}
+
+int osc_set_cta_pair(int mode) {
+  if (mode != -1 && mode != 1 && mode != 2) return OSC_ERR_ARG;
+  return g_pair.exchange(mode);
 }
 
 int osc_build_table(const uint16_t* Xcal, int S, int K, int G, float alpha, int min_hits, int8_t* L,

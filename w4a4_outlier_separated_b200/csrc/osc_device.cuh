@@ -217,6 +217,103 @@ __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t n) {
 constexpr uint32_t FMT_MXF4_E2M1 = 1;   // E2M1 in the mxf4 / mxf4nvf4 kinds
 constexpr uint32_t FMT_F8_E4M3 = 0;     // E4M3 in the mxf8f6f4 kind
 
+// ---- clusters and the CTA pair (cta_group::2) ---------------------------------------------
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory offset in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on an mbarrier that may live in another CTA of the cluster.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(cluster_addr) : "memory");
+}
+// TMA loads of the pair form: the data lands in this CTA's shared memory, the transaction
+// bytes are counted on `bar`, which may be the leader CTA's barrier.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* m, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      :: "r"(dst), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* m, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+      :: "r"(dst), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(bar) : "memory");
+}
+
+// tcgen05 with a selectable CTA group. Every tcgen05 instruction of a kernel uses the same
+// group: 1 = one CTA, 2 = the CTA pair of a 2-CTA cluster (M = 256 MMAs, operands split
+// across the two CTAs' shared memory, issued by the pair's leader).
+template <int CG> __device__ __forceinline__ void tc_alloc(uint32_t dst_smem, uint32_t ncols) {
+  if constexpr (CG == 1) asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(dst_smem), "r"(ncols));
+  else asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(dst_smem), "r"(ncols));
+}
+template <int CG> __device__ __forceinline__ void tc_relinquish() {
+  if constexpr (CG == 1) asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  else asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+}
+template <int CG> __device__ __forceinline__ void tc_dealloc(uint32_t taddr, uint32_t ncols) {
+  if constexpr (CG == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols));
+  else asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols));
+}
+// Commit: arrive on `bar` (in this CTA and, for the pair, in both CTAs at the same offset)
+// once the issuing thread's earlier tcgen05 ops are done.
+template <int CG> __device__ __forceinline__ void tc_commit_to(uint32_t bar) {
+  if constexpr (CG == 1) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
+  } else {
+    const uint16_t mask = 0x3;
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 :: "r"(bar), "h"(mask) : "memory");
+  }
+}
+template <int CG> __device__ __forceinline__ void tc_cp_atom(uint32_t taddr, uint64_t sdesc) {
+  if constexpr (CG == 1) asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
+  else asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
+}
+#define OSC_TC_MMA_BS(NAME, KINDSTR)                                                                        \
+  template <int CG> __device__ __forceinline__ void NAME(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, \
+                                                         uint32_t sfa, uint32_t sfb, uint32_t acc) {        \
+    if constexpr (CG == 1)                                                                                  \
+      asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"                                        \
+                   "tcgen05.mma.cta_group::1." KINDSTR " [%0], %1, %2, %3, [%5], [%6], p;\n\t}"            \
+                   :: "r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb) : "memory");         \
+    else                                                                                                    \
+      asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"                                        \
+                   "tcgen05.mma.cta_group::2." KINDSTR " [%0], %1, %2, %3, [%5], [%6], p;\n\t}"            \
+                   :: "r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb) : "memory");         \
+  }
+OSC_TC_MMA_BS(tc_mma_mxf4_b32_g, "kind::mxf4.block_scale.block32")
+OSC_TC_MMA_BS(tc_mma_mxf4_b16_g, "kind::mxf4nvf4.block_scale.block16")
+OSC_TC_MMA_BS(tc_mma_mxf8_g, "kind::mxf8f6f4.block_scale.block32")
+#undef OSC_TC_MMA_BS
+template <int CG> __device__ __forceinline__ void tc_mma_bf16_g(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if constexpr (CG == 1)
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+  else
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+// Instruction descriptors with the MMA's M (128 for one CTA, 256 for the pair).
+__host__ __device__ constexpr uint32_t idesc_bs_m(uint32_t fmt, uint32_t m, uint32_t n, uint32_t sfa_id, uint32_t sfb_id) {
+  return (sfb_id << 4) | (fmt << 7) | (fmt << 10) | ((n >> 3) << 17) | (1u << 23) | ((m >> 4) << 24) | (sfa_id << 29);
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_m(uint32_t m, uint32_t n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+
 // TMEM -> registers: 32 lanes x 32 consecutive 32-bit columns per warp (lane = row).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(

@@ -56,10 +56,12 @@ struct GemmParams {
 };
 
 struct GemmMaps {
-  CUtensorMap a, b, ca, cb, y;
+  CUtensorMap a, b, sfa, sfb, ca, cb, y;
 };
 
-cudaError_t launch_gemm(int kind, int bn, const GemmMaps& maps, const GemmParams& p, int grid, cudaStream_t s);
+// cg = 1: one CTA per 128-row tile; cg = 2: a 2-CTA cluster per 256-row tile (bn = 256).
+// grid is a multiple of cg; m_tiles in p counts (128 * cg)-row tiles.
+cudaError_t launch_gemm(int kind, int bn, int cg, const GemmMaps& maps, const GemmParams& p, int grid, cudaStream_t s);
 
 struct TableParams {
   const uint16_t* X;   // S x K bf16

@@ -5,17 +5,21 @@
 // the equation of the OSC page ("W4A4量化技术：OSC框架如何实现高效LLM部署",
 // coreui.cn/article/2607942.html), §3.2: a 4-bit base path (block-scaled MXFP4, E8M0 scales)
 // plus a 16-bit compensation path for the table's outlier channels. Both run in one kernel:
-// the compensation tiles (B: 128 x 64 bf16, W_L: BN x 64 bf16) flow through the same TMA
+// the compensation tiles (B: 128 x 64 bf16, W_L: rows x 64 bf16) flow through the same TMA
 // ring as the FP4 tiles (both are 128-byte rows) and their kind::f16 MMAs accumulate into the
 // same TMEM accumulator right after the FP4 k-loop, so B * W_L costs no extra pass over Y.
 // The same kernel serves the MXFP8 fallback of §4 (E4M3 x E4M3, per-32 E8M0) and the
 // per-expert grouped form for MoE layers.
 //
 // Structure: persistent CTAs (one per SM), 8 warps.
-//   warp 0 (one lane)   TMA producer: A/B operand tiles (128B swizzle) + scale atoms (bulk copy)
+//   warp 0 (one lane)   TMA producer: operand tiles (128B swizzle) and scale atoms
 //   warp 1 (one lane)   MMA issuer: tcgen05.cp scales -> TMEM, tcgen05.mma, tcgen05.commit
 //   warp 2              TMEM allocator
 //   warps 4..7          epilogue: tcgen05.ld (lane quadrant = warp % 4) -> bf16 -> smem -> TMA store
+// CG = 2 runs the CTA pair of a 2-CTA cluster as one M = 256 tile: each CTA loads its 128
+// rows of A and half of the BN rows of B, the leader issues cta_group::2 MMAs over both
+// CTAs' shared memory, and each CTA's TMEM holds its 128 rows of the accumulator. Per SM this
+// halves the B traffic of a 128 x BN tile for the same tensor work.
 // Scales live in TMEM as the block-scaled MMA expects: a 512-byte atom (128 rows x 4 slots)
 // is copied with tcgen05.cp 32x128b.warpx4 into 4 columns; row r's slot s is byte s%4 of
 // column (r / 32) of its atom; the MMA's scale-factor id picks the byte.
@@ -24,16 +28,18 @@
 
 namespace osc {
 
-template <int BN, int KIND>
+template <int BN, int KIND, int CG>
 struct GemmCfg {
   static constexpr bool FP8 = KIND == KIND_MXF8_B32;
   static constexpr int V = KIND == KIND_MXF4_B16 ? 16 : 32;        // scale slot width
   static constexpr int ELEMS = FP8 ? 128 : 256;                      // K elements per stage (128 bytes)
   static constexpr int APS = ELEMS / (4 * V);                        // scale atoms per stage
+  static constexpr int MMA_M = 128 * CG;
+  static constexpr int BROWS = BN / CG;                              // B rows this CTA loads
   static constexpr int A_BYTES = 128 * 128;
-  static constexpr int B_BYTES = BN * 128;
+  static constexpr int B_BYTES = BROWS * 128;
   static constexpr int SFA_BYTES = APS * 512;
-  static constexpr int SFB_BYTES = (BN / 128) * APS * 512;
+  static constexpr int SFB_BYTES = (BN / 128) * APS * 512;           // every CTA holds all BN rows
   static constexpr int STAGE_RAW = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
   static constexpr int STAGING_BYTES = 4 * 32 * 128;                 // one 32x64 bf16 tile per epilogue warp
@@ -48,19 +54,23 @@ struct GemmCfg {
   static constexpr int SFA_COL = ACC_STAGES * BN;
   static constexpr int SFB_COL = SFA_COL + SFA_COLS;
   static constexpr int TMEM_COLS = 512;
+  static constexpr uint32_t MAIN_TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // per CTA and stage
+  static constexpr uint32_t COMP_TX = A_BYTES + B_BYTES;
   static_assert(SFB_COL + SFB_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(STAGES >= 2, "smem budget");
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "tile width");
+  static_assert(CG == 1 || (CG == 2 && BN == 256), "the CTA pair uses 256-wide tiles");
 };
 
 struct TileInfo {
-  int m0, n0, e, kl;
+  int m0, n0, e, kl;   // m0: this CTA's first row
 };
 
-__device__ __forceinline__ TileInfo tile_info(int t, const GemmParams& p, int bn) {
+template <int CG>
+__device__ __forceinline__ TileInfo tile_info(int t, const GemmParams& p, int bn, int rank) {
   TileInfo ti;
-  const int mb = t % p.m_tiles, nb = t / p.m_tiles;
-  ti.m0 = mb * 128;
+  const int mb = t % p.m_tiles, nb = t / p.m_tiles;     // m_tiles counts (128 * CG)-row tiles
+  ti.m0 = mb * 128 * CG + 128 * rank;
   ti.n0 = nb * bn;
   if (p.num_groups == 0) {
     ti.e = 0;
@@ -72,12 +82,13 @@ __device__ __forceinline__ TileInfo tile_info(int t, const GemmParams& p, int bn
   return ti;
 }
 
-template <int BN, int KIND>
+template <int BN, int KIND, int CG>
 __global__ void __launch_bounds__(256, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+            const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
             const __grid_constant__ CUtensorMap tmCA, const __grid_constant__ CUtensorMap tmCB,
             const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
-  using C = GemmCfg<BN, KIND>;
+  using C = GemmCfg<BN, KIND, CG>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
@@ -95,79 +106,96 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (2 * C::STAGES + 5) + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = CG == 2 ? (int)cluster_ctarank() : 0;
+  const bool leader = rank == 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(accf_bar(a), 1); mbar_init(acce_bar(a), 4); }
+    for (int a = 0; a < 2; ++a) { mbar_init(accf_bar(a), 1); mbar_init(acce_bar(a), 4 * CG); }
     mbar_init(tear_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB); tma_prefetch_desc(&tmY);
-    if (p.K_L > 0 || p.num_groups > 0) { tma_prefetch_desc(&tmCA); tma_prefetch_desc(&tmCB); }
+    tma_prefetch_desc(&tmSFA); tma_prefetch_desc(&tmSFB);
+    if (p.K_L > 0) { tma_prefetch_desc(&tmCA); tma_prefetch_desc(&tmCB); }
   }
-  if (warp == 2) { tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS); tmem_relinquish(); }
+  if (warp == 2) { tc_alloc<CG>(smem_u32(tmem_slot), C::TMEM_COLS); tc_relinquish<CG>(); }
   tc_fence_before();
-  __syncthreads();
+  __syncwarp();                          // the cluster barrier below is warp-aligned
+  if constexpr (CG == 2) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   const int num_tiles = p.m_tiles * p.n_tiles;
   const int n_k = p.K / C::ELEMS;
   const int n_rb = (p.N + 127) / 128;
+  const int unit = blockIdx.x / CG, nunits = gridDim.x / CG;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------------ TMA producer
     int stage = 0; uint32_t phase = 0;
     long long fills = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      const TileInfo ti = tile_info(t, p, BN);
-      const int rb0 = ti.n0 / 128;
-      int nrb = n_rb - rb0; if (nrb > BN / 128) nrb = BN / 128;
-      const uint32_t main_bytes = C::A_BYTES + C::B_BYTES + C::SFA_BYTES + nrb * C::APS * 512;
-      const uint8_t* sfa_tile = p.SFA + ((size_t)(ti.m0 / 128) * p.nslot4) * 512;
-      const uint8_t* sfb_grp = p.SFB + (size_t)ti.e * n_rb * p.nslot4 * 512;
+    for (int t = unit; t < num_tiles; t += nunits) {
+      const TileInfo ti = tile_info<CG>(t, p, BN, rank);
+      const int brow = ti.n0 + rank * C::BROWS;
       bool ok = true;
       for (int ks = 0; ks < n_k && ok; ++ks) {
         if (!(ok = mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, p.status))) break;
-        const uint32_t fb = full_bar(stage);
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(fb, main_bytes);
-        tma_load_2d(st, &tmA, ks * 128, ti.m0, fb);
-        tma_load_3d(st + C::A_BYTES, &tmB, ks * 128, ti.n0, ti.e, fb);
-        bulk_load(st + C::A_BYTES + C::B_BYTES, sfa_tile + (size_t)ks * C::APS * 512, C::SFA_BYTES, fb);
-        for (int r = 0; r < nrb; ++r)
-          bulk_load(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES + r * C::APS * 512,
-                    sfb_grp + ((size_t)(rb0 + r) * p.nslot4 + (size_t)ks * C::APS) * 512, C::APS * 512, fb);
+        if constexpr (CG == 1) {
+          const uint32_t fb = full_bar(stage);
+          mbar_arrive_expect_tx(fb, C::MAIN_TX);
+          tma_load_2d(st, &tmA, ks * 128, ti.m0, fb);
+          tma_load_3d(st + C::A_BYTES, &tmB, ks * 128, brow, ti.e, fb);
+          tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFA, 0, ks * C::APS, ti.m0 / 128, fb);
+          tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, 0, ks * C::APS,
+                      ti.e * n_rb + ti.n0 / 128, fb);
+        } else {
+          const uint32_t fb = mapa_shared(full_bar(stage), 0);     // the leader counts both CTAs' bytes
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * C::MAIN_TX);
+          tma_load_2d_pair(st, &tmA, ks * 128, ti.m0, fb);
+          tma_load_3d_pair(st + C::A_BYTES, &tmB, ks * 128, brow, ti.e, fb);
+          tma_load_3d_pair(st + C::A_BYTES + C::B_BYTES, &tmSFA, 0, ks * C::APS, ti.m0 / 128, fb);
+          tma_load_3d_pair(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, 0, ks * C::APS,
+                           ti.e * n_rb + ti.n0 / 128, fb);
+        }
         ++fills;
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
       const int n_c = (ti.kl + 63) / 64;
       for (int c = 0; c < n_c && ok; ++c) {
         if (!(ok = mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, p.status))) break;
-        const uint32_t fb = full_bar(stage);
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(fb, C::A_BYTES + C::B_BYTES);
-        tma_load_2d(st, &tmCA, c * 64, ti.m0, fb);
-        tma_load_3d(st + C::A_BYTES, &tmCB, c * 64, ti.n0, ti.e, fb);
+        if constexpr (CG == 1) {
+          const uint32_t fb = full_bar(stage);
+          mbar_arrive_expect_tx(fb, C::COMP_TX);
+          tma_load_2d(st, &tmCA, c * 64, ti.m0, fb);
+          tma_load_3d(st + C::A_BYTES, &tmCB, c * 64, brow, ti.e, fb);
+        } else {
+          const uint32_t fb = mapa_shared(full_bar(stage), 0);
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * C::COMP_TX);
+          tma_load_2d_pair(st, &tmCA, c * 64, ti.m0, fb);
+          tma_load_3d_pair(st + C::A_BYTES, &tmCB, c * 64, brow, ti.e, fb);
+        }
         ++fills;
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
       if (!ok) break;
     }
-    if (*abort_flag) {
-      // let the copies this thread armed land before the CTA exits
+    if (*abort_flag && leader) {
+      // let the copies armed on this CTA's barriers land before the CTA exits
       const long long last = fills < C::STAGES ? fills : C::STAGES;
       for (long long f = fills - last; f < fills; ++f) {
         volatile int never = 0;
         mbar_wait(full_bar((int)(f % C::STAGES)), (uint32_t)((f / C::STAGES) & 1), &never, nullptr, 100000000ull);
       }
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------------------------------------------------ MMA issuer
     int stage = 0; uint32_t phase = 0;
     int acc = 0; uint32_t aphase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      const TileInfo ti = tile_info(t, p, BN);
+    for (int t = unit; t < num_tiles && ok; t += nunits) {
+      const TileInfo ti = tile_info<CG>(t, p, BN, rank);
       if (!(ok = mbar_wait(acce_bar(acc), aphase ^ 1, abort_flag, p.status))) break;
       tc_fence_after();
       const uint32_t d = tmem + acc * BN;
@@ -179,10 +207,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         const uint32_t s_sfb = s_sfa + C::SFA_BYTES;
 #pragma unroll
         for (int a = 0; a < C::APS; ++a) {
-          tc_cp_scale_atom(tmem + C::SFA_COL + 4 * a, desc_scale_atom(s_sfa + 512 * a));
+          tc_cp_atom<CG>(tmem + C::SFA_COL + 4 * a, desc_scale_atom(s_sfa + 512 * a));
 #pragma unroll
           for (int r = 0; r < BN / 128; ++r)
-            tc_cp_scale_atom(tmem + C::SFB_COL + a * (BN / 32) + 4 * r, desc_scale_atom(s_sfb + (r * C::APS + a) * 512));
+            tc_cp_atom<CG>(tmem + C::SFB_COL + a * (BN / 32) + 4 * r, desc_scale_atom(s_sfb + (r * C::APS + a) * 512));
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -191,17 +219,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           const uint32_t accum = (ks > 0 || j > 0) ? 1u : 0u;
           if constexpr (KIND == KIND_MXF4_B32) {
             const uint32_t sf = 2 * (j & 1), atom = j >> 1;
-            tc_mma_mxf4_b32(d, ad, bd, idesc_block_scaled(FMT_MXF4_E2M1, BN, sf, sf),
-                            tmem + C::SFA_COL + 4 * atom, tmem + C::SFB_COL + atom * (BN / 32), accum);
+            tc_mma_mxf4_b32_g<CG>(d, ad, bd, idesc_bs_m(FMT_MXF4_E2M1, C::MMA_M, BN, sf, sf),
+                                  tmem + C::SFA_COL + 4 * atom, tmem + C::SFB_COL + atom * (BN / 32), accum);
           } else if constexpr (KIND == KIND_MXF4_B16) {
-            tc_mma_mxf4_b16(d, ad, bd, idesc_block_scaled(FMT_MXF4_E2M1, BN, 0, 0),
-                            tmem + C::SFA_COL + 4 * j, tmem + C::SFB_COL + j * (BN / 32), accum);
+            tc_mma_mxf4_b16_g<CG>(d, ad, bd, idesc_bs_m(FMT_MXF4_E2M1, C::MMA_M, BN, 0, 0),
+                                  tmem + C::SFA_COL + 4 * j, tmem + C::SFB_COL + j * (BN / 32), accum);
           } else {
-            tc_mma_mxf8(d, ad, bd, idesc_block_scaled(FMT_F8_E4M3, BN, j, j),
-                        tmem + C::SFA_COL, tmem + C::SFB_COL, accum);
+            tc_mma_mxf8_g<CG>(d, ad, bd, idesc_bs_m(FMT_F8_E4M3, C::MMA_M, BN, j, j),
+                              tmem + C::SFA_COL, tmem + C::SFB_COL, accum);
           }
         }
-        tc_commit(empty_bar(stage));
+        tc_commit_to<CG>(empty_bar(stage));
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
       const int n_c = (ti.kl + 63) / 64;
@@ -211,17 +239,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
         const int nm = min(4, (ti.kl - 64 * c) / 16);
         for (int j = 0; j < nm; ++j)
-          tc_mma_bf16(d, desc_kmajor_sw128(st + 32 * j), desc_kmajor_sw128(st + C::A_BYTES + 32 * j),
-                      idesc_bf16(BN), 1u);
-        tc_commit(empty_bar(stage));
+          tc_mma_bf16_g<CG>(d, desc_kmajor_sw128(st + 32 * j), desc_kmajor_sw128(st + C::A_BYTES + 32 * j),
+                            idesc_bf16_m(C::MMA_M, BN), 1u);
+        tc_commit_to<CG>(empty_bar(stage));
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
       if (!ok) break;
-      tc_commit(accf_bar(acc));
+      tc_commit_to<CG>(accf_bar(acc));
       if (C::ACC_STAGES == 2) { acc ^= 1; if (acc == 0) aphase ^= 1; } else { aphase ^= 1; }
     }
     if (*abort_flag) {
-      tc_commit(tear_bar);
+      tc_commit_to<CG>(tear_bar);
       volatile int never = 0;
       mbar_wait(tear_bar, 0, &never, nullptr, 100000000ull);
     }
@@ -231,8 +259,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const uint32_t stg = s_staging + q * (32 * 128);
     uint8_t* stg_ptr = smem + C::STAGES * C::STAGE_BYTES + q * (32 * 128);
     int acc = 0; uint32_t aphase = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      const TileInfo ti = tile_info(t, p, BN);
+    for (int t = unit; t < num_tiles; t += nunits) {
+      const TileInfo ti = tile_info<CG>(t, p, BN, rank);
       if (!mbar_wait(accf_bar(acc), aphase, abort_flag, p.status)) break;
       tc_fence_after();
       const int row = ti.m0 + 32 * q + lane;
@@ -260,7 +288,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acce_bar(acc));
+      if (lane == 0) {
+        if constexpr (CG == 1) mbar_arrive(acce_bar(acc));
+        else mbar_arrive_cluster(mapa_shared(acce_bar(acc), 0));
+      }
       if (C::ACC_STAGES == 2) { acc ^= 1; if (acc == 0) aphase ^= 1; } else { aphase ^= 1; }
 
       const bool rows_live = ti.m0 + 32 * q < p.M;
@@ -284,35 +315,58 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   }
 
   tc_fence_before();
-  __syncthreads();
+  __syncwarp();                          // role lanes rejoin their warps before the aligned barrier
+  if constexpr (CG == 2) cluster_sync(); else __syncthreads();
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    tc_dealloc<CG>(tmem, C::TMEM_COLS);
   }
 }
 
-template <int BN, int KIND>
+template <int BN, int KIND, int CG>
 static cudaError_t launch_one(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t s) {
-  using C = GemmCfg<BN, KIND>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_TOTAL);
+  using C = GemmCfg<BN, KIND, CG>;
+  static int attr_done[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, KIND, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_TOTAL);
     if (e != cudaSuccess) return e;
-    attr_done = true;
+    attr_done[dev] = 1;
   }
-  gemm_kernel<BN, KIND><<<grid, 256, C::SMEM_TOTAL, s>>>(m.a, m.b, m.ca, m.cb, m.y, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_TOTAL;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<BN, KIND, CG>, m.a, m.b, m.sfa, m.sfb, m.ca, m.cb, m.y, p);
 }
 
-cudaError_t launch_gemm(int kind, int bn, const GemmMaps& maps, const GemmParams& p, int grid, cudaStream_t s) {
+cudaError_t launch_gemm(int kind, int bn, int cg, const GemmMaps& maps, const GemmParams& p, int grid, cudaStream_t s) {
+  if (cg == 2) {
+    if (bn != 256) return cudaErrorInvalidValue;
+    if (kind == KIND_MXF4_B32) return launch_one<256, KIND_MXF4_B32, 2>(maps, p, grid, s);
+    if (kind == KIND_MXF4_B16) return launch_one<256, KIND_MXF4_B16, 2>(maps, p, grid, s);
+    if (kind == KIND_MXF8_B32) return launch_one<256, KIND_MXF8_B32, 2>(maps, p, grid, s);
+    return cudaErrorInvalidValue;
+  }
   if (bn == 256) {
-    if (kind == KIND_MXF4_B32) return launch_one<256, KIND_MXF4_B32>(maps, p, grid, s);
-    if (kind == KIND_MXF4_B16) return launch_one<256, KIND_MXF4_B16>(maps, p, grid, s);
-    if (kind == KIND_MXF8_B32) return launch_one<256, KIND_MXF8_B32>(maps, p, grid, s);
+    if (kind == KIND_MXF4_B32) return launch_one<256, KIND_MXF4_B32, 1>(maps, p, grid, s);
+    if (kind == KIND_MXF4_B16) return launch_one<256, KIND_MXF4_B16, 1>(maps, p, grid, s);
+    if (kind == KIND_MXF8_B32) return launch_one<256, KIND_MXF8_B32, 1>(maps, p, grid, s);
   } else if (bn == 128) {
-    if (kind == KIND_MXF4_B32) return launch_one<128, KIND_MXF4_B32>(maps, p, grid, s);
-    if (kind == KIND_MXF4_B16) return launch_one<128, KIND_MXF4_B16>(maps, p, grid, s);
-    if (kind == KIND_MXF8_B32) return launch_one<128, KIND_MXF8_B32>(maps, p, grid, s);
+    if (kind == KIND_MXF4_B32) return launch_one<128, KIND_MXF4_B32, 1>(maps, p, grid, s);
+    if (kind == KIND_MXF4_B16) return launch_one<128, KIND_MXF4_B16, 1>(maps, p, grid, s);
+    if (kind == KIND_MXF8_B32) return launch_one<128, KIND_MXF8_B32, 1>(maps, p, grid, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -7,9 +7,10 @@
 // high-precision buffer B and zero it, then microscale the zeroed group (a tighter scale).
 // §4: the W2 fallback microscales to FP8 instead, with no separation.
 //
-// Work split: one thread owns 8 consecutive channels (one 16-byte load); the G/8 threads of
-// a group reduce the amax with warp shuffles; a warp covers 256 consecutive channels of one
-// row, so loads and the packed code stores are fully coalesced.
+// Work split: a warp owns one 256-channel segment over a few rows; each lane owns 8
+// consecutive channels (one 16-byte load per row) and works out once which of them is a table
+// channel; the G/8 lanes of a group reduce the amax with warp shuffles. Loads and the packed
+// code stores are fully coalesced (512 and 128 contiguous bytes per warp and row).
 #include "osc_device.cuh"
 #include "osc_internal.h"
 
@@ -20,20 +21,6 @@ namespace osc {
 // (r % 32) * 16 + (r / 32 % 4) * 4, atoms ordered by (row block, slot4).
 __device__ __forceinline__ size_t scale_word_offset(int row, int slot4, int nslot4) {
   return ((size_t)(row >> 7) * nslot4 + slot4) * 512u + (size_t)((row & 31) * 16 + ((row >> 5) & 3) * 4);
-}
-
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
-      : "=r"(r) : "f"(hi), "f"(lo));
-  return r;   // low nibble = lo, high nibble = hi
-}
-
-__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
-  uint32_t r;
-  asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\tcvt.u32.u16 %0, t;\n\t}"
-      : "=r"(r) : "f"(hi), "f"(lo));
-  return r;   // low byte = lo, high byte = hi
 }
 
 // Codes whose magnitude rounds to zero take the sign of the input (so -0.1 -> 0x8 / 0x80),
@@ -55,210 +42,211 @@ __device__ __forceinline__ uint32_t e4m3_fix_zero_sign(uint32_t h, uint32_t w0, 
   return (h & ~z) | (s & z);
 }
 
-// Stage one table in shared memory with each entry's column in B (exclusive scan over the
-// valid entries). Entries >= G, and entries beyond K_L columns, are reported and dropped.
-template <int G>
-__device__ __forceinline__ int stage_table(const int8_t* __restrict__ L, int Kg, int K_L, int8_t* Ls,
-                                           int16_t* pos, int* s_warp, int* status) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = (Kg + 255) / 256;
-  int local = 0;
-  for (int i = tid * per; i < min(Kg, tid * per + per); ++i) {
-    int v = L[i];
-    if (v >= G) { record_status(status, DEV_BAD_TABLE); v = -1; }
-    Ls[i] = (int8_t)v;
-    local += (v >= 0);
-  }
-  int incl = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int t = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += t;
-  }
-  if (lane == 31) s_warp[warp] = incl;
-  __syncthreads();
-  int base = 0, total = 0;
-  for (int w = 0; w < 8; ++w) { if (w < warp) base += s_warp[w]; total += s_warp[w]; }
-  int run = base + incl - local;
-  for (int i = tid * per; i < min(Kg, tid * per + per); ++i) {
-    if (Ls[i] >= 0) {
-      if (run >= K_L) { record_status(status, DEV_BAD_TABLE); Ls[i] = -1; }
-      pos[i] = (int16_t)run;
-      ++run;
-    }
-  }
-  __syncthreads();
-  return total < K_L ? total : K_L;
+// Eight E2M1 codes from eight fp32 values (already scaled by 2^-e), packed low nibble first.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&x)[8]) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 a, b, c, d;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 a, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 d, %8, %7;\n\t"
+      "mov.b32 %0, {a, b, c, d};\n\t}"
+      : "=r"(r) : "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]), "f"(x[4]), "f"(x[5]), "f"(x[6]), "f"(x[7]));
+  return r;
 }
 
-// One 16-byte chunk (8 channels k0..k0+7 of one row): extraction through the staged table,
-// group amax over the G/8 lanes of the group, E8M0 exponent, E2M1/E4M3 codes and the scale
-// word. Called by all 32 lanes of a warp together (the shuffles span the warp).
+// Four E4M3 codes, low byte first.
+__device__ __forceinline__ uint32_t cvt_e4m3x4(float x0, float x1, float x2, float x3) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 a, b;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 a, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 b, %4, %3;\n\t"
+      "mov.b32 %0, {a, b};\n\t}"
+      : "=r"(r) : "f"(x0), "f"(x1), "f"(x2), "f"(x3));
+  return r;
+}
+
+// What one lane needs to know about its 8 channels of a 256-channel segment, independent of
+// the row: whether the segment slot holds the table's channel, which of the 8 it is, and its
+// column in B. Computed once per warp task from the table with ballots (no shared memory).
+struct LaneTable {
+  int has;     // 1 if one of this lane's 8 channels is the group's table channel
+  int eidx;    // which of the 8
+  int pos;     // its column in B
+  int count;   // valid entries in the whole table (min K_L)
+};
+
+template <int G>
+__device__ __forceinline__ LaneTable lane_table(const int8_t* __restrict__ L, int Kg, int K_L, int seg, int lane,
+                                                int* status) {
+  constexpr int LPG = G / 8;                              // lanes per group
+  const int g0 = seg * 256 / G;                           // first group of the segment
+  const int glane = g0 + lane / LPG;
+  const unsigned full = 0xffffffffu;
+  int before = 0;
+  for (int j = 0; j < g0; j += 32) {
+    const int k = j + lane;
+    int v = (k < g0) ? (int)L[k] : -1;
+    before += __popc(__ballot_sync(full, v >= 0 && v < G));
+  }
+  int l = L[glane];
+  if (l >= G) { if (lane % LPG == 0) record_status(status, DEV_BAD_TABLE); l = -1; }
+  const unsigned firsts = __ballot_sync(full, (lane % LPG == 0) && l >= 0);
+  const int fl = (lane / LPG) * LPG;                      // first lane of my group
+  LaneTable t;
+  t.pos = before + __popc(firsts & ((1u << fl) - 1u));
+  t.eidx = l - (lane % LPG) * 8;
+  t.has = (l >= 0 && t.eidx >= 0 && t.eidx < 8) ? 1 : 0;
+  if (t.has && t.pos >= K_L) { record_status(status, DEV_BAD_TABLE); t.has = 0; }
+  t.count = 0;
+  if (seg == 0) {                                         // only segment 0 writes the pad columns
+    int c = 0;
+    for (int j = 0; j < Kg; j += 32) {
+      const int k = j + lane;
+      int v = (k < Kg) ? (int)L[k] : -1;
+      c += __popc(__ballot_sync(full, v >= 0 && v < G));
+    }
+    t.count = c < K_L ? c : K_L;
+  }
+  return t;
+}
+
+// One row of one lane: extraction, group amax (G/8 lanes), exponent, codes, scale word.
+// All 32 lanes of the warp call it together (shuffles).
 template <int G, bool FP8, bool TABLE>
-__device__ __forceinline__ void quant_chunk(uint32_t (&w)[4], int row, int kc, int K, const int8_t* Ls,
-                                            const int16_t* pos, int count, int K_L, uint16_t* __restrict__ B,
-                                            uint8_t* __restrict__ Q, uint8_t* __restrict__ S) {
+__device__ __forceinline__ void quant_row(uint4 raw, int row, int seg, int lane, int K, const LaneTable& t, int K_L,
+                                          uint16_t* __restrict__ B, uint8_t* __restrict__ Q, uint8_t* __restrict__ S,
+                                          bool store_q) {
   constexpr int V = FP8 ? 32 : (G == 16 ? 16 : 32);      // scale slot width
   constexpr int GL = (FP8 ? 32 : G) / 8;                   // lanes per amax group
   constexpr int EMAX = FP8 ? 8 : 2;
-  const int k0 = kc * 8;
+  uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
   if constexpr (TABLE) {
-    const int g = k0 / G;
-    const int l = Ls[g];
-    const int off = l - (k0 % G);
-    if (l >= 0 && off >= 0 && off < 8) {
-      const uint32_t sh = (off & 1) * 16;
-      B[(size_t)row * K_L + pos[g]] = (uint16_t)(w[off >> 1] >> sh);
-      w[off >> 1] &= ~(0xFFFFu << sh);           // the slot becomes +0
+    if (t.has) {
+      const int j = t.eidx >> 1;
+      const uint32_t sh = (t.eidx & 1) * 16;
+      if (store_q) B[(size_t)row * K_L + t.pos] = (uint16_t)(w[j] >> sh);
+      w[j] &= ~(0xFFFFu << sh);                  // the slot becomes +0
     }
-    if (kc == 0)
-      for (int i = count; i < K_L; ++i) B[(size_t)row * K_L + i] = 0;
+    if (store_q && seg == 0 && lane == 0)
+      for (int i = t.count; i < K_L; ++i) B[(size_t)row * K_L + i] = 0;
   }
-
-  // group amax on the bf16 magnitude bits (monotone for finite values)
-  uint32_t am = 0;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) am = max(am, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+  // amax over the magnitudes: for finite bf16 values |x| orders like its 15 low bits
+  const uint32_t a0 = w[0] & 0x7FFF7FFFu, a1 = w[1] & 0x7FFF7FFFu, a2 = w[2] & 0x7FFF7FFFu, a3 = w[3] & 0x7FFF7FFFu;
+  uint32_t mm = __vmaxu2(__vmaxu2(a0, a1), __vmaxu2(a2, a3));
+  uint32_t am = max(mm & 0xFFFFu, mm >> 16);
 #pragma unroll
   for (int o = 1; o < GL; o <<= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
   const int eb = (int)(am >> 7);
   const int e = (eb == 0) ? -127 : max(eb - 127 - EMAX, -127);
   const float f = __uint_as_float((uint32_t)(127 - e) << 23);   // 2^-e, exact
-
   float x[8];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     x[2 * j] = __uint_as_float(w[j] << 16) * f;
     x[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u) * f;
   }
+  const size_t chunk = (size_t)row * (K / 8) + seg * 32 + lane;
   if constexpr (!FP8) {
-    uint32_t q = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) q |= cvt_e2m1x2(x[2 * j], x[2 * j + 1]) << (8 * j);
-    q = e2m1_fix_zero_sign(q, w);
-    reinterpret_cast<uint32_t*>(Q)[(size_t)row * (K / 8) + kc] = q;
+    uint32_t q = e2m1_fix_zero_sign(cvt_e2m1x8(x), w);
+    if (store_q) reinterpret_cast<uint32_t*>(Q)[chunk] = q;
   } else {
-    uint32_t h0 = cvt_e4m3x2(x[0], x[1]) | (cvt_e4m3x2(x[2], x[3]) << 16);
-    uint32_t h1 = cvt_e4m3x2(x[4], x[5]) | (cvt_e4m3x2(x[6], x[7]) << 16);
-    h0 = e4m3_fix_zero_sign(h0, w[0], w[1]);
-    h1 = e4m3_fix_zero_sign(h1, w[2], w[3]);
-    reinterpret_cast<uint2*>(Q)[(size_t)row * (K / 8) + kc] = make_uint2(h0, h1);
+    uint32_t h0 = e4m3_fix_zero_sign(cvt_e4m3x4(x[0], x[1], x[2], x[3]), w[0], w[1]);
+    uint32_t h1 = e4m3_fix_zero_sign(cvt_e4m3x4(x[4], x[5], x[6], x[7]), w[2], w[3]);
+    if (store_q) reinterpret_cast<uint2*>(Q)[chunk] = make_uint2(h0, h1);
   }
-
-  // scale codes: the lane that starts a 4-slot word gathers it and stores 32 bits
+  // the lane that starts a 4-slot word gathers it and stores 32 bits
   const uint32_t code = (uint32_t)(e + 127);
   constexpr int SL = V / 8;                   // lanes per slot
   const uint32_t c1 = __shfl_down_sync(0xffffffffu, code, SL);
   const uint32_t c2 = __shfl_down_sync(0xffffffffu, code, 2 * SL);
   const uint32_t c3 = __shfl_down_sync(0xffffffffu, code, 3 * SL);
-  if (kc % (4 * SL) == 0) {
-    const int slot4 = k0 / (4 * V);
+  if (lane % (4 * SL) == 0) {
+    const int slot4 = (seg * 256 + lane * 8) / (4 * V);
     *reinterpret_cast<uint32_t*>(S + scale_word_offset(row, slot4, K / V / 4)) =
         code | (c1 << 8) | (c2 << 16) | (c3 << 24);
   }
 }
 
+constexpr int QROWS = 8;   // rows per warp task (divides 128, so a task never leaves a 128-row block)
+
+// Dense form. A warp task is one 256-channel segment x QROWS rows; the lane's table facts are
+// worked out once per task. Rows from M up to the next multiple of 128 only get zero scales.
 template <int G, bool FP8, bool TABLE>
 __global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
-  constexpr int V = FP8 ? 32 : (G == 16 ? 16 : 32);
-  extern __shared__ __align__(16) unsigned char qsm[];
-  int8_t* Ls = reinterpret_cast<int8_t*>(qsm);
-  int16_t* pos = reinterpret_cast<int16_t*>(qsm + ((p.Kg + 15) & ~15));
-  __shared__ int s_warp[8];
-  const int K = p.K, M = p.M;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int count = 0;
-  if constexpr (TABLE) count = stage_table<G>(p.L, p.Kg, p.K_L, Ls, pos, s_warp, p.status);
-
-  const int cpr = K / 8;                        // 16-byte chunks per row
-  const long long total = (long long)M * cpr;   // a multiple of 32 (K % 256 == 0)
-  const long long gwarp = (long long)blockIdx.x * 8 + warp;
-  const long long nwarps = (long long)gridDim.x * 8;
-  constexpr int U = 2;                          // two independent 16-byte loads in flight per thread
-  for (long long base = gwarp * 32 * U; base < total; base += nwarps * 32 * U) {
-    uint4 raw[U];
+  const int lane = threadIdx.x & 31;
+  const int nseg = p.K / 256;
+  const int mpad = (p.M + 127) / 128 * 128;
+  const int tasks = nseg * (mpad / QROWS);
+  const int cpr = p.K / 8;
+  for (int task = blockIdx.x * 8 + (threadIdx.x >> 5); task < tasks; task += gridDim.x * 8) {
+    const int seg = task % nseg;
+    const int r0 = (task / nseg) * QROWS;
+    LaneTable t{};
+    if constexpr (TABLE) t = lane_table<G>(p.L, p.Kg, p.K_L, seg, lane, p.status);
+    const uint4* src = reinterpret_cast<const uint4*>(p.X) + seg * 32 + lane;
 #pragma unroll
-    for (int u = 0; u < U; ++u)
-      if (base + u * 32 < total) raw[u] = __ldcs(reinterpret_cast<const uint4*>(p.X) + base + u * 32 + lane);
+    for (int h = 0; h < QROWS; h += 4) {
+      uint4 raw[4];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (base + u * 32 >= total) break;          // warp-uniform
-      const long long c = base + u * 32 + lane;
-      const int row = (int)(c / cpr);
-      const int kc = (int)(c - (long long)row * cpr);
-      uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-      quant_chunk<G, FP8, TABLE>(w, row, kc, K, Ls, pos, count, p.K_L, p.B, p.Q, p.S);
+      for (int u = 0; u < 4; ++u) {
+        const int r = r0 + h + u;
+        raw[u] = r < p.M ? __ldcs(src + (size_t)r * cpr) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = r0 + h + u;
+        quant_row<G, FP8, TABLE>(raw[u], r, seg, lane, p.K, t, p.K_L, p.B, p.Q, p.S, r < p.M);
+      }
     }
-  }
-
-  // rows between M and the next multiple of 128 hold zero scales (2^-127)
-  const int nslot4 = K / V / 4;
-  const int mpad = (M + 127) / 128 * 128;
-  const long long npad = (long long)(mpad - M) * nslot4;
-  for (long long i = (long long)blockIdx.x * 256 + tid; i < npad; i += (long long)gridDim.x * 256) {
-    const int row = M + (int)(i / nslot4);
-    const int s4 = (int)(i % nslot4);
-    *reinterpret_cast<uint32_t*>(p.S + scale_word_offset(row, s4, nslot4)) = 0u;
   }
 }
 
-// Grouped (MoE) form: each CTA takes whole 128-row blocks of the padded row space; a block
-// belongs to one expert, whose table is staged once. Rows past the expert's token count are
-// padding and are written as zeros (codes 0, scale 2^-127, B 0).
+// Grouped (MoE) form over the padded row space: a task's rows lie in one 128-row block, which
+// belongs to one expert; rows past the expert's token count are padding and come out as zeros.
 template <int G>
 __global__ void __launch_bounds__(256) quantize_grouped_kernel(GroupedQuantParams p) {
-  extern __shared__ __align__(16) unsigned char qsm[];
-  int8_t* Ls = reinterpret_cast<int8_t*>(qsm);
-  int16_t* pos = reinterpret_cast<int16_t*>(qsm + ((p.Kg + 15) & ~15));
-  __shared__ int s_warp[8];
-  const int K = p.K;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int cpr = K / 8;
-  const int nblocks = p.Mp / 128;
-  for (int mb = blockIdx.x; mb < nblocks; mb += gridDim.x) {
-    const int e = __ldg(p.mblock_expert + mb);
-    const int cnt = __ldg(p.off + e + 1) - __ldg(p.off + e);
+  const int lane = threadIdx.x & 31;
+  const int nseg = p.K / 256;
+  const int tasks = nseg * (p.Mp / QROWS);
+  const int cpr = p.K / 8;
+  for (int task = blockIdx.x * 8 + (threadIdx.x >> 5); task < tasks; task += gridDim.x * 8) {
+    const int seg = task % nseg;
+    const int r0 = (task / nseg) * QROWS;
+    const int e = __ldg(p.mblock_expert + r0 / 128);
     const int src0 = __ldg(p.off + e);
+    const int cnt = __ldg(p.off + e + 1) - src0;
     const int prow0 = __ldg(p.poff + e);
-    __syncthreads();                               // the previous block's table readers are done
-    const int count = stage_table<G>(p.L + (size_t)e * p.Kg, p.Kg, p.K_L, Ls, pos, s_warp, p.status);
-    const int total = 128 * cpr;                   // chunks in this block, a multiple of 32
-    for (int base = warp * 64; base < total; base += 8 * 64) {
-      uint4 raw[2];
-      int rows[2], kcs[2];
+    const LaneTable t = lane_table<G>(p.L + (size_t)e * p.Kg, p.Kg, p.K_L, seg, lane, p.status);
+    const uint4* src = reinterpret_cast<const uint4*>(p.X) + seg * 32 + lane;
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int c = base + u * 32 + lane;
-        rows[u] = mb * 128 + c / cpr;
-        kcs[u] = c % cpr;
-        const int local = rows[u] - prow0;
-        raw[u] = make_uint4(0u, 0u, 0u, 0u);
-        if (base + u * 32 < total && local < cnt)
-          raw[u] = __ldcs(reinterpret_cast<const uint4*>(p.X + (size_t)(src0 + local) * K) + kcs[u]);
+    for (int h = 0; h < QROWS; h += 4) {
+      uint4 raw[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int local = r0 + h + u - prow0;
+        raw[u] = local < cnt ? __ldcs(src + (size_t)(src0 + local) * cpr) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        if (base + u * 32 >= total) break;         // warp-uniform
-        uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-        quant_chunk<G, false, true>(w, rows[u], kcs[u], K, Ls, pos, count, p.K_L, p.B, p.Q, p.S);
-      }
+      for (int u = 0; u < 4; ++u)
+        quant_row<G, false, true>(raw[u], r0 + h + u, seg, lane, p.K, t, p.K_L, p.B, p.Q, p.S, true);
     }
   }
 }
 
 template <int G, bool FP8, bool TABLE>
 static cudaError_t launch_quant(const QuantParams& p, int grid, cudaStream_t s) {
-  size_t smem = TABLE ? (size_t)((p.Kg + 15) & ~15) + (size_t)p.Kg * 2 : 0;
-  quantize_kernel<G, FP8, TABLE><<<grid, 256, smem, s>>>(p);
+  quantize_kernel<G, FP8, TABLE><<<grid, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 
+static int quant_grid(long long tasks, int num_sms) {
+  const long long want = (tasks + 7) / 8;
+  return (int)std::max<long long>(1, std::min<long long>(want, (long long)num_sms * 8));
+}
+
 cudaError_t launch_quantize(const QuantParams& p, bool fp8, int num_sms, cudaStream_t s) {
-  const long long chunks = (long long)p.M * (p.K / 8);
-  long long want = (chunks + 511) / 512;                 // 256 threads x 2 chunks
-  const long long pad_words = (long long)((p.M + 127) / 128 * 128 - p.M) * (p.K / 128);
-  want = std::max(want, (pad_words + 255) / 256);
-  const int grid = (int)std::min<long long>(std::max<long long>(want, 1), (long long)num_sms * 8);
+  const int grid = quant_grid((long long)(p.K / 256) * ((p.M + 127) / 128 * 128 / QROWS), num_sms);
   const bool table = p.L != nullptr;
   if (fp8) return launch_quant<32, true, false>(p, grid, s);
   switch (p.G) {
@@ -270,14 +258,12 @@ cudaError_t launch_quantize(const QuantParams& p, bool fp8, int num_sms, cudaStr
 }
 
 cudaError_t launch_quantize_grouped(const GroupedQuantParams& p, int num_sms, cudaStream_t s) {
-  const int nblocks = p.Mp / 128;
-  if (nblocks == 0) return cudaSuccess;
-  const int grid = std::min(nblocks, num_sms * 4);
-  const size_t smem = (size_t)((p.Kg + 15) & ~15) + (size_t)p.Kg * 2;
+  if (p.Mp == 0) return cudaSuccess;
+  const int grid = quant_grid((long long)(p.K / 256) * (p.Mp / QROWS), num_sms);
   switch (p.G) {
-    case 16: quantize_grouped_kernel<16><<<grid, 256, smem, s>>>(p); break;
-    case 32: quantize_grouped_kernel<32><<<grid, 256, smem, s>>>(p); break;
-    case 64: quantize_grouped_kernel<64><<<grid, 256, smem, s>>>(p); break;
+    case 16: quantize_grouped_kernel<16><<<grid, 256, 0, s>>>(p); break;
+    case 32: quantize_grouped_kernel<32><<<grid, 256, 0, s>>>(p); break;
+    case 64: quantize_grouped_kernel<64><<<grid, 256, 0, s>>>(p); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -55,6 +55,7 @@ def lib() -> ctypes.CDLL:
             "osc_linear_grouped": ([P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P], i32),
             "osc_status": ([P, P], i32),
             "osc_set_tile_n": ([i32], i32),
+            "osc_set_cta_pair": ([i32], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -102,6 +103,10 @@ def osc_table_kl(L) -> int:
 
 def osc_set_tile_n(bn: int) -> int:
     return int(lib().osc_set_tile_n(bn))
+
+
+def osc_set_cta_pair(mode: int) -> int:
+    return int(lib().osc_set_cta_pair(mode))
 
 
 # ---- raw calls (outputs given) -----------------------------------------------------------------
