@@ -103,7 +103,7 @@ OSC_API int osc_build_table(const uint16_t* Xcal, int S, int K, int G, float alp
 /* §3.2, Figure 2 (online): extraction + zeroing through the table, then MXFP4 quantization
  * of the zeroed tensor. X (M x K bf16) -> QX (M x K/2), SX (osc_scale_bytes(M, K, G)),
  * B (M x K_L bf16). L may be NULL (no table: plain MXFP4; then K_L must be 0 and B may be
- * NULL). X is not modified. */
+ * NULL). X is not modified. With a table, K/G may be at most 1024. */
 OSC_API int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int K_L,
                  uint8_t* QX, uint8_t* SX, uint16_t* B, osc_stream_t stream);
 

@@ -149,8 +149,8 @@ int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
   }
   {
     uint64_t d[2] = {(uint64_t)N, (uint64_t)M}, st[1] = {(uint64_t)N * 2};
-    uint32_t box[2] = {64, 32};
-    if ((rc = make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, d, st, box, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+    uint32_t box[2] = {32, 32};
+    if ((rc = make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, d, st, box, CU_TENSOR_MAP_SWIZZLE_64B))) return rc;
   }
   osc::GemmParams p;
   std::memset(&p, 0, sizeof(p));
@@ -246,7 +246,7 @@ int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int K_
   if (!X || !QX || !SX || M < 0 || K <= 0 || K_L < 0) return OSC_ERR_ARG;
   if (L == nullptr && K_L != 0) return OSC_ERR_ARG;
   if (L != nullptr && K_L > 0 && !B) return OSC_ERR_ARG;
-  if (K_L > 32767) return OSC_ERR_ARG;
+  if (K_L > 32767 || (L != nullptr && K / G > 1024)) return OSC_ERR_ARG;
   if (!a16(X) || !a16(QX) || !a16(SX) || (B && !a16(B))) return OSC_ERR_ALIGN;
   if (K % 256 != 0 || K_L % 16 != 0) return OSC_ERR_ALIGN;
   DeviceState* ds = nullptr;

@@ -15,7 +15,9 @@
 //   warp 0 (one lane)   TMA producer: operand tiles (128B swizzle) and scale atoms
 //   warp 1 (one lane)   MMA issuer: tcgen05.cp scales -> TMEM, tcgen05.mma, tcgen05.commit
 //   warp 2              TMEM allocator
-//   warps 4..7          epilogue: tcgen05.ld (lane quadrant = warp % 4) -> bf16 -> smem -> TMA store
+//   warps 4..11         epilogue, two warps per TMEM lane quadrant (warp % 4), each owning half
+//                       of the accumulator columns: tcgen05.ld all of them in one round trip,
+//                       release the accumulator, then bf16 -> smem -> TMA store
 // CG = 2 runs the CTA pair of a 2-CTA cluster as one M = 256 tile: each CTA loads its 128
 // rows of A and half of the BN rows of B, the leader issues cta_group::2 MMAs over both
 // CTAs' shared memory, and each CTA's TMEM holds its 128 rows of the accumulator. Per SM this
@@ -42,7 +44,9 @@ struct GemmCfg {
   static constexpr int SFB_BYTES = (BN / 128) * APS * 512;           // every CTA holds all BN rows
   static constexpr int STAGE_RAW = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
-  static constexpr int STAGING_BYTES = 4 * 32 * 128;                 // one 32x64 bf16 tile per epilogue warp
+  static constexpr int EPI_WARPS = 8;                                // two per TMEM lane quadrant
+  static constexpr int EPI_COLS = BN / 2;                            // accumulator columns per epilogue warp
+  static constexpr int STAGING_BYTES = EPI_WARPS * 32 * 64;          // one 32x32 bf16 tile per epilogue warp
   static constexpr int BAR_BYTES = 1024;
   static constexpr int SMEM_LIMIT = 232448;
   static constexpr int STAGES_FIT = (SMEM_LIMIT - STAGING_BYTES - BAR_BYTES - 1024) / STAGE_BYTES;
@@ -82,8 +86,10 @@ __device__ __forceinline__ TileInfo tile_info(int t, const GemmParams& p, int bn
   return ti;
 }
 
+constexpr int GEMM_THREADS = 384;
+
 template <int BN, int KIND, int CG>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
             const __grid_constant__ CUtensorMap tmCA, const __grid_constant__ CUtensorMap tmCB,
@@ -110,7 +116,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   const bool leader = rank == 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(accf_bar(a), 1); mbar_init(acce_bar(a), 4 * CG); }
+    for (int a = 0; a < 2; ++a) { mbar_init(accf_bar(a), 1); mbar_init(acce_bar(a), C::EPI_WARPS * CG); }
     mbar_init(tear_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -255,36 +261,47 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ epilogue
-    const int q = warp & 3;
-    const uint32_t stg = s_staging + q * (32 * 128);
-    uint8_t* stg_ptr = smem + C::STAGES * C::STAGE_BYTES + q * (32 * 128);
+    const int q = warp & 3;                            // TMEM lane quadrant of this warp
+    const int half = (warp - 4) >> 2;                  // which half of the accumulator columns
+    const int ew = warp - 4;
+    const uint32_t stg = s_staging + ew * (32 * 64);
+    uint8_t* stg_ptr = smem + C::STAGES * C::STAGE_BYTES + ew * (32 * 64);
+    constexpr int NCH = C::EPI_COLS / 32;              // 32-column chunks per warp (4 or 2)
     int acc = 0; uint32_t aphase = 0;
     for (int t = unit; t < num_tiles; t += nunits) {
       const TileInfo ti = tile_info<CG>(t, p, BN, rank);
       if (!mbar_wait(accf_bar(acc), aphase, abort_flag, p.status)) break;
       tc_fence_after();
       const int row = ti.m0 + 32 * q + lane;
-      uint32_t packed[BN / 2];
+      const int c0 = half * C::EPI_COLS;               // first accumulator column of this warp
+      const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + acc * BN + c0;
+      uint32_t packed[C::EPI_COLS / 2];
 #pragma unroll
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        uint32_t r[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + acc * BN + ch * 32, r);
+      for (int ch = 0; ch < NCH; ch += 2) {            // two chunks per TMEM round trip
+        uint32_t r[2][32];
+        tmem_ld32(tbase + ch * 32, r[0]);
+        tmem_ld32(tbase + ch * 32 + 32, r[1]);
         tmem_ld_wait();
-        if (p.Yf32 != nullptr && row < p.M) {
-          const int col0 = ti.n0 + ch * 32;
-          float* dst = p.Yf32 + (size_t)row * p.N + col0;
-          if (col0 + 32 <= p.N) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              reinterpret_cast<float4*>(dst)[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                                              __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-          } else {
-            for (int i = 0; i < 32 && col0 + i < p.N; ++i) dst[i] = __uint_as_float(r[i]);
+        for (int u = 0; u < 2; ++u) {
+          if (p.Yf32 != nullptr && row < p.M) {
+            const int col0 = ti.n0 + c0 + (ch + u) * 32;
+            float* dst = p.Yf32 + (size_t)row * p.N + col0;
+            if (col0 + 32 <= p.N) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                reinterpret_cast<float4*>(dst)[i] = make_float4(__uint_as_float(r[u][4 * i]), __uint_as_float(r[u][4 * i + 1]),
+                                                                __uint_as_float(r[u][4 * i + 2]), __uint_as_float(r[u][4 * i + 3]));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)         // fully unrolled: r stays in registers
+                if (col0 + i < p.N) dst[i] = __uint_as_float(r[u][i]);
+            }
           }
-        }
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          packed[ch * 16 + i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+          for (int i = 0; i < 16; ++i)
+            packed[(ch + u) * 16 + i] = pack_bf16x2(__uint_as_float(r[u][2 * i]), __uint_as_float(r[u][2 * i + 1]));
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -296,19 +313,22 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 
       const bool rows_live = ti.m0 + 32 * q < p.M;
 #pragma unroll
-      for (int cc = 0; cc < BN / 64; ++cc) {
-        if (!rows_live || ti.n0 + cc * 64 >= p.N) continue;     // warp-uniform
+      for (int cc = 0; cc < NCH; ++cc) {
+        const int col = ti.n0 + c0 + cc * 32;
+        if (!rows_live || col >= p.N) continue;        // warp-uniform
         if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
+        // 32 rows x 64 bytes in the 64-byte swizzle the store map uses: 16-byte chunk c of
+        // row r sits at chunk c ^ ((r / 2) % 4)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 v = make_uint4(packed[cc * 32 + 4 * i], packed[cc * 32 + 4 * i + 1],
-                                     packed[cc * 32 + 4 * i + 2], packed[cc * 32 + 4 * i + 3]);
-          *reinterpret_cast<uint4*>(stg_ptr + lane * 128 + ((i ^ (lane & 7)) * 16)) = v;
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = make_uint4(packed[cc * 16 + 4 * i], packed[cc * 16 + 4 * i + 1],
+                                     packed[cc * 16 + 4 * i + 2], packed[cc * 16 + 4 * i + 3]);
+          *reinterpret_cast<uint4*>(stg_ptr + lane * 64 + ((i ^ ((lane >> 1) & 3)) * 16)) = v;
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) { tma_store_2d(&tmY, stg, ti.n0 + cc * 64, ti.m0 + 32 * q); bulk_commit(); }
+        if (lane == 0) { tma_store_2d(&tmY, stg, col, ti.m0 + 32 * q); bulk_commit(); }
       }
     }
     if (lane == 0) bulk_wait<0>();
@@ -338,7 +358,7 @@ static cudaError_t launch_one(const GemmMaps& m, const GemmParams& p, int grid, 
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(256, 1, 1);
+  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_TOTAL;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];

@@ -23,25 +23,6 @@ __device__ __forceinline__ size_t scale_word_offset(int row, int slot4, int nslo
   return ((size_t)(row >> 7) * nslot4 + slot4) * 512u + (size_t)((row & 31) * 16 + ((row >> 5) & 3) * 4);
 }
 
-// Codes whose magnitude rounds to zero take the sign of the input (so -0.1 -> 0x8 / 0x80),
-// whatever the conversion instruction does with negative values that round to zero.
-__device__ __forceinline__ uint32_t e2m1_fix_zero_sign(uint32_t p, const uint32_t (&w)[4]) {
-  uint32_t nz = (p | (p >> 1) | (p >> 2)) & 0x11111111u;
-  uint32_t zpos = ((~nz) & 0x11111111u) << 3;
-  uint32_t s = 0;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) s |= (((w[j] >> 12) & 0x8u) | ((w[j] >> 24) & 0x80u)) << (8 * j);
-  return (p & ~zpos) | (s & zpos);
-}
-
-__device__ __forceinline__ uint32_t e4m3_fix_zero_sign(uint32_t h, uint32_t w0, uint32_t w1) {
-  uint32_t m = h & 0x7F7F7F7Fu;
-  uint32_t nz = ((m + 0x7F7F7F7Fu) | m) & 0x80808080u;
-  uint32_t z = (~nz) & 0x80808080u;
-  uint32_t s = ((w0 >> 8) & 0x80u) | ((w0 >> 16) & 0x8000u) | ((w1 << 8) & 0x800000u) | (w1 & 0x80000000u);
-  return (h & ~z) | (s & z);
-}
-
 // Eight E2M1 codes from eight fp32 values (already scaled by 2^-e), packed low nibble first.
 __device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&x)[8]) {
   uint32_t r;
@@ -148,11 +129,13 @@ __device__ __forceinline__ void quant_row(uint4 raw, int row, int seg, int lane,
   }
   const size_t chunk = (size_t)row * (K / 8) + seg * 32 + lane;
   if constexpr (!FP8) {
-    uint32_t q = e2m1_fix_zero_sign(cvt_e2m1x8(x), w);
+    // the conversion keeps the sign of values that round to zero (-0.1 -> 0x8), as the
+    // element rule requires; the every-bf16-value parity tests pin that behaviour
+    uint32_t q = cvt_e2m1x8(x);
     if (store_q) reinterpret_cast<uint32_t*>(Q)[chunk] = q;
   } else {
-    uint32_t h0 = e4m3_fix_zero_sign(cvt_e4m3x4(x[0], x[1], x[2], x[3]), w[0], w[1]);
-    uint32_t h1 = e4m3_fix_zero_sign(cvt_e4m3x4(x[4], x[5], x[6], x[7]), w[2], w[3]);
+    const uint32_t h0 = cvt_e4m3x4(x[0], x[1], x[2], x[3]);
+    const uint32_t h1 = cvt_e4m3x4(x[4], x[5], x[6], x[7]);
     if (store_q) reinterpret_cast<uint2*>(Q)[chunk] = make_uint2(h0, h1);
   }
   // the lane that starts a 4-slot word gathers it and stores 32 bits
@@ -168,36 +151,77 @@ __device__ __forceinline__ void quant_row(uint4 raw, int row, int seg, int lane,
   }
 }
 
-constexpr int QROWS = 8;   // rows per warp task (divides 128, so a task never leaves a 128-row block)
+constexpr int QROWS = 8;   // rows per dense warp task (divides 128: a task never leaves a 128-row block)
+constexpr int GROWS = 8;   // rows per grouped warp task
+constexpr int MAX_KG = 1024;
 
-// Dense form. A warp task is one 256-channel segment x QROWS rows; the lane's table facts are
-// worked out once per task. Rows from M up to the next multiple of 128 only get zero scales.
+// Dense form. The CTA stages the table once: each entry's channel and its column in B
+// (exclusive count of the valid entries before it). A warp task is one 256-channel segment x
+// QROWS rows; its lanes read their table facts from shared memory. Rows from M up to the
+// next multiple of 128 only get zero scales.
 template <int G, bool FP8, bool TABLE>
 __global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
-  const int lane = threadIdx.x & 31;
+  __shared__ int8_t s_l[TABLE ? MAX_KG : 1];
+  __shared__ int16_t s_pos[TABLE ? MAX_KG : 1];
+  __shared__ int s_warp[8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int count = 0;
+  if constexpr (TABLE) {
+    const int per = (p.Kg + 255) / 256;
+    const int i0 = threadIdx.x * per, i1 = min(p.Kg, i0 + per);
+    int local = 0;
+    for (int i = i0; i < i1; ++i) {
+      int v = p.L[i];
+      if (v >= G) { record_status(p.status, DEV_BAD_TABLE); v = -1; }
+      s_l[i] = (int8_t)v;
+      local += v >= 0;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    int run = incl - local;
+    for (int w = 0; w < 8; ++w) { if (w < warp) run += s_warp[w]; count += s_warp[w]; }
+    for (int i = i0; i < i1; ++i)
+      if (s_l[i] >= 0) {
+        if (run >= p.K_L) { record_status(p.status, DEV_BAD_TABLE); s_l[i] = -1; }
+        s_pos[i] = (int16_t)run++;
+      }
+    count = min(count, p.K_L);
+    __syncthreads();
+  }
   const int nseg = p.K / 256;
   const int mpad = (p.M + 127) / 128 * 128;
   const int tasks = nseg * (mpad / QROWS);
   const int cpr = p.K / 8;
-  for (int task = blockIdx.x * 8 + (threadIdx.x >> 5); task < tasks; task += gridDim.x * 8) {
+  for (int task = blockIdx.x * 8 + warp; task < tasks; task += gridDim.x * 8) {
     const int seg = task % nseg;
     const int r0 = (task / nseg) * QROWS;
     LaneTable t{};
-    if constexpr (TABLE) t = lane_table<G>(p.L, p.Kg, p.K_L, seg, lane, p.status);
+    if constexpr (TABLE) {
+      const int k0 = seg * 256 + lane * 8;
+      const int g = k0 / G;
+      const int l = s_l[g];
+      t.eidx = l - (k0 % G);
+      t.has = (l >= 0 && t.eidx >= 0 && t.eidx < 8) ? 1 : 0;
+      t.pos = s_pos[g];
+      t.count = count;
+    }
     const uint4* src = reinterpret_cast<const uint4*>(p.X) + seg * 32 + lane;
+    uint4 raw[QROWS];                               // all of the task's loads in flight at once
 #pragma unroll
-    for (int h = 0; h < QROWS; h += 4) {
-      uint4 raw[4];
+    for (int u = 0; u < QROWS; ++u) {
+      const int r = r0 + u;
+      raw[u] = r < p.M ? __ldcs(src + (size_t)r * cpr) : make_uint4(0u, 0u, 0u, 0u);
+    }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = r0 + h + u;
-        raw[u] = r < p.M ? __ldcs(src + (size_t)r * cpr) : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = r0 + h + u;
-        quant_row<G, FP8, TABLE>(raw[u], r, seg, lane, p.K, t, p.K_L, p.B, p.Q, p.S, r < p.M);
-      }
+    for (int u = 0; u < QROWS; ++u) {
+      const int r = r0 + u;
+      quant_row<G, FP8, TABLE>(raw[u], r, seg, lane, p.K, t, p.K_L, p.B, p.Q, p.S, r < p.M);
     }
   }
 }
@@ -208,29 +232,26 @@ template <int G>
 __global__ void __launch_bounds__(256) quantize_grouped_kernel(GroupedQuantParams p) {
   const int lane = threadIdx.x & 31;
   const int nseg = p.K / 256;
-  const int tasks = nseg * (p.Mp / QROWS);
+  const int tasks = nseg * (p.Mp / GROWS);
   const int cpr = p.K / 8;
   for (int task = blockIdx.x * 8 + (threadIdx.x >> 5); task < tasks; task += gridDim.x * 8) {
     const int seg = task % nseg;
-    const int r0 = (task / nseg) * QROWS;
+    const int r0 = (task / nseg) * GROWS;
     const int e = __ldg(p.mblock_expert + r0 / 128);
     const int src0 = __ldg(p.off + e);
     const int cnt = __ldg(p.off + e + 1) - src0;
     const int prow0 = __ldg(p.poff + e);
     const LaneTable t = lane_table<G>(p.L + (size_t)e * p.Kg, p.Kg, p.K_L, seg, lane, p.status);
     const uint4* src = reinterpret_cast<const uint4*>(p.X) + seg * 32 + lane;
+    uint4 raw[GROWS];
 #pragma unroll
-    for (int h = 0; h < QROWS; h += 4) {
-      uint4 raw[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int local = r0 + h + u - prow0;
-        raw[u] = local < cnt ? __ldcs(src + (size_t)(src0 + local) * cpr) : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        quant_row<G, false, true>(raw[u], r0 + h + u, seg, lane, p.K, t, p.K_L, p.B, p.Q, p.S, true);
+    for (int u = 0; u < GROWS; ++u) {
+      const int local = r0 + u - prow0;
+      raw[u] = local < cnt ? __ldcs(src + (size_t)(src0 + local) * cpr) : make_uint4(0u, 0u, 0u, 0u);
     }
+#pragma unroll
+    for (int u = 0; u < GROWS; ++u)
+      quant_row<G, false, true>(raw[u], r0 + u, seg, lane, p.K, t, p.K_L, p.B, p.Q, p.S, true);
   }
 }
 
@@ -247,6 +268,7 @@ static int quant_grid(long long tasks, int num_sms) {
 
 cudaError_t launch_quantize(const QuantParams& p, bool fp8, int num_sms, cudaStream_t s) {
   const int grid = quant_grid((long long)(p.K / 256) * ((p.M + 127) / 128 * 128 / QROWS), num_sms);
+  if (p.L != nullptr && p.Kg > MAX_KG) return cudaErrorInvalidValue;
   const bool table = p.L != nullptr;
   if (fp8) return launch_quant<32, true, false>(p, grid, s);
   switch (p.G) {
@@ -259,7 +281,7 @@ cudaError_t launch_quantize(const QuantParams& p, bool fp8, int num_sms, cudaStr
 
 cudaError_t launch_quantize_grouped(const GroupedQuantParams& p, int num_sms, cudaStream_t s) {
   if (p.Mp == 0) return cudaSuccess;
-  const int grid = quant_grid((long long)(p.K / 256) * (p.Mp / QROWS), num_sms);
+  const int grid = quant_grid((long long)(p.K / 256) * (p.Mp / GROWS), num_sms);
   switch (p.G) {
     case 16: quantize_grouped_kernel<16><<<grid, 256, 0, s>>>(p); break;
     case 32: quantize_grouped_kernel<32><<<grid, 256, 0, s>>>(p); break;
