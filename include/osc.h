@@ -148,7 +148,8 @@ OSC_API int osc_grouped_plan(const int* counts, int E, int* off, int* poff, int*
 /* Per-expert extraction + MXFP4 quantization. X: off[E] x K bf16 (device). off, poff,
  * mblock_expert: device copies of the plan. L: E x K/G (device), expert e's table at e*K/G.
  * Outputs over the padded rows: QX (Mp x K/2), SX (osc_scale_bytes(Mp, K, G)),
- * B (Mp x K_L bf16, K_L a common width >= every expert's entry count); pad rows are 0. */
+ * B (Mp x K_L bf16, K_L a common width >= every expert's entry count); pad rows are 0.
+ * E x K/G may be at most about 68000 table entries (they are staged in shared memory). */
 OSC_API int osc_quantize_grouped(const uint16_t* X, int E, const int* off, const int* poff,
                          const int* mblock_expert, int Mp, int K, int G, const int8_t* L,
                          int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B, osc_stream_t stream);

@@ -34,6 +34,8 @@ struct GroupedQuantParams {
   int* status;
 };
 cudaError_t launch_quantize_grouped(const GroupedQuantParams& p, int num_sms, cudaStream_t s);
+// shared memory the grouped quantize needs to stage every expert's table
+size_t grouped_quant_smem(int E, int Kg);
 cudaError_t launch_gather_wl(const uint16_t* W, int N, int K, int G, const int8_t* L, int K_L, uint16_t* WL,
                              int* status, int num_sms, cudaStream_t s);
 
