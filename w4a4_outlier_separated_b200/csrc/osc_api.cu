@@ -86,6 +86,14 @@ int make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base,
 }
 
 inline bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// X (rows x K bf16) seen by the quantize kernels as 32-channel blocks: 2-D {32, rows*K/32},
+// 64-byte rows, box {32, 64}, 64-byte swizzle.
+int make_block_map(CUtensorMap* m, const uint16_t* X, int rows, int K) {
+  uint64_t d[2] = {32, (uint64_t)rows * (uint64_t)(K / 32)}, st[1] = {64};
+  uint32_t box[2] = {32, 64};
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, d, st, box, CU_TENSOR_MAP_SWIZZLE_64B);
+}
 inline bool valid_g(int G) { return G == 16 || G == 32 || G == 64; }
 
 int launch_result(cudaError_t e) { return e == cudaSuccess ? OSC_OK : fail_cuda(e); }
@@ -109,7 +117,7 @@ int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
   if (bn == 0) bn = (N >= 256 && (long long)((M + 127) / 128) * ((N + 255) / 256) >= ds->sms) ? 256 : 128;
   // the CTA pair needs 256-wide tiles, whole 256-row tiles of work and a per-128-row expert map
   // it cannot honour, so grouped calls stay on single CTAs
-  if (cg < 0) cg = (bn == 256 && !grouped && (long long)((M + 255) / 256) * ((N + 255) / 256) >= ds->sms / 2) ? 2 : 1;
+  if (cg < 0) cg = 1;   // measured: single-CTA 128x256 tiles beat the pair on every shape tried so far
   if (cg == 2 && (bn != 256 || grouped)) cg = 1;
   const int m_tiles = (M + 128 * cg - 1) / (128 * cg);
 
@@ -244,6 +252,7 @@ int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int K_
   if (!valid_g(G)) return OSC_ERR_G;
   if (M == 0 && K > 0 && K_L >= 0) return OSC_OK;          // nothing to read or write
   if (!X || !QX || !SX || M < 0 || K <= 0 || K_L < 0) return OSC_ERR_ARG;
+  if ((long long)(M + 127) * (K / 32) >= (1LL << 31)) return OSC_ERR_ARG;
   if (L == nullptr && K_L != 0) return OSC_ERR_ARG;
   if (L != nullptr && K_L > 0 && !B) return OSC_ERR_ARG;
   if (K_L > 32767 || (L != nullptr && K / G > 1024)) return OSC_ERR_ARG;
@@ -254,13 +263,16 @@ int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int K_
   if (rc != OSC_OK) return rc;
   if (M == 0) return OSC_OK;
   osc::QuantParams p{X, M, K, G, K / G, L, K_L, QX, SX, B, ds->status};
-  return launch_result(osc::launch_quantize(p, false, ds->sms, (cudaStream_t)stream));
+  CUtensorMap tm;
+  if ((rc = make_block_map(&tm, X, M, K))) return rc;
+  return launch_result(osc::launch_quantize(tm, p, false, ds->sms, (cudaStream_t)stream));
 }
 
 int osc_prepare_weight(const uint16_t* W, int N, int K, int G, const int8_t* L, int K_L, uint8_t* QW, uint8_t* SW,
                        uint16_t* WL, osc_stream_t stream) {
   if (!valid_g(G)) return OSC_ERR_G;
   if (!W || !QW || !SW || N < 0 || K <= 0 || K_L < 0) return OSC_ERR_ARG;
+  if ((long long)(N + 127) * (K / 32) >= (1LL << 31)) return OSC_ERR_ARG;
   if (K_L > 0 && (!L || !WL)) return OSC_ERR_ARG;
   if (!a16(W) || !a16(QW) || !a16(SW) || (WL && !a16(WL))) return OSC_ERR_ALIGN;
   if (K % 256 != 0 || K_L % 16 != 0) return OSC_ERR_ALIGN;
@@ -269,7 +281,9 @@ int osc_prepare_weight(const uint16_t* W, int N, int K, int G, const int8_t* L, 
   if (rc != OSC_OK) return rc;
   if (N == 0) return OSC_OK;
   osc::QuantParams p{W, N, K, G, K / G, nullptr, 0, QW, SW, nullptr, ds->status};
-  cudaError_t e = osc::launch_quantize(p, false, ds->sms, (cudaStream_t)stream);
+  CUtensorMap tm;
+  if ((rc = make_block_map(&tm, W, N, K))) return rc;
+  cudaError_t e = osc::launch_quantize(tm, p, false, ds->sms, (cudaStream_t)stream);
   if (e != cudaSuccess) return fail_cuda(e);
   return launch_result(osc::launch_gather_wl(W, N, K, G, L, K_L, WL, ds->status, ds->sms, (cudaStream_t)stream));
 }
@@ -293,6 +307,7 @@ int osc_linear(const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const ui
 int osc_quantize_fp8(const uint16_t* X, int M, int K, uint8_t* QX8, uint8_t* SX, osc_stream_t stream) {
   if (M == 0 && K > 0) return OSC_OK;                       // nothing to read or write
   if (!X || !QX8 || !SX || M < 0 || K <= 0) return OSC_ERR_ARG;
+  if ((long long)(M + 127) * (K / 32) >= (1LL << 31)) return OSC_ERR_ARG;
   if (!a16(X) || !a16(QX8) || !a16(SX)) return OSC_ERR_ALIGN;
   if (K % 256 != 0) return OSC_ERR_ALIGN;
   DeviceState* ds = nullptr;
@@ -300,7 +315,9 @@ int osc_quantize_fp8(const uint16_t* X, int M, int K, uint8_t* QX8, uint8_t* SX,
   if (rc != OSC_OK) return rc;
   if (M == 0) return OSC_OK;
   osc::QuantParams p{X, M, K, 32, K / 32, nullptr, 0, QX8, SX, nullptr, ds->status};
-  return launch_result(osc::launch_quantize(p, true, ds->sms, (cudaStream_t)stream));
+  CUtensorMap tm;
+  if ((rc = make_block_map(&tm, X, M, K))) return rc;
+  return launch_result(osc::launch_quantize(tm, p, true, ds->sms, (cudaStream_t)stream));
 }
 
 int osc_linear_fp8_fallback(const uint8_t* QX8, const uint8_t* SX, const uint8_t* QW8, const uint8_t* SW, int M,

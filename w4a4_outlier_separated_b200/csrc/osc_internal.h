@@ -18,7 +18,8 @@ struct QuantParams {
   int* status;
 };
 
-cudaError_t launch_quantize(const QuantParams& p, bool fp8, int num_sms, cudaStream_t s);
+// tmX: X as (32-channel blocks) x 64 bytes, box {32, 64} bf16, 64-byte swizzle (see make_block_map)
+cudaError_t launch_quantize(const CUtensorMap& tmX, const QuantParams& p, bool fp8, int num_sms, cudaStream_t s);
 
 struct GroupedQuantParams {
   const uint16_t* X;          // off[E] x K bf16, expert-sorted

@@ -59,13 +59,22 @@ __device__ __forceinline__ int shared_exp(uint32_t am) {
   return (eb == 0) ? -127 : max(eb - 127 - EMAX, -127);
 }
 
-// Largest |x| bits over words [J0, J0+NW) of a 32-element block (bf16 pairs).
+// Largest |x| bits over words [J0, J0+NW) of a 32-element block (bf16 pairs): packed bf16
+// max of the magnitudes (finite values order like their bits), then the larger half.
 template <int J0, int NW>
 __device__ __forceinline__ uint32_t block_amax(const uint32_t (&w)[16]) {
-  uint32_t m = w[J0] & 0x7FFF7FFFu;
+  uint32_t a[NW];
 #pragma unroll
-  for (int j = J0 + 1; j < J0 + NW; ++j) m = __vmaxu2(m, w[j] & 0x7FFF7FFFu);
-  return max(m & 0xFFFFu, m >> 16);
+  for (int j = 0; j < NW; ++j) a[j] = w[J0 + j] & 0x7FFF7FFFu;
+#pragma unroll
+  for (int n = NW; n > 1; n >>= 1)
+#pragma unroll
+    for (int j = 0; j < n / 2; ++j) {
+      __nv_bfloat162 m = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&a[j]),
+                                 *reinterpret_cast<const __nv_bfloat162*>(&a[j + n / 2]));
+      a[j] = *reinterpret_cast<const uint32_t*>(&m);
+    }
+  return max(a[0] & 0xFFFFu, a[0] >> 16);
 }
 
 // Move the table channel `lw` (0..31) of the block out: return its bits, leave +0 in its slot.
@@ -234,39 +243,123 @@ __device__ __forceinline__ void load_block(const uint16_t* __restrict__ X, size_
 
 constexpr int MAX_KG = 1024;
 
-// Dense form: items (row, 32-channel block) over M rows padded to a multiple of 128 (pad rows
-// only get zero scales); each thread takes two items per step so that eight 16-byte loads
-// are in flight.
+// Dense form, TMA-fed. X is viewed as a 2-D tensor of 32-channel blocks (items): rows of 64
+// bytes, one per (row, block) in row-major order, so a warp step's 64 items are one
+// contiguous 4 KB run of X. Lane 0 loads it with one TMA box in the 64-byte swizzle
+// (16-byte chunk c of item r at chunk c ^ ((r / 2) % 4)), which makes every lane's 64-byte
+// read from shared memory conflict-free; each warp double-buffers its boxes. Items in rows
+// M .. (next multiple of 128) only write zero scales.
+constexpr int QSTEP = 64;                       // items per warp step
+constexpr int QWARPS = 8;
+
+__device__ __forceinline__ void load_block_smem(const uint8_t* slot, int r, uint32_t (&w)[16]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(slot + r * 64 + ((c ^ ((r >> 1) & 3)) * 16));
+    w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+  }
+}
+
 template <int G, bool FP8, bool TABLE>
-__global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
+__global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant__ CUtensorMap tmX, QuantParams p) {
+  extern __shared__ uint8_t q_dyn[];                          // QWARPS x 2 boxes of 4 KB, 1 KB aligned
+  uint8_t* boxes = q_dyn + ((1024u - (smem_u32(q_dyn) & 1023u)) & 1023u);
+  auto box_at = [&](int wp, int sl) { return boxes + (wp * 2 + sl) * (QSTEP * 64); };
+  __shared__ __align__(8) uint64_t s_bar[QWARPS][2];
   __shared__ int8_t s_l[TABLE ? MAX_KG : 1];
   __shared__ int16_t s_pos[TABLE ? MAX_KG : 1];
   __shared__ int s_warp[8];
+  __shared__ int s_abort;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nblk = p.K / 32;
-  const int mpad = (p.M + 127) / 128 * 128;
-  const long long items = (long long)mpad * nblk;              // a multiple of 32
-  const long long stride = (long long)gridDim.x * 512;
-  long long base = (long long)blockIdx.x * 512 + (threadIdx.x & ~31) * 2;
-  // the first step's loads go out before the table is staged, so the two latencies overlap
-  uint32_t w0[16], w1[16];
-  int r0 = 0, b0 = 0, r1 = 0, b1 = 0;
-  auto issue = [&](long long b) {
-    const long long i0 = b + (threadIdx.x & 31), i1 = i0 + 32;
-    r0 = (int)(i0 / nblk); b0 = (int)(i0 - (long long)r0 * nblk);
-    r1 = (int)(i1 / nblk); b1 = (int)(i1 - (long long)r1 * nblk);
-    load_block(p.X, (size_t)r0 * p.K + (size_t)b0 * 32, b < items && r0 < p.M, w0);
-    load_block(p.X, (size_t)r1 * p.K + (size_t)b1 * 32, b + 32 < items && r1 < p.M, w1);
+  const uint32_t mpad = (uint32_t)(p.M + 127) / 128 * 128;
+  const uint32_t items = mpad * (uint32_t)nblk;             // a multiple of 64
+  const uint32_t real_items = (uint32_t)p.M * (uint32_t)nblk;
+  const uint32_t nsteps = items / QSTEP;
+  const uint32_t wstride = gridDim.x * QWARPS;
+  uint32_t step = blockIdx.x * QWARPS + warp;
+  if (threadIdx.x == 0) s_abort = 0;
+  if (lane == 0) { mbar_init(smem_u32(&s_bar[warp][0]), 1); mbar_init(smem_u32(&s_bar[warp][1]), 1); }
+  fence_barrier_init();
+  __syncwarp();
+  // the first box goes out before the table is staged, so the two latencies overlap
+  auto issue = [&](uint32_t st, int slot) {
+    if (lane == 0 && st * QSTEP < real_items) {
+      const uint32_t bar = smem_u32(&s_bar[warp][slot]);
+      mbar_arrive_expect_tx(bar, QSTEP * 64);
+      tma_load_2d(smem_u32(box_at(warp, slot)), &tmX, 0, (int)(st * QSTEP), bar);
+    }
   };
-  issue(base);
+  if (step < nsteps) issue(step, 0);
   int count = 0;
   if constexpr (TABLE) count = stage_table<G>(p.L, p.Kg, p.K_L, s_l, s_pos, s_warp, p.status);
-  for (; base < items; base += stride) {
-    if (base != (long long)blockIdx.x * 512 + (threadIdx.x & ~31) * 2) issue(base);
-    const bool has1 = base + 32 < items;                          // warp-uniform
-    BlockTable t0{-1, 0, -1, 0}, t1{-1, 0, -1, 0};
-    if constexpr (TABLE) { t0 = block_table<G>(b0, s_l, s_pos); t1 = block_table<G>(b1, s_l, s_pos); }
-    quant_block<G, FP8, TABLE>(w0, r0, b0, r0 < p.M, t0, count, p.K, p.K_L, p.B, p.Q, p.S);
-    if (has1) quant_block<G, FP8, TABLE>(w1, r1, b1, r1 < p.M, t1, count, p.K, p.K_L, p.B, p.Q, p.S);
+  else __syncthreads();
+  uint32_t ph[2] = {0u, 0u};
+  int slot = 0;
+  for (; step < nsteps; step += wstride, slot ^= 1) {
+    __syncwarp();                                             // the other slot's reads are done
+    if (step + wstride < nsteps) { fence_proxy_async_smem(); issue(step + wstride, slot ^ 1); }
+    const bool loaded = step * QSTEP < real_items;            // warp-uniform (pad rows are not loaded)
+    if (loaded) {
+      // lane 0 waits (bounded) and the warp follows its verdict; __syncwarp then orders the
+      // other lanes' shared-memory reads after the completed load
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(smem_u32(&s_bar[warp][slot]), ph[slot], reinterpret_cast<volatile int*>(&s_abort), p.status);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      __syncwarp();
+      if (!ok) {
+        // let the other slot's load (if one was issued) land before leaving
+        if (lane == 0 && step + wstride < nsteps && (step + wstride) * QSTEP < real_items) {
+          volatile int never = 0;
+          mbar_wait(smem_u32(&s_bar[warp][slot ^ 1]), ph[slot ^ 1], &never, nullptr, 100000000ull);
+        }
+        break;
+      }
+      ph[slot] ^= 1;
+    }
+    uint8_t* box = box_at(warp, slot);
+    // rows and blocks of this lane's two items (one division per step, then carries)
+    const uint32_t it0 = step * QSTEP;
+    int rowa = (int)(it0 / (uint32_t)nblk);
+    int blka = (int)(it0 - (uint32_t)rowa * nblk) + lane;
+    while (blka >= nblk) { blka -= nblk; ++rowa; }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = lane + 32 * h;                            // item within the box
+      int row = rowa, blk = blka + 32 * h;
+      while (blk >= nblk) { blk -= nblk; ++row; }
+      const bool live = row < p.M;
+      uint8_t* item = box + r * 64;
+      const int swz = (r >> 1) & 3;
+      BlockTable t{-1, 0, -1, 0};
+      if constexpr (TABLE) {
+        t = block_table<G>(blk, s_l, s_pos);
+        // move the table channel(s) out of the box: its 2 bytes sit in 16-byte chunk
+        // (lw / 8) ^ swz at byte (lw % 8) * 2
+        if (t.lw0 >= 0) {
+          uint16_t* pv = reinterpret_cast<uint16_t*>(item + (((t.lw0 >> 3) ^ swz) * 16) + (t.lw0 & 7) * 2);
+          const uint16_t v = loaded ? *pv : (uint16_t)0;
+          if (loaded) *pv = 0;
+          if (live) p.B[(size_t)row * p.K_L + t.pos0] = v;
+        }
+        if (G == 16 && t.lw1 >= 0) {
+          uint16_t* pv = reinterpret_cast<uint16_t*>(item + (((t.lw1 >> 3) ^ swz) * 16) + (t.lw1 & 7) * 2);
+          const uint16_t v = loaded ? *pv : (uint16_t)0;
+          if (loaded) *pv = 0;
+          if (live) p.B[(size_t)row * p.K_L + t.pos1] = v;
+        }
+        if (live && blk == 0)
+          for (int i = count; i < p.K_L; ++i) p.B[(size_t)row * p.K_L + i] = 0;
+      }
+      uint32_t w[16];
+      if (loaded && live) load_block_smem(box, r, w);
+      else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) w[j] = 0u;
+      }
+      const BlockTable none{-1, 0, -1, 0};
+      quant_block<G, FP8, false>(w, row, blk, live, none, count, p.K, p.K_L, p.B, p.Q, p.S);
+    }
   }
 }
 
@@ -307,22 +400,41 @@ __global__ void __launch_bounds__(256) quantize_grouped_kernel(GroupedQuantParam
   }
 }
 
+constexpr int QSMEM = QWARPS * 2 * QSTEP * 64 + 1024;
+
 template <int G, bool FP8, bool TABLE>
-static cudaError_t launch_quant(const QuantParams& p, int grid, cudaStream_t s) {
-  quantize_kernel<G, FP8, TABLE><<<grid, 256, 0, s>>>(p);
+static cudaError_t launch_quant(const CUtensorMap& tmX, const QuantParams& p, int grid, cudaStream_t s) {
+  static int attr_done[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(quantize_tma_kernel<G, FP8, TABLE>, cudaFuncAttributeMaxDynamicSharedMemorySize, QSMEM);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = 1;
+  }
+  quantize_tma_kernel<G, FP8, TABLE><<<grid, 256, QSMEM, s>>>(tmX, p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_quantize(const QuantParams& p, bool fp8, int num_sms, cudaStream_t s) {
-  const long long items = (long long)((p.M + 127) / 128 * 128) * (p.K / 32);
-  const int grid = (int)std::max<long long>(1, std::min<long long>((items + 511) / 512, (long long)num_sms * 6));
+cudaError_t launch_quantize(const CUtensorMap& tmX, const QuantParams& p, bool fp8, int num_sms, cudaStream_t s) {
+  // warp steps are spread so that the busiest warp does as few steps more than the average
+  // as possible (1..3 CTAs per SM; more resident warps break ties)
+  const long long steps = (long long)((p.M + 127) / 128 * 128) * (p.K / 32) / QSTEP;
+  int grid = 1;
+  double best = -1.0;
+  for (int k = 1; k <= 3; ++k) {
+    const long long ctas = std::max<long long>(1, std::min<long long>((steps + QWARPS - 1) / QWARPS, (long long)num_sms * k));
+    const long long warps = ctas * QWARPS;
+    const double eff = (double)steps / (double)(warps * ((steps + warps - 1) / warps));
+    if (eff >= best - 1e-9) { best = eff; grid = (int)ctas; }
+  }
   const bool table = p.L != nullptr;
   if (table && p.Kg > MAX_KG) return cudaErrorInvalidValue;
-  if (fp8) return launch_quant<32, true, false>(p, grid, s);
+  if (fp8) return launch_quant<32, true, false>(tmX, p, grid, s);
   switch (p.G) {
-    case 16: return table ? launch_quant<16, false, true>(p, grid, s) : launch_quant<16, false, false>(p, grid, s);
-    case 32: return table ? launch_quant<32, false, true>(p, grid, s) : launch_quant<32, false, false>(p, grid, s);
-    case 64: return table ? launch_quant<64, false, true>(p, grid, s) : launch_quant<64, false, false>(p, grid, s);
+    case 16: return table ? launch_quant<16, false, true>(tmX, p, grid, s) : launch_quant<16, false, false>(tmX, p, grid, s);
+    case 32: return table ? launch_quant<32, false, true>(tmX, p, grid, s) : launch_quant<32, false, false>(tmX, p, grid, s);
+    case 64: return table ? launch_quant<64, false, true>(tmX, p, grid, s) : launch_quant<64, false, false>(tmX, p, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
