@@ -91,7 +91,7 @@ inline bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) =
 // 64-byte rows, box {32, 64}, 64-byte swizzle.
 int make_block_map(CUtensorMap* m, const uint16_t* X, int rows, int K) {
   uint64_t d[2] = {32, (uint64_t)rows * (uint64_t)(K / 32)}, st[1] = {64};
-  uint32_t box[2] = {32, 64};
+  uint32_t box[2] = {32, (uint32_t)osc::QUANT_STEP_ITEMS};
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, d, st, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 inline bool valid_g(int G) { return G == 16 || G == 32 || G == 64; }
@@ -117,7 +117,9 @@ int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
   if (bn == 0) bn = (N >= 256 && (long long)((M + 127) / 128) * ((N + 255) / 256) >= ds->sms) ? 256 : 128;
   // the CTA pair needs 256-wide tiles, whole 256-row tiles of work and a per-128-row expert map
   // it cannot honour, so grouped calls stay on single CTAs
-  if (cg < 0) cg = 1;   // measured: single-CTA 128x256 tiles beat the pair on every shape tried so far
+  // measured on the B200: the 2-CTA pair wins once there are at least two 256x256 tiles per
+  // pair of SMs (FFN 4096x24576x4096: 4.58 vs 4.40 PFLOP/s); below that they tie or it loses
+  if (cg < 0) cg = (bn == 256 && !grouped && (long long)((M + 255) / 256) * ((N + 255) / 256) >= 2LL * ds->sms) ? 2 : 1;
   if (cg == 2 && (bn != 256 || grouped)) cg = 1;
   const int m_tiles = (M + 128 * cg - 1) / (128 * cg);
 

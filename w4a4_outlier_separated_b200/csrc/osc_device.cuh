@@ -276,6 +276,13 @@ template <int CG> __device__ __forceinline__ void tc_commit_to(uint32_t bar) {
                  :: "r"(bar), "h"(mask) : "memory");
   }
 }
+// Commit that arrives only on this CTA's barrier (no multicast), for either CTA group.
+template <int CG> __device__ __forceinline__ void tc_commit_local(uint32_t bar) {
+  if constexpr (CG == 1)
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
+  else
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
+}
 template <int CG> __device__ __forceinline__ void tc_cp_atom(uint32_t taddr, uint64_t sdesc) {
   if constexpr (CG == 1) asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
   else asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");

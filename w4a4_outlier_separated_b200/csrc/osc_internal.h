@@ -18,7 +18,11 @@ struct QuantParams {
   int* status;
 };
 
-// tmX: X as (32-channel blocks) x 64 bytes, box {32, 64} bf16, 64-byte swizzle (see make_block_map)
+// Items (32-channel blocks) per warp step of the quantize kernels = height of the TMA box
+// the host encodes for X.
+constexpr int QUANT_STEP_ITEMS = 64;
+// tmX: X as (32-channel blocks) x 64 bytes, box {32, QUANT_STEP_ITEMS}, 64-byte swizzle
+// (see make_block_map)
 cudaError_t launch_quantize(const CUtensorMap& tmX, const QuantParams& p, bool fp8, int num_sms, cudaStream_t s);
 
 struct GroupedQuantParams {

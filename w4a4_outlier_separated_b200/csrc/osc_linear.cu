@@ -13,8 +13,11 @@
 //
 // Structure: persistent CTAs (one per SM), 8 warps.
 //   warp 0 (one lane)   TMA producer: operand tiles (128B swizzle) and scale atoms
-//   warp 1 (one lane)   MMA issuer: tcgen05.cp scales -> TMEM, tcgen05.mma, tcgen05.commit
+//   warp 1 (one lane)   MMA issuer: tcgen05.mma, tcgen05.commit
 //   warp 2              TMEM allocator
+//   warp 3 (one lane)   scale copier: per stage, tcgen05.cp of the stage's scale atoms into
+//                       that stage's own TMEM scale set; copies issued by a thread other than
+//                       the MMA issuer overlap the MMAs instead of queueing in front of them
 //   warps 4..11         epilogue, two warps per TMEM lane quadrant (warp % 4), each owning half
 //                       of the accumulator columns: tcgen05.ld all of them in one round trip,
 //                       release the accumulator, then bf16 -> smem -> TMA store
@@ -54,13 +57,14 @@ struct GemmCfg {
   static constexpr int SMEM_TOTAL = STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES + 1024;
   static constexpr int SFA_COLS = APS * 4;
   static constexpr int SFB_COLS = APS * (BN / 32);
-  static constexpr int ACC_STAGES = (2 * BN + SFA_COLS + SFB_COLS <= 512) ? 2 : 1;
-  static constexpr int SFA_COL = ACC_STAGES * BN;
+  static constexpr int SF_SET = SFA_COLS + SFB_COLS;                 // TMEM columns of one stage's scales
+  static constexpr int ACC_STAGES = (2 * BN + STAGES * SF_SET <= 512) ? 2 : 1;
+  static constexpr int SFA_COL = ACC_STAGES * BN;                    // scale set s starts at SFA_COL + s * SF_SET
   static constexpr int SFB_COL = SFA_COL + SFA_COLS;
   static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t MAIN_TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // per CTA and stage
   static constexpr uint32_t COMP_TX = A_BYTES + B_BYTES;
-  static_assert(SFB_COL + SFB_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(SFA_COL + STAGES * SF_SET <= TMEM_COLS, "TMEM budget");
   static_assert(STAGES >= 2, "smem budget");
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "tile width");
   static_assert(CG == 1 || (CG == 2 && BN == 256), "the CTA pair uses 256-wide tiles");
@@ -108,8 +112,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   auto accf_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + a); };
   auto acce_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 2 + a); };
   const uint32_t tear_bar = bar0 + 8u * (2 * C::STAGES + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 8 * (2 * C::STAGES + 5));
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (2 * C::STAGES + 5) + 8);
+  const uint32_t tear2_bar = bar0 + 8u * (2 * C::STAGES + 5);
+  auto sfready_bar = [&](int s) { return bar0 + 8u * (2 * C::STAGES + 6 + s); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 8 * (3 * C::STAGES + 6));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (3 * C::STAGES + 6) + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = CG == 2 ? (int)cluster_ctarank() : 0;
@@ -118,6 +124,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(accf_bar(a), 1); mbar_init(acce_bar(a), C::EPI_WARPS * CG); }
     mbar_init(tear_bar, 1);
+    mbar_init(tear2_bar, 1);
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(sfready_bar(s), 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB); tma_prefetch_desc(&tmY);
@@ -207,17 +215,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       const uint32_t d = tmem + acc * BN;
       for (int ks = 0; ks < n_k; ++ks) {
         if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, p.status))) break;
+        if (!(ok = mbar_wait(sfready_bar(stage), phase, abort_flag, p.status))) break;   // scales in TMEM
         tc_fence_after();
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
-        const uint32_t s_sfa = st + C::A_BYTES + C::B_BYTES;
-        const uint32_t s_sfb = s_sfa + C::SFA_BYTES;
-#pragma unroll
-        for (int a = 0; a < C::APS; ++a) {
-          tc_cp_atom<CG>(tmem + C::SFA_COL + 4 * a, desc_scale_atom(s_sfa + 512 * a));
-#pragma unroll
-          for (int r = 0; r < BN / 128; ++r)
-            tc_cp_atom<CG>(tmem + C::SFB_COL + a * (BN / 32) + 4 * r, desc_scale_atom(s_sfb + (r * C::APS + a) * 512));
-        }
+        const uint32_t sfo = tmem + stage * C::SF_SET;      // this stage's scale set
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const uint64_t ad = desc_kmajor_sw128(st + 32 * j);
@@ -226,13 +227,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           if constexpr (KIND == KIND_MXF4_B32) {
             const uint32_t sf = 2 * (j & 1), atom = j >> 1;
             tc_mma_mxf4_b32_g<CG>(d, ad, bd, idesc_bs_m(FMT_MXF4_E2M1, C::MMA_M, BN, sf, sf),
-                                  tmem + C::SFA_COL + 4 * atom, tmem + C::SFB_COL + atom * (BN / 32), accum);
+                                  sfo + C::SFA_COL + 4 * atom, sfo + C::SFB_COL + atom * (BN / 32), accum);
           } else if constexpr (KIND == KIND_MXF4_B16) {
             tc_mma_mxf4_b16_g<CG>(d, ad, bd, idesc_bs_m(FMT_MXF4_E2M1, C::MMA_M, BN, 0, 0),
-                                  tmem + C::SFA_COL + 4 * j, tmem + C::SFB_COL + j * (BN / 32), accum);
+                                  sfo + C::SFA_COL + 4 * j, sfo + C::SFB_COL + j * (BN / 32), accum);
           } else {
             tc_mma_mxf8_g<CG>(d, ad, bd, idesc_bs_m(FMT_F8_E4M3, C::MMA_M, BN, j, j),
-                              tmem + C::SFA_COL, tmem + C::SFB_COL, accum);
+                              sfo + C::SFA_COL, sfo + C::SFB_COL, accum);
           }
         }
         tc_commit_to<CG>(empty_bar(stage));
@@ -241,6 +242,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       const int n_c = (ti.kl + 63) / 64;
       for (int c = 0; c < n_c && ok; ++c) {
         if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, p.status))) break;
+        if (!(ok = mbar_wait(sfready_bar(stage), phase, abort_flag, p.status))) break;   // keeps phases aligned
         tc_fence_after();
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
         const int nm = min(4, (ti.kl - 64 * c) / 16);
@@ -258,6 +260,44 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       tc_commit_to<CG>(tear_bar);
       volatile int never = 0;
       mbar_wait(tear_bar, 0, &never, nullptr, 100000000ull);
+    }
+  } else if (warp == 3 && lane == 0 && leader) {
+    // ------------------------------------------------------------------ scale copier
+    // Walks the same stage sequence as the MMA issuer. A stage's scale set is free once the
+    // stage's data has landed again (the producer refills a stage only after the MMAs that
+    // read it - and its scale set - have completed).
+    int stage = 0; uint32_t phase = 0;
+    bool ok = true;
+    for (int t = unit; t < num_tiles && ok; t += nunits) {
+      const TileInfo ti = tile_info<CG>(t, p, BN, rank);
+      for (int ks = 0; ks < n_k; ++ks) {
+        if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, p.status))) break;
+        tc_fence_after();
+        const uint32_t st = sbase + stage * C::STAGE_BYTES;
+        const uint32_t s_sfa = st + C::A_BYTES + C::B_BYTES;
+        const uint32_t s_sfb = s_sfa + C::SFA_BYTES;
+        const uint32_t sfo = tmem + stage * C::SF_SET;
+#pragma unroll
+        for (int a = 0; a < C::APS; ++a) {
+          tc_cp_atom<CG>(sfo + C::SFA_COL + 4 * a, desc_scale_atom(s_sfa + 512 * a));
+#pragma unroll
+          for (int r = 0; r < BN / 128; ++r)
+            tc_cp_atom<CG>(sfo + C::SFB_COL + a * (BN / 32) + 4 * r, desc_scale_atom(s_sfb + (r * C::APS + a) * 512));
+        }
+        tc_commit_local<CG>(sfready_bar(stage));
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+      }
+      const int n_c = (ti.kl + 63) / 64;
+      for (int c = 0; c < n_c && ok; ++c) {                  // compensation stages carry no scales
+        if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, p.status))) break;
+        mbar_arrive(sfready_bar(stage));
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+    if (*abort_flag) {
+      tc_commit_local<CG>(tear2_bar);
+      volatile int never = 0;
+      mbar_wait(tear2_bar, 0, &never, nullptr, 100000000ull);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ epilogue

@@ -249,8 +249,9 @@ constexpr int MAX_KG = 1024;
 // (16-byte chunk c of item r at chunk c ^ ((r / 2) % 4)), which makes every lane's 64-byte
 // read from shared memory conflict-free; each warp double-buffers its boxes. Items in rows
 // M .. (next multiple of 128) only write zero scales.
-constexpr int QSTEP = 64;                       // items per warp step
+constexpr int QSTEP = QUANT_STEP_ITEMS;         // items per warp step (= the TMA box height)
 constexpr int QWARPS = 8;
+constexpr int QMAXK = 3;                        // CTAs per SM the shared memory allows
 
 __device__ __forceinline__ void load_block_smem(const uint8_t* slot, int r, uint32_t (&w)[16]) {
 #pragma unroll
@@ -324,7 +325,7 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
     int blka = (int)(it0 - (uint32_t)rowa * nblk) + lane;
     while (blka >= nblk) { blka -= nblk; ++rowa; }
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < QSTEP / 32; ++h) {
       const int r = lane + 32 * h;                            // item within the box
       int row = rowa, blk = blka + 32 * h;
       while (blk >= nblk) { blk -= nblk; ++row; }
@@ -352,7 +353,7 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
           for (int i = count; i < p.K_L; ++i) p.B[(size_t)row * p.K_L + i] = 0;
       }
       uint32_t w[16];
-      if (loaded && live) load_block_smem(box, r, w);
+      if (loaded) load_block_smem(box, r, w);                 // rows past M arrive zero-filled
       else {
 #pragma unroll
         for (int j = 0; j < 16; ++j) w[j] = 0u;
@@ -422,7 +423,7 @@ cudaError_t launch_quantize(const CUtensorMap& tmX, const QuantParams& p, bool f
   const long long steps = (long long)((p.M + 127) / 128 * 128) * (p.K / 32) / QSTEP;
   int grid = 1;
   double best = -1.0;
-  for (int k = 1; k <= 3; ++k) {
+  for (int k = 1; k <= QMAXK; ++k) {
     const long long ctas = std::max<long long>(1, std::min<long long>((steps + QWARPS - 1) / QWARPS, (long long)num_sms * k));
     const long long warps = ctas * QWARPS;
     const double eff = (double)steps / (double)(warps * ((steps + warps - 1) / warps));
