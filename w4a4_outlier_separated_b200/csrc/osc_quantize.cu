@@ -23,6 +23,34 @@ __device__ __forceinline__ size_t scale_word_offset(int row, int slot4, int nslo
   return ((size_t)(row >> 7) * nslot4 + slot4) * 512u + (size_t)((row & 31) * 16 + ((row >> 5) & 3) * 4);
 }
 
+// Byte offset of scale slot `slot` of a row (same layout).
+__device__ __forceinline__ size_t scale_byte_offset(int row, int slot, int nslot4) {
+  return scale_word_offset(row, slot >> 2, nslot4) + (size_t)(slot & 3);
+}
+
+// max(|a|, |b|) per bf16 half; the sign bit of the result is junk (xor of the signs).
+__device__ __forceinline__ uint32_t maxabs2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// a * b per bf16 half, round to nearest even. With b a power of two the product is exact
+// unless it falls below the normal range (|a * b| < 2^-126); such values are far below the
+// first rounding threshold of E2M1 (0.25) and E4M3 (2^-10) and keep their sign, so their
+// codes are the same as from the exact product.
+__device__ __forceinline__ uint32_t mul2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// The bf16 pair (2^-e, 2^-e) for a shared exponent e in [-127, 125].
+__device__ __forceinline__ uint32_t pow2_neg_x2(int e) {
+  const uint32_t b = (uint32_t)(127 - e) << 7;
+  return b | (b << 16);
+}
+
 // Eight E2M1 codes from eight fp32 values (already scaled by 2^-e), packed low nibble first.
 __device__ __forceinline__ uint32_t cvt_e2m1x8(float x0, float x1, float x2, float x3, float x4, float x5,
                                                float x6, float x7) {
@@ -63,18 +91,15 @@ __device__ __forceinline__ int shared_exp(uint32_t am) {
 // max of the magnitudes (finite values order like their bits), then the larger half.
 template <int J0, int NW>
 __device__ __forceinline__ uint32_t block_amax(const uint32_t (&w)[16]) {
-  uint32_t a[NW];
+  uint32_t a[NW / 2];
 #pragma unroll
-  for (int j = 0; j < NW; ++j) a[j] = w[J0 + j] & 0x7FFF7FFFu;
+  for (int j = 0; j < NW / 2; ++j) a[j] = maxabs2(w[J0 + j], w[J0 + j + NW / 2]);
 #pragma unroll
-  for (int n = NW; n > 1; n >>= 1)
+  for (int n = NW / 2; n > 1; n >>= 1)
 #pragma unroll
-    for (int j = 0; j < n / 2; ++j) {
-      __nv_bfloat162 m = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&a[j]),
-                                 *reinterpret_cast<const __nv_bfloat162*>(&a[j + n / 2]));
-      a[j] = *reinterpret_cast<const uint32_t*>(&m);
-    }
-  return max(a[0] & 0xFFFFu, a[0] >> 16);
+    for (int j = 0; j < n / 2; ++j) a[j] = maxabs2(a[j], a[j + n / 2]);
+  const uint32_t m = a[0] & 0x7FFF7FFFu;
+  return max(m & 0xFFFFu, m >> 16);
 }
 
 // Move the table channel `lw` (0..31) of the block out: return its bits, leave +0 in its slot.
@@ -91,14 +116,16 @@ __device__ __forceinline__ uint16_t take_channel(uint32_t (&w)[16], int lw) {
   return (uint16_t)(v >> sh);
 }
 
-// E2M1 codes of 16 consecutive elements (words J0..J0+7) scaled by f, as two u32 (low nibble first).
+// E2M1 codes of 16 consecutive elements (words J0..J0+7) scaled by the bf16 pair f2 =
+// (2^-e, 2^-e), as two u32 (low nibble first).
 template <int J0>
-__device__ __forceinline__ uint2 codes16(const uint32_t (&w)[16], float f) {
+__device__ __forceinline__ uint2 codes16(const uint32_t (&w)[16], uint32_t f2) {
+  uint32_t v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = mul2(w[J0 + j], f2);
   uint2 r;
-  r.x = cvt_e2m1x8(lo_f(w[J0]) * f, hi_f(w[J0]) * f, lo_f(w[J0 + 1]) * f, hi_f(w[J0 + 1]) * f,
-                   lo_f(w[J0 + 2]) * f, hi_f(w[J0 + 2]) * f, lo_f(w[J0 + 3]) * f, hi_f(w[J0 + 3]) * f);
-  r.y = cvt_e2m1x8(lo_f(w[J0 + 4]) * f, hi_f(w[J0 + 4]) * f, lo_f(w[J0 + 5]) * f, hi_f(w[J0 + 5]) * f,
-                   lo_f(w[J0 + 6]) * f, hi_f(w[J0 + 6]) * f, lo_f(w[J0 + 7]) * f, hi_f(w[J0 + 7]) * f);
+  r.x = cvt_e2m1x8(lo_f(v[0]), hi_f(v[0]), lo_f(v[1]), hi_f(v[1]), lo_f(v[2]), hi_f(v[2]), lo_f(v[3]), hi_f(v[3]));
+  r.y = cvt_e2m1x8(lo_f(v[4]), hi_f(v[4]), lo_f(v[5]), hi_f(v[5]), lo_f(v[6]), hi_f(v[6]), lo_f(v[7]), hi_f(v[7]));
   return r;
 }
 
@@ -126,11 +153,31 @@ __device__ __forceinline__ BlockTable block_table(int blk, const int8_t* Ls, con
   return t;
 }
 
-// Stage one table (Kg entries) in shared memory with each entry's B column; returns the
-// number of entries (at most K_L). Entries >= G or beyond K_L columns are reported and dropped.
+// Table entry and B column of one group packed in one word: (column << 8) | (entry & 0xFF),
+// entry -1 (0xFF) meaning none.
 template <int G>
-__device__ int stage_table(const int8_t* __restrict__ L, int Kg, int K_L, int8_t* Ls, int16_t* Ps, int* s_warp,
-                           int* status) {
+__device__ __forceinline__ BlockTable block_table_packed(int blk, const int* tab) {
+  BlockTable t{-1, 0, -1, 0};
+  if constexpr (G == 32) {
+    const int v = tab[blk], l = (int)(int8_t)(v & 0xFF);
+    if (l >= 0) { t.lw0 = l; t.pos0 = v >> 8; }
+  } else if constexpr (G == 64) {
+    const int v = tab[blk >> 1], l = (int)(int8_t)(v & 0xFF);
+    if (l >= 0 && (l >> 5) == (blk & 1)) { t.lw0 = l & 31; t.pos0 = v >> 8; }
+  } else {
+    const int2 v = *reinterpret_cast<const int2*>(tab + 2 * blk);
+    const int l0 = (int)(int8_t)(v.x & 0xFF), l1 = (int)(int8_t)(v.y & 0xFF);
+    if (l0 >= 0) { t.lw0 = l0; t.pos0 = v.x >> 8; }
+    if (l1 >= 0) { t.lw1 = 16 + l1; t.pos1 = v.y >> 8; }
+  }
+  return t;
+}
+
+// Stage one table (Kg entries) in shared memory, packed with each entry's B column; returns
+// the number of entries (at most K_L). Entries >= G or beyond K_L columns are reported and
+// dropped.
+template <int G>
+__device__ int stage_table(const int8_t* __restrict__ L, int Kg, int K_L, int* tab, int* s_warp, int* status) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int per = (Kg + 255) / 256;
   const int i0 = threadIdx.x * per, i1 = min(Kg, i0 + per);
@@ -138,7 +185,7 @@ __device__ int stage_table(const int8_t* __restrict__ L, int Kg, int K_L, int8_t
   for (int i = i0; i < i1; ++i) {
     int v = L[i];
     if (v >= G) { record_status(status, DEV_BAD_TABLE); v = -1; }
-    Ls[i] = (int8_t)v;
+    tab[i] = v;
     local += v >= 0;
   }
   int incl = local;
@@ -151,18 +198,20 @@ __device__ int stage_table(const int8_t* __restrict__ L, int Kg, int K_L, int8_t
   __syncthreads();
   int run = incl - local, count = 0;
   for (int w = 0; w < 8; ++w) { if (w < warp) run += s_warp[w]; count += s_warp[w]; }
-  for (int i = i0; i < i1; ++i)
-    if (Ls[i] >= 0) {
-      if (run >= K_L) { record_status(status, DEV_BAD_TABLE); Ls[i] = -1; }
-      Ps[i] = (int16_t)run++;
-    }
+  for (int i = i0; i < i1; ++i) {
+    const int v = tab[i];
+    if (v < 0) { tab[i] = 0xFF; continue; }
+    if (run >= K_L) { record_status(status, DEV_BAD_TABLE); tab[i] = 0xFF; }
+    else tab[i] = (run << 8) | v;
+    ++run;
+  }
   __syncthreads();
   return min(count, K_L);
 }
 
 // One item = one 32-channel block of one row: extraction, amax, exponent(s), codes, scales.
-// All 32 lanes of a warp call it together (the scale words and G = 64 amax use shuffles);
-// lanes hold consecutive blocks of the same row (K is a multiple of 256).
+// All 32 lanes of a warp call it together (for G = 64 the two blocks of a group sit on
+// neighbouring lanes and meet by a shuffle); lanes hold consecutive blocks of a row.
 template <int G, bool FP8, bool TABLE>
 __device__ __forceinline__ void quant_block(uint32_t (&w)[16], int row, int blk, bool live, const BlockTable& t,
                                             int count, int K, int K_L, uint16_t* __restrict__ B,
@@ -183,46 +232,37 @@ __device__ __forceinline__ void quant_block(uint32_t (&w)[16], int row, int blk,
   const int nblk = K / 32;
   if constexpr (FP8) {
     const int e = shared_exp<8>(block_amax<0, 16>(w));
-    const float f = __uint_as_float((uint32_t)(127 - e) << 23);
+    const uint32_t f2 = pow2_neg_x2(e);
     uint32_t c[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      c[j] = cvt_e4m3x4(lo_f(w[2 * j]) * f, hi_f(w[2 * j]) * f, lo_f(w[2 * j + 1]) * f, hi_f(w[2 * j + 1]) * f);
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t v0 = mul2(w[2 * j], f2), v1 = mul2(w[2 * j + 1], f2);
+      c[j] = cvt_e4m3x4(lo_f(v0), hi_f(v0), lo_f(v1), hi_f(v1));
+    }
     if (live) {
       uint4* dst = reinterpret_cast<uint4*>(Q + (size_t)row * K + (size_t)blk * 32);
       dst[0] = make_uint4(c[0], c[1], c[2], c[3]);
       dst[1] = make_uint4(c[4], c[5], c[6], c[7]);
     }
-    const uint32_t code = (uint32_t)(e + 127);
-    const uint32_t c1 = __shfl_down_sync(0xffffffffu, code, 1);
-    const uint32_t c2 = __shfl_down_sync(0xffffffffu, code, 2);
-    const uint32_t c3 = __shfl_down_sync(0xffffffffu, code, 3);
-    if ((blk & 3) == 0)
-      *reinterpret_cast<uint32_t*>(S + scale_word_offset(row, blk >> 2, nblk / 4)) = code | (c1 << 8) | (c2 << 16) | (c3 << 24);
+    S[scale_byte_offset(row, blk, nblk / 4)] = (uint8_t)(e + 127);
   } else if constexpr (G == 16) {
     const int e0 = shared_exp<2>(block_amax<0, 8>(w));
     const int e1 = shared_exp<2>(block_amax<8, 8>(w));
-    const uint2 q0 = codes16<0>(w, __uint_as_float((uint32_t)(127 - e0) << 23));
-    const uint2 q1 = codes16<8>(w, __uint_as_float((uint32_t)(127 - e1) << 23));
+    const uint2 q0 = codes16<0>(w, pow2_neg_x2(e0));
+    const uint2 q1 = codes16<8>(w, pow2_neg_x2(e1));
     if (live) *reinterpret_cast<uint4*>(Q + (size_t)row * (K / 2) + (size_t)blk * 16) = make_uint4(q0.x, q0.y, q1.x, q1.y);
-    const uint32_t pair = (uint32_t)(e0 + 127) | ((uint32_t)(e1 + 127) << 8);   // slots 2*blk, 2*blk+1
-    const uint32_t nxt = __shfl_down_sync(0xffffffffu, pair, 1);
-    if ((blk & 1) == 0)
-      *reinterpret_cast<uint32_t*>(S + scale_word_offset(row, blk >> 1, nblk / 2)) = pair | (nxt << 16);
+    // slots 2*blk and 2*blk + 1: two neighbouring bytes of one scale word
+    *reinterpret_cast<uint16_t*>(S + scale_byte_offset(row, 2 * blk, nblk / 2)) =
+        (uint16_t)((uint32_t)(e0 + 127) | ((uint32_t)(e1 + 127) << 8));
   } else {
     uint32_t am = block_amax<0, 16>(w);
     if constexpr (G == 64) am = max(am, __shfl_xor_sync(0xffffffffu, am, 1));
     const int e = shared_exp<2>(am);
-    const float f = __uint_as_float((uint32_t)(127 - e) << 23);
-    const uint2 q0 = codes16<0>(w, f);
-    const uint2 q1 = codes16<8>(w, f);
+    const uint32_t f2 = pow2_neg_x2(e);
+    const uint2 q0 = codes16<0>(w, f2);
+    const uint2 q1 = codes16<8>(w, f2);
     if (live) *reinterpret_cast<uint4*>(Q + (size_t)row * (K / 2) + (size_t)blk * 16) = make_uint4(q0.x, q0.y, q1.x, q1.y);
-    const uint32_t code = (uint32_t)(e + 127);
-    const uint32_t c1 = __shfl_down_sync(0xffffffffu, code, 1);
-    const uint32_t c2 = __shfl_down_sync(0xffffffffu, code, 2);
-    const uint32_t c3 = __shfl_down_sync(0xffffffffu, code, 3);
-    if ((blk & 3) == 0)
-      *reinterpret_cast<uint32_t*>(S + scale_word_offset(row, blk >> 2, nblk / 4)) = code | (c1 << 8) | (c2 << 16) | (c3 << 24);
+    S[scale_byte_offset(row, blk, nblk / 4)] = (uint8_t)(e + 127);
   }
   (void)lane;
 }
@@ -267,8 +307,7 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
   uint8_t* boxes = q_dyn + ((1024u - (smem_u32(q_dyn) & 1023u)) & 1023u);
   auto box_at = [&](int wp, int sl) { return boxes + (wp * 2 + sl) * (QSTEP * 64); };
   __shared__ __align__(8) uint64_t s_bar[QWARPS][2];
-  __shared__ int8_t s_l[TABLE ? MAX_KG : 1];
-  __shared__ int16_t s_pos[TABLE ? MAX_KG : 1];
+  __shared__ __align__(8) int s_tab[TABLE ? MAX_KG : 2];
   __shared__ int s_warp[8];
   __shared__ int s_abort;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -293,9 +332,9 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
   };
   if (step < nsteps) issue(step, 0);
   int count = 0;
-  if constexpr (TABLE) count = stage_table<G>(p.L, p.Kg, p.K_L, s_l, s_pos, s_warp, p.status);
+  if constexpr (TABLE) count = stage_table<G>(p.L, p.Kg, p.K_L, s_tab, s_warp, p.status);
   else __syncthreads();
-  uint32_t ph[2] = {0u, 0u};
+  uint32_t phbits = 0;                                        // bit s: parity of slot s's next phase
   int slot = 0;
   for (; step < nsteps; step += wstride, slot ^= 1) {
     __syncwarp();                                             // the other slot's reads are done
@@ -305,18 +344,18 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
       // lane 0 waits (bounded) and the warp follows its verdict; __syncwarp then orders the
       // other lanes' shared-memory reads after the completed load
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(smem_u32(&s_bar[warp][slot]), ph[slot], reinterpret_cast<volatile int*>(&s_abort), p.status);
+      if (lane == 0) ok = mbar_wait(smem_u32(&s_bar[warp][slot]), (phbits >> slot) & 1u, reinterpret_cast<volatile int*>(&s_abort), p.status);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       __syncwarp();
       if (!ok) {
         // let the other slot's load (if one was issued) land before leaving
         if (lane == 0 && step + wstride < nsteps && (step + wstride) * QSTEP < real_items) {
           volatile int never = 0;
-          mbar_wait(smem_u32(&s_bar[warp][slot ^ 1]), ph[slot ^ 1], &never, nullptr, 100000000ull);
+          mbar_wait(smem_u32(&s_bar[warp][slot ^ 1]), (phbits >> (slot ^ 1)) & 1u, &never, nullptr, 100000000ull);
         }
         break;
       }
-      ph[slot] ^= 1;
+      phbits ^= 1u << slot;
     }
     uint8_t* box = box_at(warp, slot);
     // rows and blocks of this lane's two items (one division per step, then carries)
@@ -334,7 +373,7 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
       const int swz = (r >> 1) & 3;
       BlockTable t{-1, 0, -1, 0};
       if constexpr (TABLE) {
-        t = block_table<G>(blk, s_l, s_pos);
+        t = block_table_packed<G>(blk, s_tab);
         // move the table channel(s) out of the box: its 2 bytes sit in 16-byte chunk
         // (lw / 8) ^ swz at byte (lw % 8) * 2
         if (t.lw0 >= 0) {
