@@ -85,6 +85,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// ---- programmatic dependent launch -----------------------------------------------------------
+// The library's kernels are launched with programmatic stream serialization: a kernel may start
+// while the previous kernel of the stream is still running, so every thread runs
+// grid_dep_wait() before it reads or writes memory that kernel may touch; grid_dep_launch()
+// lets the next kernel of the stream be scheduled early (its CTAs start as SMs free up and
+// then wait in their own grid_dep_wait()).
+
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- TMA and bulk copies ------------------------------------------------------------------
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {

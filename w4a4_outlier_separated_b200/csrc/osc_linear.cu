@@ -138,6 +138,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   if constexpr (CG == 2) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();                       // the previous kernel's writes (Q_X, S_X, B) are visible
+  if (threadIdx.x == 0) grid_dep_launch();
 
   const int num_tiles = p.m_tiles * p.n_tiles;
   const int n_k = p.K / C::ELEMS;
@@ -401,13 +403,15 @@ static cudaError_t launch_one(const GemmMaps& m, const GemmParams& p, int grid, 
   cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_TOTAL;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CG;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, gemm_kernel<BN, KIND, CG>, m.a, m.b, m.sfa, m.sfb, m.ca, m.cb, m.y, p);
 }
 

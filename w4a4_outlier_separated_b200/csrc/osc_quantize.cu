@@ -322,6 +322,10 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
   if (lane == 0) { mbar_init(smem_u32(&s_bar[warp][0]), 1); mbar_init(smem_u32(&s_bar[warp][1]), 1); }
   fence_barrier_init();
   __syncwarp();
+  // X, L and the outputs are free of the previous kernel. No early trigger for the next one:
+  // quantize CTAs are small enough to share SMs, so an early-launched next grid would hold SM
+  // slots while it waits; the next kernel is released when this grid completes.
+  grid_dep_wait();
   // the first box goes out before the table is staged, so the two latencies overlap
   auto issue = [&](uint32_t st, int slot) {
     if (lane == 0 && st * QSTEP < real_items) {
@@ -452,8 +456,17 @@ static cudaError_t launch_quant(const CUtensorMap& tmX, const QuantParams& p, in
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
   }
-  quantize_tma_kernel<G, FP8, TABLE><<<grid, 256, QSMEM, s>>>(tmX, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = QSMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_tma_kernel<G, FP8, TABLE>, tmX, p);
 }
 
 cudaError_t launch_quantize(const CUtensorMap& tmX, const QuantParams& p, bool fp8, int num_sms, cudaStream_t s) {
