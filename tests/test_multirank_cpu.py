@@ -1,0 +1,92 @@
+"""Multi-rank host logic of bench.py on the CPU: two `gloo` ranks (world size 2) take the
+element-wise max of their timings, every rank sees the same result, the whole-job throughput is
+the weak-scaling sum, and under a launcher only rank 0 runs the reference arm."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+WORKER = r"""
+import datetime, json, os, sys
+sys.path.insert(0, os.environ["OSC_ROOT"])
+import torch.distributed as dist
+import bench
+ws, rank, local = bench.dist_env()
+dist.init_process_group("gloo", rank=rank, world_size=ws, timeout=datetime.timedelta(seconds=60))
+mine = [1.0 + rank, 10.0 - rank, 5.0 + 0.5 * rank]
+out = bench.max_over_ranks(mine, "cpu")
+dist.barrier()
+dist.destroy_process_group()
+print(json.dumps({"rank": rank, "local": local, "ws": ws, "out": out}))
+"""
+
+
+def _free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _launch(ws: int, code: str, extra_env=None):
+    port = _free_port()
+    procs = []
+    for r in range(ws):
+        env = dict(os.environ, MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(r), LOCAL_RANK=str(r),
+                   WORLD_SIZE=str(ws), OSC_ROOT=ROOT, CUDA_VISIBLE_DEVICES="")
+        env.update(extra_env or {})
+        procs.append(subprocess.Popen([sys.executable, "-c", code], env=env, stdout=subprocess.PIPE,
+                                      stderr=subprocess.PIPE, text=True))
+    outs = []
+    for p in procs:
+        try:
+            o, e = p.communicate(timeout=180)
+        except subprocess.TimeoutExpired:
+            for q in procs:
+                q.kill()
+            pytest.fail("a rank did not finish")
+        assert p.returncode == 0, e[-2000:]
+        outs.append(o)
+    return outs
+
+
+def test_max_over_ranks_gloo_world2():
+    outs = _launch(2, WORKER)
+    res = sorted((json.loads(o.strip().splitlines()[-1]) for o in outs), key=lambda d: d["rank"])
+    assert [d["rank"] for d in res] == [0, 1] and all(d["ws"] == 2 for d in res)
+    assert [d["local"] for d in res] == [0, 1]
+    for d in res:
+        assert d["out"] == [2.0, 10.0, 5.5]          # element-wise max, identical on every rank
+
+
+def test_single_process_passthrough_and_weak_scaling():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks([3.0, 4.5], "cpu") == [3.0, 4.5]
+    flops = 2.0 * 2048 * 6144 * 4096
+    one = bench.weak_scaling_tflops(1, flops, 0.040)
+    assert abs(one - flops / 40e-6 / 1e12) < 1e-9
+    # N ranks, each with its own batch in the same (max) time: N times the work per second
+    assert abs(bench.weak_scaling_tflops(4, flops, 0.040) - 4 * one) < 1e-9
+
+
+REF_WORKER = r"""
+import os, sys
+sys.path.insert(0, os.environ["OSC_ROOT"])
+import bench
+args = type("A", (), {"steps": 1, "warmup": 0, "gpus": 2})()
+res = bench.run_reference(args)
+print("NONE" if res is None else "LINE")
+"""
+
+
+def test_reference_arm_runs_on_rank0_only():
+    """Under a launcher the oracle arm runs on rank 0; other ranks return without work."""
+    env = dict(os.environ, RANK="1", LOCAL_RANK="1", WORLD_SIZE="2", OSC_ROOT=ROOT, CUDA_VISIBLE_DEVICES="")
+    out = subprocess.run([sys.executable, "-c", REF_WORKER], env=env, capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert out.stdout.strip().splitlines()[-1] == "NONE"
