@@ -14,9 +14,9 @@
 // Structure: persistent CTAs (one per SM), 8 warps.
 //   warp 0 (one lane)   TMA producer: operand tiles (128B swizzle) and scale atoms
 //   warp 1 (one lane)   MMA issuer: tcgen05.mma, tcgen05.commit
-//   warp 2              TMEM allocator
-//   warp 3 (one lane)   scale copier: per stage, tcgen05.cp of the stage's scale atoms into
-//                       that stage's own TMEM scale set; copies issued by a thread other than
+//   warp 2              TMEM allocator, then (one lane) scale copier of odd stages
+//   warp 3 (one lane)   scale copier of even stages: tcgen05.cp of a stage's scale atoms into
+//                       that stage's own TMEM scale set; copies issued by threads other than
 //                       the MMA issuer overlap the MMAs instead of queueing in front of them
 //   warps 4..11         epilogue, two warps per TMEM lane quadrant (warp % 4), each owning half
 //                       of the accumulator columns: tcgen05.ld all of them in one round trip,
@@ -114,8 +114,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   const uint32_t tear_bar = bar0 + 8u * (2 * C::STAGES + 4);
   const uint32_t tear2_bar = bar0 + 8u * (2 * C::STAGES + 5);
   auto sfready_bar = [&](int s) { return bar0 + 8u * (2 * C::STAGES + 6 + s); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 8 * (3 * C::STAGES + 6));
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (3 * C::STAGES + 6) + 8);
+  const uint32_t tear3_bar = bar0 + 8u * (3 * C::STAGES + 6);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 8 * (3 * C::STAGES + 7));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (3 * C::STAGES + 7) + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = CG == 2 ? (int)cluster_ctarank() : 0;
@@ -125,6 +126,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     for (int a = 0; a < 2; ++a) { mbar_init(accf_bar(a), 1); mbar_init(acce_bar(a), C::EPI_WARPS * CG); }
     mbar_init(tear_bar, 1);
     mbar_init(tear2_bar, 1);
+    mbar_init(tear3_bar, 1);
     for (int s = 0; s < C::STAGES; ++s) mbar_init(sfready_bar(s), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -263,43 +265,48 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       volatile int never = 0;
       mbar_wait(tear_bar, 0, &never, nullptr, 100000000ull);
     }
-  } else if (warp == 3 && lane == 0 && leader) {
-    // ------------------------------------------------------------------ scale copier
-    // Walks the same stage sequence as the MMA issuer. A stage's scale set is free once the
-    // stage's data has landed again (the producer refills a stage only after the MMAs that
-    // read it - and its scale set - have completed).
+  } else if ((warp == 3 || warp == 2) && lane == 0 && leader) {
+    // ------------------------------------------------------------------ scale copiers
+    // Two copier threads (warps 3 and 2; warp 2 is free once TMEM is allocated) take alternate
+    // stages of the sequence the MMA issuer walks: six atom copies take about one stage of MMA
+    // time when issued beside running MMAs, so a single copier falls behind. A stage's scale
+    // set is free once the stage's data has landed again (the producer refills a stage only
+    // after the MMAs that read it - and its scale set - have completed).
+    const uint32_t mine = warp == 3 ? 0u : 1u;
     int stage = 0; uint32_t phase = 0;
+    uint32_t seq = 0;                                      // position in the stage sequence
     bool ok = true;
     for (int t = unit; t < num_tiles && ok; t += nunits) {
       const TileInfo ti = tile_info<CG>(t, p, BN, rank);
-      for (int ks = 0; ks < n_k; ++ks) {
-        if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, p.status))) break;
-        tc_fence_after();
-        const uint32_t st = sbase + stage * C::STAGE_BYTES;
-        const uint32_t s_sfa = st + C::A_BYTES + C::B_BYTES;
-        const uint32_t s_sfb = s_sfa + C::SFA_BYTES;
-        const uint32_t sfo = tmem + stage * C::SF_SET;
-#pragma unroll
-        for (int a = 0; a < C::APS; ++a) {
-          tc_cp_atom<CG>(sfo + C::SFA_COL + 4 * a, desc_scale_atom(s_sfa + 512 * a));
-#pragma unroll
-          for (int r = 0; r < BN / 128; ++r)
-            tc_cp_atom<CG>(sfo + C::SFB_COL + a * (BN / 32) + 4 * r, desc_scale_atom(s_sfb + (r * C::APS + a) * 512));
-        }
-        tc_commit_local<CG>(sfready_bar(stage));
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
-      }
       const int n_c = (ti.kl + 63) / 64;
-      for (int c = 0; c < n_c && ok; ++c) {                  // compensation stages carry no scales
-        if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, p.status))) break;
-        mbar_arrive(sfready_bar(stage));
+      for (int i = 0; i < n_k + n_c; ++i, ++seq) {
+        if ((seq & 1u) == mine) {
+          if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, p.status))) break;
+          if (i < n_k) {
+            tc_fence_after();
+            const uint32_t s_sfa = sbase + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
+            const uint32_t s_sfb = s_sfa + C::SFA_BYTES;
+            const uint32_t sfo = tmem + stage * C::SF_SET;
+#pragma unroll
+            for (int a = 0; a < C::APS; ++a) {
+              tc_cp_atom<CG>(sfo + C::SFA_COL + 4 * a, desc_scale_atom(s_sfa + 512 * a));
+#pragma unroll
+              for (int r = 0; r < BN / 128; ++r)
+                tc_cp_atom<CG>(sfo + C::SFB_COL + a * (BN / 32) + 4 * r, desc_scale_atom(s_sfb + (r * C::APS + a) * 512));
+            }
+            tc_commit_local<CG>(sfready_bar(stage));
+          } else {
+            mbar_arrive(sfready_bar(stage));               // compensation stages carry no scales
+          }
+        }
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
     }
     if (*abort_flag) {
-      tc_commit_local<CG>(tear2_bar);
+      const uint32_t tb = warp == 3 ? tear2_bar : tear3_bar;
+      tc_commit_local<CG>(tb);
       volatile int never = 0;
-      mbar_wait(tear2_bar, 0, &never, nullptr, 100000000ull);
+      mbar_wait(tb, 0, &never, nullptr, 100000000ull);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ epilogue
