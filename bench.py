@@ -5,9 +5,9 @@ N=6144, G=32, table from Algorithm 1 (alpha=5) on 3x512 calibration tokens; synt
 inputs with the outlier structure of the OSC page (its Qwen3 activations are not available).
 One step = osc_quantize(X) + osc_linear over one batch with the weights prepared offline.
 The metric counts the useful 2*M*N*K flops per step (the compensation flops are reported
-apart). The K timed steps run as one CUDA graph and rotate over 4 input sets (each with its
-own copy of the prepared weights, ~245 MB in all, twice the L2), so no step finds its inputs
-in L2; per-kernel durations (for the roofline) come from graphs of K launches of one kernel.
+apart). The K timed steps run as one CUDA graph and rotate over 8 input sets (each with its
+own copy of the prepared weights, ~490 MB in all), so no step finds its inputs in L2;
+per-kernel durations (for the roofline) come from graphs of K launches of one kernel.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl osc|reference]
 
@@ -187,9 +187,10 @@ def run_osc(args):
     stream = torch.cuda.current_stream()
 
     # R rotating input sets, each with its own copy of the prepared weights, so that the sets
-    # together (~245 MB) exceed the 126 MB L2: a step never finds its inputs in L2 from the
-    # previous use of its set, as with distinct layers in a forward pass
-    R = 4
+    # together (~490 MB; ~170 MB for the quantize's X and outputs alone) exceed the 126 MB L2:
+    # a launch never finds its inputs in L2 from the previous use of its set, as with distinct
+    # layers in a forward pass
+    R = 8
     sets = []
     for i in range(R):
         QX, SX, B = osc.alloc_quantize_outputs(M_, K_, G_, K_L, "cuda")
@@ -310,7 +311,7 @@ def run_osc(args):
                        "global_batch": ws * M_, "K": K_, "N": N_, "G": G_, "K_L": K_L,
                        "table": "Algorithm 1, alpha=5, min_hits=5, 1536 calibration tokens",
                        "parallelism": f"dp{ws} (token rows, no collective)",
-                       "l2": "inputs larger than L2: steps rotate over 4 input sets with their own weight copies (~245 MB)",
+                       "l2": "inputs larger than L2: launches rotate over 8 input sets with their own weight copies (~490 MB; quantize inputs+outputs alone ~170 MB)",
                        "launch": "the K timed steps replayed as one CUDA graph captured from the C-ABI calls; "
                                  "per-kernel times from graphs of K launches of each kernel alone",
                        "compute": "MXFP4 E2M1 x E2M1 block-scaled + BF16 compensation, fp32 accumulate, bf16 out"},

@@ -117,9 +117,11 @@ int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
   if (bn == 0) bn = (N >= 256 && (long long)((M + 127) / 128) * ((N + 255) / 256) >= ds->sms) ? 256 : 128;
   // the CTA pair needs 256-wide tiles, whole 256-row tiles of work and a per-128-row expert map
   // it cannot honour, so grouped calls stay on single CTAs
-  // measured on the B200: the 2-CTA pair wins once there are at least two 256x256 tiles per
-  // pair of SMs (FFN 4096x24576x4096: 4.58 vs 4.40 PFLOP/s); below that they tie or it loses
-  if (cg < 0) cg = (bn == 256 && !grouped && (long long)((M + 255) / 256) * ((N + 255) / 256) >= 2LL * ds->sms) ? 2 : 1;
+  // measured on the B200 (launches back to back, cold inputs): the 2-CTA pair is faster for
+  // every 256-wide product with more than 128 rows - QKV 2048x6144x4096 29.6 vs 30.9 us,
+  // 8192x6144x4096 94.4 vs 100.0 us, FFN 4096x24576x4096 193.4 vs 195.6 us; with 128 rows or
+  // fewer half of its 256-row tile would be empty
+  if (cg < 0) cg = (bn == 256 && !grouped && M > 128) ? 2 : 1;
   if (cg == 2 && (bn != 256 || grouped)) cg = 1;
   const int m_tiles = (M + 128 * cg - 1) / (128 * cg);
 

@@ -326,7 +326,8 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
   // quantize CTAs are small enough to share SMs, so an early-launched next grid would hold SM
   // slots while it waits; the next kernel is released when this grid completes.
   grid_dep_wait();
-  // the first box goes out before the table is staged, so the two latencies overlap
+  // both of the warp's first boxes go out before the table is staged, so the whole first
+  // wave of loads is in flight while the table comes in
   auto issue = [&](uint32_t st, int slot) {
     if (lane == 0 && st * QSTEP < real_items) {
       const uint32_t bar = smem_u32(&s_bar[warp][slot]);
@@ -335,14 +336,13 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
     }
   };
   if (step < nsteps) issue(step, 0);
+  if (step + wstride < nsteps) issue(step + wstride, 1);
   int count = 0;
   if constexpr (TABLE) count = stage_table<G>(p.L, p.Kg, p.K_L, s_tab, s_warp, p.status);
   else __syncthreads();
   uint32_t phbits = 0;                                        // bit s: parity of slot s's next phase
   int slot = 0;
   for (; step < nsteps; step += wstride, slot ^= 1) {
-    __syncwarp();                                             // the other slot's reads are done
-    if (step + wstride < nsteps) { fence_proxy_async_smem(); issue(step + wstride, slot ^ 1); }
     const bool loaded = step * QSTEP < real_items;            // warp-uniform (pad rows are not loaded)
     if (loaded) {
       // lane 0 waits (bounded) and the warp follows its verdict; __syncwarp then orders the
@@ -404,6 +404,8 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
       const BlockTable none{-1, 0, -1, 0};
       quant_block<G, FP8, false>(w, row, blk, live, none, count, p.K, p.K_L, p.B, p.Q, p.S);
     }
+    __syncwarp();                                             // every lane is done with this slot
+    if (step + 2 * wstride < nsteps) { fence_proxy_async_smem(); issue(step + 2 * wstride, slot); }
   }
 }
 
