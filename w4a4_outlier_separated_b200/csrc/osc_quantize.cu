@@ -472,16 +472,16 @@ static cudaError_t launch_quant(const CUtensorMap& tmX, const QuantParams& p, in
 }
 
 cudaError_t launch_quantize(const CUtensorMap& tmX, const QuantParams& p, bool fp8, int num_sms, cudaStream_t s) {
-  // warp steps are spread so that the busiest warp does as few steps more than the average
-  // as possible (1..3 CTAs per SM; more resident warps break ties)
+  // 1..3 CTAs per SM: the fewest steps for the busiest warp (the critical path), and on a tie
+  // the most resident warps (more warps per scheduler hide more of each warp's latency)
   const long long steps = (long long)((p.M + 127) / 128 * 128) * (p.K / 32) / QSTEP;
   int grid = 1;
-  double best = -1.0;
+  long long best = -1;
   for (int k = 1; k <= QMAXK; ++k) {
     const long long ctas = std::max<long long>(1, std::min<long long>((steps + QWARPS - 1) / QWARPS, (long long)num_sms * k));
     const long long warps = ctas * QWARPS;
-    const double eff = (double)steps / (double)(warps * ((steps + warps - 1) / warps));
-    if (eff >= best - 1e-9) { best = eff; grid = (int)ctas; }
+    const long long busiest = (steps + warps - 1) / warps;
+    if (best < 0 || busiest <= best) { best = busiest; grid = (int)ctas; }
   }
   const bool table = p.L != nullptr;
   if (table && p.Kg > MAX_KG) return cudaErrorInvalidValue;
