@@ -316,8 +316,14 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
   const uint32_t items = mpad * (uint32_t)nblk;             // a multiple of 64
   const uint32_t real_items = (uint32_t)p.M * (uint32_t)nblk;
   const uint32_t nsteps = items / QSTEP;
-  const uint32_t wstride = gridDim.x * QWARPS;
-  uint32_t step = blockIdx.x * QWARPS + warp;
+  // CTA b takes a contiguous run of nsteps / grid steps (one more for the first nsteps % grid
+  // CTAs), so the left-over steps fall on different SMs and a CTA's loads cover one stretch of
+  // X; its warps take the run's steps round robin
+  const uint32_t wstride = QWARPS;
+  const uint32_t per = nsteps / gridDim.x, extra = nsteps % gridDim.x;
+  const uint32_t cta_first = blockIdx.x * per + min(blockIdx.x, extra);
+  const uint32_t cta_end = cta_first + per + (blockIdx.x < extra ? 1u : 0u);
+  uint32_t step = cta_first + warp;
   if (threadIdx.x == 0) s_abort = 0;
   if (lane == 0) { mbar_init(smem_u32(&s_bar[warp][0]), 1); mbar_init(smem_u32(&s_bar[warp][1]), 1); }
   fence_barrier_init();
@@ -335,14 +341,14 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
       tma_load_2d(smem_u32(box_at(warp, slot)), &tmX, 0, (int)(st * QSTEP), bar);
     }
   };
-  if (step < nsteps) issue(step, 0);
-  if (step + wstride < nsteps) issue(step + wstride, 1);
+  if (step < cta_end) issue(step, 0);
+  if (step + wstride < cta_end) issue(step + wstride, 1);
   int count = 0;
   if constexpr (TABLE) count = stage_table<G>(p.L, p.Kg, p.K_L, s_tab, s_warp, p.status);
   else __syncthreads();
   uint32_t phbits = 0;                                        // bit s: parity of slot s's next phase
   int slot = 0;
-  for (; step < nsteps; step += wstride, slot ^= 1) {
+  for (; step < cta_end; step += wstride, slot ^= 1) {
     const bool loaded = step * QSTEP < real_items;            // warp-uniform (pad rows are not loaded)
     if (loaded) {
       // lane 0 waits (bounded) and the warp follows its verdict; __syncwarp then orders the
@@ -353,7 +359,7 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
       __syncwarp();
       if (!ok) {
         // let the other slot's load (if one was issued) land before leaving
-        if (lane == 0 && step + wstride < nsteps && (step + wstride) * QSTEP < real_items) {
+        if (lane == 0 && step + wstride < cta_end && (step + wstride) * QSTEP < real_items) {
           volatile int never = 0;
           mbar_wait(smem_u32(&s_bar[warp][slot ^ 1]), (phbits >> (slot ^ 1)) & 1u, &never, nullptr, 100000000ull);
         }
@@ -405,7 +411,7 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
       quant_block<G, FP8, false>(w, row, blk, live, none, count, p.K, p.K_L, p.B, p.Q, p.S);
     }
     __syncwarp();                                             // every lane is done with this slot
-    if (step + 2 * wstride < nsteps) { fence_proxy_async_smem(); issue(step + 2 * wstride, slot); }
+    if (step + 2 * wstride < cta_end) { fence_proxy_async_smem(); issue(step + 2 * wstride, slot); }
   }
 }
 
@@ -472,15 +478,16 @@ static cudaError_t launch_quant(const CUtensorMap& tmX, const QuantParams& p, in
 }
 
 cudaError_t launch_quantize(const CUtensorMap& tmX, const QuantParams& p, bool fp8, int num_sms, cudaStream_t s) {
-  // 1..3 CTAs per SM: the fewest steps for the busiest warp (the critical path), and on a tie
-  // the most resident warps (more warps per scheduler hide more of each warp's latency)
+  // 1..3 CTAs per SM: the fewest steps for the busiest warp (the critical path; a CTA's run of
+  // ceil(steps / CTAs) steps is shared by its QWARPS warps), and on a tie the most resident warps
+  // (more warps per scheduler hide more of each warp's latency)
   const long long steps = (long long)((p.M + 127) / 128 * 128) * (p.K / 32) / QSTEP;
   int grid = 1;
   long long best = -1;
   for (int k = 1; k <= QMAXK; ++k) {
     const long long ctas = std::max<long long>(1, std::min<long long>((steps + QWARPS - 1) / QWARPS, (long long)num_sms * k));
     const long long warps = ctas * QWARPS;
-    const long long busiest = (steps + warps - 1) / warps;
+    const long long busiest = ((steps + ctas - 1) / ctas + QWARPS - 1) / QWARPS;
     if (best < 0 || busiest <= best) { best = busiest; grid = (int)ctas; }
   }
   const bool table = p.L != nullptr;
