@@ -161,8 +161,8 @@ int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
   }
   {
     uint64_t d[2] = {(uint64_t)N, (uint64_t)M}, st[1] = {(uint64_t)N * 2};
-    uint32_t box[2] = {32, 32};
-    if ((rc = make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, d, st, box, CU_TENSOR_MAP_SWIZZLE_64B))) return rc;
+    uint32_t box[2] = {16, 32};
+    if ((rc = make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, d, st, box, CU_TENSOR_MAP_SWIZZLE_32B))) return rc;
   }
   osc::GemmParams p;
   std::memset(&p, 0, sizeof(p));

@@ -49,7 +49,7 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
   static constexpr int EPI_WARPS = 8;                                // two per TMEM lane quadrant
   static constexpr int EPI_COLS = BN / 2;                            // accumulator columns per epilogue warp
-  static constexpr int STAGING_BYTES = EPI_WARPS * 32 * 64;          // one 32x32 bf16 tile per epilogue warp
+  static constexpr int STAGING_BYTES = EPI_WARPS * 32 * 32;          // one 32x16 bf16 tile per epilogue warp
   static constexpr int BAR_BYTES = 1024;
   static constexpr int SMEM_LIMIT = 232448;
   static constexpr int STAGES_FIT = (SMEM_LIMIT - STAGING_BYTES - BAR_BYTES - 1024) / STAGE_BYTES;
@@ -313,8 +313,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const int q = warp & 3;                            // TMEM lane quadrant of this warp
     const int half = (warp - 4) >> 2;                  // which half of the accumulator columns
     const int ew = warp - 4;
-    const uint32_t stg = s_staging + ew * (32 * 64);
-    uint8_t* stg_ptr = smem + C::STAGES * C::STAGE_BYTES + ew * (32 * 64);
+    const uint32_t stg = s_staging + ew * (32 * 32);
+    uint8_t* stg_ptr = smem + C::STAGES * C::STAGE_BYTES + ew * (32 * 32);
     constexpr int NCH = C::EPI_COLS / 32;              // 32-column chunks per warp (4 or 2)
     int acc = 0; uint32_t aphase = 0;
     for (int t = unit; t < num_tiles; t += nunits) {
@@ -362,18 +362,18 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 
       const bool rows_live = ti.m0 + 32 * q < p.M;
 #pragma unroll
-      for (int cc = 0; cc < NCH; ++cc) {
-        const int col = ti.n0 + c0 + cc * 32;
-        if (!rows_live || col >= p.N) continue;        // warp-uniform
+      for (int cc = 0; cc < 2 * NCH; ++cc) {           // 16-column pieces
+        const int col = ti.n0 + c0 + cc * 16;
+        if (!rows_live || col >= p.N) continue;        // warp-uniform (N is a multiple of 16)
         if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
-        // 32 rows x 64 bytes in the 64-byte swizzle the store map uses: 16-byte chunk c of
-        // row r sits at chunk c ^ ((r / 2) % 4)
+        // 32 rows x 32 bytes in the 32-byte swizzle the store map uses: 16-byte chunk c of
+        // row r sits at chunk c ^ ((r / 4) % 2)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 v = make_uint4(packed[cc * 16 + 4 * i], packed[cc * 16 + 4 * i + 1],
-                                     packed[cc * 16 + 4 * i + 2], packed[cc * 16 + 4 * i + 3]);
-          *reinterpret_cast<uint4*>(stg_ptr + lane * 64 + ((i ^ ((lane >> 1) & 3)) * 16)) = v;
+        for (int i = 0; i < 2; ++i) {
+          const uint4 v = make_uint4(packed[cc * 8 + 4 * i], packed[cc * 8 + 4 * i + 1],
+                                     packed[cc * 8 + 4 * i + 2], packed[cc * 8 + 4 * i + 3]);
+          *reinterpret_cast<uint4*>(stg_ptr + lane * 32 + ((i ^ ((lane >> 2) & 1)) * 16)) = v;
         }
         fence_proxy_async_smem();
         __syncwarp();
