@@ -486,7 +486,6 @@ cudaError_t launch_quantize(const CUtensorMap& tmX, const QuantParams& p, bool f
   long long best = -1;
   for (int k = 1; k <= QMAXK; ++k) {
     const long long ctas = std::max<long long>(1, std::min<long long>((steps + QWARPS - 1) / QWARPS, (long long)num_sms * k));
-    const long long warps = ctas * QWARPS;
     const long long busiest = ((steps + ctas - 1) / ctas + QWARPS - 1) / QWARPS;
     if (best < 0 || busiest <= best) { best = busiest; grid = (int)ctas; }
   }
