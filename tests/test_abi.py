@@ -94,3 +94,48 @@ def test_argument_checks_return_before_any_cuda_call(lib):
     assert lib.osc_set_tile_n(96) == -1
     assert lib.osc_set_tile_n(128) == 0 and lib.osc_set_tile_n(0) == 128
     _ = p
+
+
+def test_argument_limits_of_every_entry_point(lib):
+    """Each entry point rejects out-of-range or misaligned arguments with the documented code
+    before touching a device: table longer than 1024 groups, K_L above 32767, row counts whose
+    scale indexing would overflow, bad group sizes, missing buffers, unaligned K or row padding."""
+    V, I = ctypes.c_void_p, ctypes.c_int
+    buf = (ctypes.c_uint8 * 4096)()
+    p16 = V((ctypes.addressof(buf) + 15) // 16 * 16)
+    q = lib.osc_quantize
+    q.argtypes = [V, I, I, I, V, I, V, V, V, V]
+    assert q(p16, 4, 33024, 32, p16, 0, p16, p16, None, None) == -1        # K / G = 1032 > 1024 with a table
+    assert q(p16, 4, 4096, 32, p16, 32784, p16, p16, p16, None) == -1      # K_L > 32767
+    assert q(p16, 1 << 30, 256, 32, None, 0, p16, p16, None, None) == -1   # (M + 127) * K / 32 >= 2^31
+    assert q(p16, 4, 256, 32, p16, 16, p16, p16, None, None) == -1         # K_L > 0 needs B
+    assert q(p16, 0, 256, 32, None, 0, None, None, None, None) == 0        # M = 0: no-op, NULLs allowed
+    w = lib.osc_prepare_weight
+    w.argtypes = [V, I, I, I, V, I, V, V, V, V]
+    assert w(p16, 4, 256, 48, None, 0, p16, p16, None, None) == -3         # G
+    assert w(p16, 4, 256, 32, None, 16, p16, p16, p16, None) == -1         # K_L > 0 needs L
+    assert w(p16, 4, 512, 32, p16, 8, p16, p16, p16, None) == -2           # K_L % 16
+    f8 = lib.osc_quantize_fp8
+    f8.argtypes = [V, I, I, V, V, V]
+    assert f8(p16, 4, 384, p16, p16, None) == -2                           # K % 256
+    assert f8(None, 4, 256, p16, p16, None) == -1
+    lf8 = lib.osc_linear_fp8_fallback
+    lf8.argtypes = [V, V, V, V, I, I, I, V, V, V]
+    assert lf8(p16, p16, p16, p16, 4, 40, 256, p16, None, None) == -2     # N % 16
+    assert lf8(p16, p16, p16, p16, -1, 32, 256, p16, None, None) == -1    # M < 0
+    bt = lib.osc_build_table
+    bt.argtypes = [V, I, I, I, ctypes.c_float, I, V, V]
+    assert bt(p16, 8, 250, 32, 5.0, 5, p16, None) == -1                    # K % G
+    assert bt(p16, 8, 256, 8, 5.0, 5, p16, None) == -3                     # G
+    qg = lib.osc_quantize_grouped
+    qg.argtypes = [V, I, V, V, V, I, I, I, V, I, V, V, V, V]
+    assert qg(p16, 2, p16, p16, p16, 200, 256, 32, p16, 0, p16, p16, None, None) == -2   # Mp % 128
+    assert qg(p16, 2, p16, p16, p16, 256, 256, 32, None, 0, p16, p16, None, None) == -1  # tables required
+    lg = lib.osc_linear_grouped
+    lg.argtypes = [V, V, V, V, V, V, V, V, I, I, I, I, I, I, V, V, V]
+    assert lg(p16, p16, None, p16, p16, None, p16, None, 2, 200, 256, 256, 32, 0, p16, None, None) == -2  # Mp % 128
+    assert lg(p16, p16, None, p16, p16, None, None, None, 2, 256, 256, 256, 32, 0, p16, None, None) == -1  # no map
+    lib.osc_set_cta_pair.argtypes = [I]
+    assert lib.osc_set_cta_pair(3) == -1
+    prev = lib.osc_set_cta_pair(1)
+    assert lib.osc_set_cta_pair(prev) == 1
