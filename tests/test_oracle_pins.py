@@ -209,6 +209,23 @@ def test_table_tie_goes_to_lowest_channel(oracle):
     assert list(L) == [5]
     X = np.zeros((S, G))                     # all-zero group: no events
     assert list(oracle.build_table(I.bf16_bits(X), G, 5.0, 1)) == [-1]
+    X = np.full((S, G), 0.25)                # two channels share the token's maximum:
+    X[:, 9] = X[:, 4] = 50.0                 # the event goes to the lower one on every token
+    assert list(oracle.build_table(I.bf16_bits(X), G, 5.0, 5)) == [4]
+    nh, nt = oracle.density(I.bf16_bits(X), G, np.array([9], np.int8), 5.0)
+    assert nt[0] == S and nh[0] == 0
+
+
+def test_table_min_hits_boundary(oracle):
+    """A channel needs at least min_hits events: exactly min_hits qualifies, one fewer does not."""
+    S, G = 30, 32
+    X = np.full((S, 2 * G), 0.5)
+    X[:5, 0 * G + 11] = 60.0                 # group 0: 5 events
+    X[:4, 1 * G + 20] = 60.0                 # group 1: 4 events
+    Xb = I.bf16_bits(X)
+    assert list(oracle.build_table(Xb, G, alpha=5.0, min_hits=5)) == [11, -1]
+    assert list(oracle.build_table(Xb, G, alpha=5.0, min_hits=4)) == [11, 20]
+    assert list(oracle.build_table(Xb, G, alpha=5.0, min_hits=6)) == [-1, -1]
 
 
 def test_event_threshold_closed_form(oracle):
@@ -220,6 +237,13 @@ def test_event_threshold_closed_form(oracle):
         X[:, 4] = a
         nh, nt = oracle.density(I.bf16_bits(X), G, np.array([4], np.int8), alpha)
         assert nt[0] == 6 * expect and nh[0] == nt[0], (a, thr)
+    # exact equality is an event ("at least alpha times the mean"): [155, 27 x 31] gives
+    # 32 * 155 = 4960 = 5 * (155 + 31 * 27), every term exact in bf16 and in the fp32 sum
+    for a, b, expect in [(155.0, 27.0, 1), (154.0, 27.0, 0)]:
+        X = np.full((6, G), b)
+        X[:, 4] = a
+        nh, nt = oracle.density(I.bf16_bits(X), G, np.array([4], np.int8), alpha)
+        assert nt[0] == 6 * expect, (a, b)
     # alpha + 1 raises the threshold: a = 6 stops being an event at alpha = 6 (thr = 7.15)
     X = np.ones((6, G)); X[:, 4] = 6.0
     assert oracle.density(I.bf16_bits(X), G, np.array([4], np.int8), 6.0)[1][0] == 0
@@ -308,6 +332,27 @@ def test_linear_equals_matmul_of_dequantized(oracle):
     assert np.array_equal(r2["Y"], r["Y"][rows])
 
 
+@pytest.mark.parametrize("G", [16, 64])
+def test_linear_equals_matmul_of_dequantized_group_sizes(oracle, G):
+    """The same identity with 16-wide scale slots (G = 16) and 64-groups sharing one exponent
+    over two 32-slots (G = 64), on activations with fixed outlier channels."""
+    st = I.make_structure(1024, 0.7, seed=21)
+    X = I.gen_tokens(st, 12, seed=22)
+    W = I.bf16_bits(np.random.default_rng(23).standard_normal((24, 1024)) * 0.02)
+    L = I.planted_table(st, G)
+    K_L = I.pad16(oracle.table_count(L))
+    cw, ew, WL = oracle.osc_prepare_weight(W, G, L, K_L)
+    r = oracle.osc_forward(X, G, L, K_L, cw, ew, WL)
+    assert r["ex"].shape == (12, 1024 // (16 if G == 16 else 32))
+    want = oracle.mx_dequantize(r["cx"], r["ex"]) @ oracle.mx_dequantize(cw, ew).T
+    want += I.bf16_to_f32(r["B"]).astype(np.float64) @ I.bf16_to_f32(WL).astype(np.float64).T
+    assert np.allclose(r["Y"], want, rtol=1e-12, atol=1e-12)
+    xf = I.bf16_to_f32(X).astype(np.float64)
+    wf = I.bf16_to_f32(W).astype(np.float64)
+    rel = np.abs(r["Y"] - xf @ wf.T).max() / np.abs(xf @ wf.T).max()
+    assert rel < 0.25                                        # a 4-bit product, not a wrong one
+
+
 def _representable(rng, rows, K, V=32, e_range=(-8, 3)):
     """Rows whose every V-block is exactly an E2M1 grid times 2^e, with the block max at 4 or 6."""
     grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
@@ -351,6 +396,22 @@ def test_all_minus_one_table_is_mxfp4_direct(oracle):
     cx, ex = oracle.mx_quantize(c.X, 32)
     direct = oracle.mx_dequantize(cx, ex) @ oracle.mx_dequantize(cw, ew).T
     assert np.allclose(r["Y"], direct, rtol=1e-12, atol=1e-12)
+
+
+def test_weight_codes_do_not_depend_on_table(oracle):
+    """Weight side (§3.3): W is microscaled along K as it is; the table only selects the W_L
+    columns. So Q_W and S_W are those of the empty table, and the table's weight columns keep
+    their codes (they meet zeroed activation codes in the base product)."""
+    rng = np.random.default_rng(13)
+    W = I.bf16_bits(rng.standard_normal((20, 256)) * 0.02)
+    W[:, 2 * 32 + 0] = I.bf16_bits(np.full(20, 0.5))           # a weight column that sets its
+    L = np.array([-1, 3, 0, -1, 31, -1, -1, 9], np.int8)       # block's scale, in the table
+    cw, ew, WL = oracle.osc_prepare_weight(W, 32, L, 16)
+    cw0, ew0, _ = oracle.osc_prepare_weight(W, 32, np.full(8, -1, np.int8), 0)
+    assert np.array_equal(cw, cw0) and np.array_equal(ew, ew0)
+    assert np.all(cw[:, 64] == oracle.mx_quantize(W[:, 64:96], 32)[0][:, 0])
+    assert np.array_equal(WL[:, :4], W[:, [1 * 32 + 3, 2 * 32 + 0, 4 * 32 + 31, 7 * 32 + 9]])
+    assert np.all(WL[:, 4:] == 0)
 
 
 def test_fp8_fallback_exact_on_representable(oracle):
