@@ -9,7 +9,12 @@ apart). The K timed steps run as one CUDA graph and rotate over 8 input sets (ea
 own copy of the prepared weights, ~490 MB in all), so no step finds its inputs in L2;
 per-kernel durations (for the roofline) come from graphs of K launches of one kernel.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl osc|reference]
+At one GPU the line also carries "scope_rows": the other rows of the path measured the same way
+on their own workloads (FFN up/gate at G = 16/32/64, the K = 12288 down projection as OSC and
+as the MXFP8 fallback, the grouped MoE expert layers, and the MXFP8 W8A8 comparator at the QKV
+shape beside OSC at G = 16/32/64, as in the OSC page's Table 2).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl osc|reference] [--no-rows]
 
 Prints one JSON line (rank 0). Under torchrun each rank runs its own batch (weak scaling; the
 token rows shard with no data-path collective); time = max over ranks.
@@ -41,6 +46,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["osc", "reference"], default="osc")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements beside the headline")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
 
@@ -417,6 +423,254 @@ def weight_bound(wl, steps: int):
     return out
 
 
+# ---- the other rows of the hot path, each on its own workload ---------------------------------
+
+def quant_bytes(M: int, K: int, G: int, K_L: int, fp8: bool = False) -> int:
+    """Algorithmic bytes of one quantize launch: X read (bf16), codes, one E8M0 byte per scale
+    slot (16 elements for G = 16, else 32), and B (bf16, K_L columns)."""
+    if fp8:
+        return M * K * 2 + M * K + M * K // 32
+    return M * K * 2 + M * K // 2 + M * K // (16 if G == 16 else 32) + M * K_L * 2
+
+
+def _timed_graphs(fns, steps: int):
+    """Capture `steps` calls fn(0..steps-1) of each callable as one CUDA graph, replay each once
+    to warm it, then time one replay with events on the launching stream. Returns ms per call."""
+    import torch
+    gs = torch.cuda.Stream()
+    graphs = []
+    with torch.cuda.stream(gs):
+        for fn in fns:
+            fn(0)
+        gs.synchronize()
+        for fn in fns:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=gs):
+                for i in range(steps):
+                    fn(i)
+            graphs.append(g)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    out = []
+    for g in graphs:
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out.append(e0.elapsed_time(e1) / steps)
+    del graphs
+    return out
+
+
+def _to_dev(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to("cuda")
+
+
+def _status_ok():
+    from w4a4_outlier_separated_b200 import osc
+    code, raw = osc.osc_status()
+    if code != 0:
+        raise RuntimeError(f"device status {code} ({raw})")
+
+
+def _row_record(name, M, K, N, G, K_L, s_ms, q_ms, l_ms, useful_flops, qbytes, tc_peak, peaks, R):
+    return {"workload": name, "M": M, "K": K, "N": N, "G": G, "K_L": K_L, "input_sets": R,
+            "ms_per_step": round(s_ms, 5), "TFLOPs": round(useful_flops / (s_ms * 1e-3) / 1e12, 1),
+            "linear_ms": round(l_ms, 5),
+            "linear_frac": round(useful_flops / (l_ms * 1e-3) / 1e12 / tc_peak, 4),
+            "quantize_ms": round(q_ms, 5),
+            "quantize_GBps": round(qbytes / (q_ms * 1e-3) / 1e9, 1),
+            "quantize_hbm_frac": round(qbytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}
+
+
+def _osc_dense_row(name, X, W, calib, G, steps, R, peaks):
+    """OSC W4A4 on one dense layer: table by Algorithm 1 on the GPU, weights prepared offline,
+    each step osc_quantize + osc_linear over one of R rotating input sets."""
+    import torch
+    from w4a4_outlier_separated_b200 import osc
+    M, K = X.shape
+    N = W.shape[0]
+    Cd = _to_dev(calib)
+    Ld = torch.empty(K // G, dtype=torch.int8, device="cuda")
+    osc.osc_build_table(Cd, G, 5.0, 5, Ld)
+    K_L = osc.osc_table_kl(Ld.cpu().numpy())
+    Wd = _to_dev(W)
+    QW, SW, WL = osc.prepare_weight(Wd, G, Ld, K_L)
+    Xd = _to_dev(X)
+    del Wd, Cd
+    sets = []
+    for i in range(R):
+        QX, SX, B = osc.alloc_quantize_outputs(M, K, G, K_L, "cuda")
+        sets.append(dict(X=Xd if i == 0 else Xd.clone(), QW=QW if i == 0 else QW.clone(),
+                         SW=SW if i == 0 else SW.clone(), WL=(WL if i == 0 else WL.clone()) if K_L else None,
+                         QX=QX, SX=SX, B=B, Y=torch.empty((M, N), dtype=torch.bfloat16, device="cuda")))
+
+    def quant(i):
+        c = sets[i % R]
+        osc.osc_quantize(c["X"], G, Ld, K_L, c["QX"], c["SX"], c["B"])
+
+    def lin(i):
+        c = sets[i % R]
+        osc.osc_linear(c["QX"], c["SX"], c["B"], c["QW"], c["SW"], c["WL"], M, N, K, G, K_L, c["Y"])
+
+    def step(i):
+        quant(i)
+        lin(i)
+
+    for i in range(max(3, R)):
+        step(i)
+    torch.cuda.synchronize()
+    s_ms, q_ms, l_ms = _timed_graphs([step, quant, lin], steps)
+    _status_ok()
+    return _row_record(name, M, K, N, G, K_L, s_ms, q_ms, l_ms, 2.0 * M * N * K, quant_bytes(M, K, G, K_L),
+                       4.0 * peaks["bf16_tflops"], peaks, R)
+
+
+def _fp8_dense_row(name, X, W, steps, R, peaks):
+    """MXFP8 (E4M3, per-32 E8M0) on one dense layer: the fallback of the OSC page's §4, and the
+    W8A8 comparator of its Table 2. Each step osc_quantize_fp8 + osc_linear_fp8_fallback."""
+    import torch
+    from w4a4_outlier_separated_b200 import osc
+    M, K = X.shape
+    N = W.shape[0]
+    Wd = _to_dev(W)
+    QW, SW, _ = osc.alloc_quantize_outputs(N, K, 32, 0, "cuda", fp8=True)
+    osc.osc_quantize_fp8(Wd, QW, SW)
+    Xd = _to_dev(X)
+    del Wd
+    sets = []
+    for i in range(R):
+        QX, SX, _ = osc.alloc_quantize_outputs(M, K, 32, 0, "cuda", fp8=True)
+        sets.append(dict(X=Xd if i == 0 else Xd.clone(), QW=QW if i == 0 else QW.clone(),
+                         SW=SW if i == 0 else SW.clone(), QX=QX, SX=SX,
+                         Y=torch.empty((M, N), dtype=torch.bfloat16, device="cuda")))
+
+    def quant(i):
+        c = sets[i % R]
+        osc.osc_quantize_fp8(c["X"], c["QX"], c["SX"])
+
+    def lin(i):
+        c = sets[i % R]
+        osc.osc_linear_fp8_fallback(c["QX"], c["SX"], c["QW"], c["SW"], M, N, K, c["Y"])
+
+    def step(i):
+        quant(i)
+        lin(i)
+
+    for i in range(max(3, R)):
+        step(i)
+    torch.cuda.synchronize()
+    s_ms, q_ms, l_ms = _timed_graphs([step, quant, lin], steps)
+    _status_ok()
+    return _row_record(name, M, K, N, 32, 0, s_ms, q_ms, l_ms, 2.0 * M * N * K, quant_bytes(M, K, 32, 0, fp8=True),
+                       2.0 * peaks["bf16_tflops"], peaks, R)
+
+
+def _moe_row(which, steps, peaks):
+    """The grouped per-expert form (MoE expert layer, 128 experts, top-8 of 4096 tokens): tables
+    per expert by Algorithm 1 on the GPU, each step osc_quantize_grouped + osc_linear_grouped.
+    Useful flops count the routed token rows only (not the padding of each expert's last block)."""
+    import torch
+    from w4a4_outlier_separated_b200 import inputs as I
+    from w4a4_outlier_separated_b200 import osc
+    case = I.moe_case(which)
+    E, K, N, G = case.E, case.K, case.N, 32
+    Ld = torch.full((E, K // G), -1, dtype=torch.int8, device="cuda")
+    for e in range(E):
+        if case.calib[e].shape[0]:
+            osc.osc_build_table(_to_dev(case.calib[e]), G, 5.0, 5, Ld[e])
+    Lh = Ld.cpu().numpy()
+    kls = np.array([osc.osc_table_kl(Lh[e]) for e in range(E)], np.int32)
+    K_L = max(16, int(kls.max()))
+    off, poff, mbe = osc.osc_grouped_plan(case.counts)
+    Mp = int(poff[-1])
+    offd, poffd, mbed, kld = off.cuda(), poff.cuda(), mbe.cuda(), torch.from_numpy(kls).cuda()
+    QW = torch.empty((E, N, K // 2), dtype=torch.uint8, device="cuda")
+    SW = torch.empty((E, osc.osc_scale_bytes(N, K, G)), dtype=torch.uint8, device="cuda")
+    WL = torch.empty((E, N, K_L), dtype=torch.int16, device="cuda")
+    for e in range(E):
+        We = _to_dev(case.W[e])
+        osc.osc_prepare_weight(We, G, Ld[e], K_L, QW[e], SW[e], WL[e])
+    Xd = _to_dev(case.X)
+    QX = torch.empty((Mp, K // 2), dtype=torch.uint8, device="cuda")
+    SX = torch.empty(osc.osc_scale_bytes(Mp, K, G), dtype=torch.uint8, device="cuda")
+    B = torch.empty((Mp, K_L), dtype=torch.int16, device="cuda")
+    Y = torch.empty((Mp, N), dtype=torch.bfloat16, device="cuda")
+
+    def quant(i):
+        osc.osc_quantize_grouped(Xd, E, offd, poffd, mbed, Mp, G, Ld, K_L, QX, SX, B)
+
+    def lin(i):
+        osc.osc_linear_grouped(QX, SX, B, QW, SW, WL, mbed, kld, E, Mp, N, K, G, K_L, Y)
+
+    def step(i):
+        quant(i)
+        lin(i)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    s_ms, q_ms, l_ms = _timed_graphs([step, quant, lin], steps)
+    _status_ok()
+    T = int(case.counts.sum())
+    rec = _row_record(f"moe_{which} E={E} top-8 of 4096 tokens", T, K, N, G, K_L, s_ms, q_ms, l_ms, 2.0 * T * N * K,
+                      quant_bytes(T, K, G, K_L), 4.0 * peaks["bf16_tflops"], peaks, 1)
+    rec.update(padded_rows=Mp, experts_with_tokens=int((case.counts > 0).sum()),
+               largest_expert=int(case.counts.max()))
+    return rec
+
+
+def scope_rows(steps: int):
+    """Every other row of the path, measured like the headline: one graph of `steps` steps
+    replayed between events, inputs rotated so that no step finds them in L2, and per-kernel
+    graphs for the rooflines. FFN up/gate at G = 16 / 32 / 64; W2 (K = 12288) as OSC and as the
+    MXFP8 fallback; the grouped MoE expert layers; and the W8A8 comparator of the page's
+    Table 2 at the QKV shape beside OSC at G = 16 / 32 / 64 (step-time ratio)."""
+    import torch
+    from w4a4_outlier_separated_b200 import inputs as I
+    peaks, _ = measured_peaks()
+    out = {}
+
+    def run(key, fn):
+        try:
+            out[key] = fn()
+        except Exception as exc:                     # recorded, so the headline line still prints
+            out[key] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+    q = I.qkv_case(M_)
+    for G in (16, 32, 64):
+        run(f"qkv_g{G}", lambda G=G: _osc_dense_row(f"qkv_proj G={G}", q.X, q.W, q.calib, G, steps, 4, peaks))
+    run("qkv_w8a8", lambda: _fp8_dense_row("qkv_proj W8A8 (MXFP8)", q.X, q.W, steps, 4, peaks))
+    w8 = out.get("qkv_w8a8", {})
+    if "ms_per_step" in w8:
+        out["table2_osc_speedup_over_w8a8"] = {
+            f"G{G}": round(w8["ms_per_step"] / out[f"qkv_g{G}"]["ms_per_step"], 3)
+            for G in (16, 32, 64) if "ms_per_step" in out.get(f"qkv_g{G}", {})}
+    del q
+    f = I.ffn_case(32)
+    for G in (16, 32, 64):
+        run(f"ffn_g{G}", lambda G=G: _osc_dense_row(f"ffn_up M=4096 K=4096 N=24576 G={G}", f.X, f.W, f.calib, G,
+                                                    steps, 2, peaks))
+    del f
+    w = I.w2_case()
+    run("w2_osc_g32", lambda: _osc_dense_row("w2_down M=4096 K=12288 N=4096 G=32", w.X, w.W, w.calib, 32, steps, 2, peaks))
+    run("w2_fp8_fallback", lambda: _fp8_dense_row("w2_down M=4096 K=12288 N=4096 MXFP8 fallback", w.X, w.W, steps, 2,
+                                                  peaks))
+    del w
+    run("moe_gateup", lambda: _moe_row("gateup", steps, peaks))
+    run("moe_down", lambda: _moe_row("down", steps, peaks))
+    out["how"] = ("per row: K steps (quantize + linear) as one CUDA graph between events, R rotating input sets "
+                  "(each with its own weight copy) so that inputs exceed L2; linear_frac against the FP4 peak "
+                  "(bf16 burst x 4), or the FP8 peak (x 2) for MXFP8; quantize bytes: X + codes + scales + B")
+    return out
+
+
 _ORACLE_PREP = {}
 
 
@@ -502,6 +756,8 @@ def main():
         return
     res, wl = run_osc(args)
     if res is not None:
+        if res["n_gpus"] == 1 and not args.no_rows:
+            res["scope_rows"] = scope_rows(min(args.steps, 50))
         if not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(wl["X"], wl["W"], wl["calib"], args.cpu_seconds)
         print(json.dumps(res), flush=True)

@@ -92,13 +92,19 @@ def test_w2_osc_full_size(oracle, osc):
 
 
 @pytest.mark.parametrize("shape,pair", [((4096, 12288, 4096), -1), ((4096, 12288, 4096), 1), ((130, 512, 144), 1),
-                                        ((130, 512, 256), 2), ((1, 256, 16), -1)])
+                                        ((130, 512, 256), 2), ((1, 256, 16), -1), ((2048, 4096, 6144), -1)])
 def test_fp8_fallback(oracle, osc, shape, pair):
+    """The MXFP8 path: the W2 fallback at full size, small ragged shapes, and the QKV shape
+    (the W8A8 comparator of the OSC page's Table 2)."""
     M, K, N = shape
     if M == 4096:
         c = I.w2_case(M=4096)
         X, W = c.X, c.W
         rows = I.sample_rows(M, 12, seed=8)
+    elif M == 2048:
+        c = I.qkv_case(2048)
+        X, W = c.X, c.W
+        rows = I.sample_rows(M, 12, seed=9)
     else:
         rng = np.random.default_rng(M)
         X = I.bf16_bits(rng.standard_normal((M, K)) * np.exp2(rng.integers(-6, 6, (M, 1))))
@@ -196,6 +202,11 @@ def _moe(oracle, osc, counts, which="gateup", rows_per_expert=None):
 
 def test_moe_grouped_small(oracle, osc):
     _moe(oracle, osc, [130, 0, 1, 257, 64, 3, 128, 40])
+
+
+def test_moe_grouped_small_down(oracle, osc):
+    """The down projection of the expert layer (K = 768: three k-stages, 24 groups)."""
+    _moe(oracle, osc, [130, 0, 1, 257, 64, 3, 128, 40], "down")
 
 
 def test_moe_grouped_full_size_gateup(oracle, osc):
