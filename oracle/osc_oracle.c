@@ -25,6 +25,14 @@
  *
  * Inputs must be finite; the functions return -1 on a non-finite input or a
  * bad argument and 0 on success.
+ *
+ * Every function here is pinned by tests/test_oracle_pins.py to something other
+ * than itself (format definitions, brute force, closed forms, invariants, library
+ * matmul), and tests/test_oracle_mutants.py checks that planted mistakes fail those
+ * pins. Parity unpinned: the output of the table build (Algorithm 1) on inputs
+ * without planted structure. It follows from the READING of the outlier event
+ * below and is pinned only where that reading fixes it (planted channels,
+ * closed-form thresholds, tie rules).
  */
 #include <math.h>
 #include <stdint.h>
