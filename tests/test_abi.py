@@ -131,6 +131,7 @@ def test_argument_limits_of_every_entry_point(lib):
     qg.argtypes = [V, I, V, V, V, I, I, I, V, I, V, V, V, V]
     assert qg(p16, 2, p16, p16, p16, 200, 256, 32, p16, 0, p16, p16, None, None) == -2   # Mp % 128
     assert qg(p16, 2, p16, p16, p16, 256, 256, 32, None, 0, p16, p16, None, None) == -1  # tables required
+    assert qg(p16, 2, p16, p16, p16, 1 << 30, 256, 32, p16, 0, p16, p16, None, None) == -1  # scale index overflow
     lg = lib.osc_linear_grouped
     lg.argtypes = [V, V, V, V, V, V, V, V, I, I, I, I, I, I, V, V, V]
     assert lg(p16, p16, None, p16, p16, None, p16, None, 2, 200, 256, 256, 32, 0, p16, None, None) == -2  # Mp % 128

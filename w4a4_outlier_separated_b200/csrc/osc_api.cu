@@ -365,6 +365,7 @@ int osc_quantize_grouped(const uint16_t* X, int E, const int* off, const int* po
     return OSC_ERR_ARG;
   if (K_L > 0 && !B) return OSC_ERR_ARG;
   if (K_L > 32767) return OSC_ERR_ARG;
+  if ((long long)(Mp + 127) * (K / 32) >= (1LL << 31)) return OSC_ERR_ARG;
   if (!a16(X) || !a16(QX) || !a16(SX) || (B && !a16(B))) return OSC_ERR_ALIGN;
   if (K % 256 != 0 || K_L % 16 != 0 || Mp % 128 != 0) return OSC_ERR_ALIGN;
   if (osc::grouped_quant_smem(E, K / G) > 200 * 1024) return OSC_ERR_ARG;   // E x K/G table entries
