@@ -211,3 +211,7 @@ def test_moe_grouped_small_down(oracle, osc):
 
 def test_moe_grouped_full_size_gateup(oracle, osc):
     _moe(oracle, osc, None, "gateup", rows_per_expert=2)
+
+
+def test_moe_grouped_full_size_down(oracle, osc):
+    _moe(oracle, osc, None, "down", rows_per_expert=2)
