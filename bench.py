@@ -624,22 +624,43 @@ def _moe_row(which, steps, peaks):
     return rec
 
 
+def _tier(X, calib, G):
+    """Automatic tier of a module input (§2.2, §2.3): table by Algorithm 1 on the calibration
+    tokens, per-group density of that table on the evaluation tokens, both on the GPU; the
+    tier rule runs on the host over the counts."""
+    import torch
+    from w4a4_outlier_separated_b200 import osc
+    K = X.shape[1]
+    Ld = torch.empty(K // G, dtype=torch.int8, device="cuda")
+    osc.osc_build_table(_to_dev(calib), G, 5.0, 5, Ld)
+    nh = torch.empty(K // G, dtype=torch.int32, device="cuda")
+    nt = torch.empty(K // G, dtype=torch.int32, device="cuda")
+    osc.osc_density(_to_dev(X), G, 5.0, Ld, nh, nt)
+    _status_ok()
+    tier, c = osc.osc_select_tier(nh.cpu().numpy(), nt.cpu().numpy())
+    return {"C_bar": round(c, 4), "tier": osc.TIERS[tier],
+            "path": "MXFP8 fallback" if tier == 0 else "OSC W4A4",
+            "table_entries": int((Ld >= 0).sum().item())}
+
+
 def scope_rows(steps: int):
     """Every other row of the path, measured like the headline: one graph of `steps` steps
     replayed between events, inputs rotated so that no step finds them in L2, and per-kernel
     graphs for the rooflines. FFN up/gate at G = 16 / 32 / 64; W2 (K = 12288) as OSC and as the
     MXFP8 fallback; the grouped MoE expert layers; and the W8A8 comparator of the page's
-    Table 2 at the QKV shape beside OSC at G = 16 / 32 / 64 (step-time ratio)."""
+    Table 2 at the QKV shape beside OSC at G = 16 / 32 / 64 (step-time ratio). "tiers" holds
+    the automatic tier of each dense module input (density on the GPU, rule on the host)."""
     import torch
     from w4a4_outlier_separated_b200 import inputs as I
     peaks, _ = measured_peaks()
     out = {}
+    tiers = {}
 
-    def run(key, fn):
+    def run(key, fn, dest=out):
         try:
-            out[key] = fn()
+            dest[key] = fn()
         except Exception as exc:                     # recorded, so the headline line still prints
-            out[key] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+            dest[key] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
 
@@ -652,19 +673,23 @@ def scope_rows(steps: int):
         out["table2_osc_speedup_over_w8a8"] = {
             f"G{G}": round(w8["ms_per_step"] / out[f"qkv_g{G}"]["ms_per_step"], 3)
             for G in (16, 32, 64) if "ms_per_step" in out.get(f"qkv_g{G}", {})}
+    run("qkv_g32", lambda: _tier(q.X, q.calib, 32), tiers)
     del q
     f = I.ffn_case(32)
     for G in (16, 32, 64):
         run(f"ffn_g{G}", lambda G=G: _osc_dense_row(f"ffn_up M=4096 K=4096 N=24576 G={G}", f.X, f.W, f.calib, G,
                                                     steps, 2, peaks))
+    run("ffn_g32", lambda: _tier(f.X, f.calib, 32), tiers)
     del f
     w = I.w2_case()
     run("w2_osc_g32", lambda: _osc_dense_row("w2_down M=4096 K=12288 N=4096 G=32", w.X, w.W, w.calib, 32, steps, 2, peaks))
     run("w2_fp8_fallback", lambda: _fp8_dense_row("w2_down M=4096 K=12288 N=4096 MXFP8 fallback", w.X, w.W, steps, 2,
                                                   peaks))
+    run("w2_g32", lambda: _tier(w.X, w.calib, 32), tiers)
     del w
     run("moe_gateup", lambda: _moe_row("gateup", steps, peaks))
     run("moe_down", lambda: _moe_row("down", steps, peaks))
+    out["tiers"] = tiers
     out["how"] = ("per row: K steps (quantize + linear) as one CUDA graph between events, R rotating input sets "
                   "(each with its own weight copy) so that inputs exceed L2; linear_frac against the FP4 peak "
                   "(bf16 burst x 4), or the FP8 peak (x 2) for MXFP8; quantize bytes: X + codes + scales + B")

@@ -100,6 +100,28 @@ OSC_API int osc_table_kl(const int8_t* L_host, int Kg);
 OSC_API int osc_build_table(const uint16_t* Xcal, int S, int K, int G, float alpha, int min_hits,
                     int8_t* L, osc_stream_t stream);
 
+/* §2.2 clustering density of a table on S x K activations X (device), with the event of
+ * osc_build_table: n_total[k] counts group k's outlier events over the S tokens and n_hit[k]
+ * those whose channel is L[k] (0 when L[k] = -1), so C_k = n_hit[k] / n_total[k]. L, n_hit
+ * and n_total are device arrays of K/G entries (int8, int32, int32). A table entry >= G is
+ * recorded in the status word (OSC_ERR_TABLE from osc_status) and counts no hits. */
+OSC_API int osc_density(const uint16_t* X, int S, int K, int G, float alpha, const int8_t* L,
+                        int* n_hit, int* n_total, osc_stream_t stream);
+
+/* Tiers of §2.3, chosen from the density of a module input. */
+enum {
+  OSC_TIER_FP8 = 0,   /* C < 35 %: MXFP8 fallback (§4) */
+  OSC_TIER_MID = 1,   /* 35 % <= C <= 60 %: static protection still helps (OSC W4A4) */
+  OSC_TIER_HIGH = 2   /* C > 60 %: static channel protection (OSC W4A4) */
+};
+
+/* HOST logic on the counts of osc_density (host arrays, Kg entries): C = mean over the groups
+ * with events (n_total > 0) of n_hit / n_total, summed in double over ascending k; *c_bar
+ * (may be NULL) receives it. Returns the tier above, or OSC_ERR_ARG for a negative count or
+ * n_hit > n_total (the arrays may be NULL when Kg = 0). With no events at all, *c_bar is NaN and the result is OSC_TIER_HIGH
+ * (nothing escapes the table; with an empty table OSC is plain MXFP4). */
+OSC_API int osc_select_tier(const int* n_hit, const int* n_total, int Kg, double* c_bar);
+
 /* §3.2, Figure 2 (online): extraction + zeroing through the table, then MXFP4 quantization
  * of the zeroed tensor. X (M x K bf16) -> QX (M x K/2), SX (osc_scale_bytes(M, K, G)),
  * B (M x K_L bf16). L may be NULL (no table: plain MXFP4; then K_L must be 0 and B may be

@@ -136,6 +136,15 @@ def test_argument_limits_of_every_entry_point(lib):
     lg.argtypes = [V, V, V, V, V, V, V, V, I, I, I, I, I, I, V, V, V]
     assert lg(p16, p16, None, p16, p16, None, p16, None, 2, 200, 256, 256, 32, 0, p16, None, None) == -2  # Mp % 128
     assert lg(p16, p16, None, p16, p16, None, None, None, 2, 256, 256, 256, 32, 0, p16, None, None) == -1  # no map
+    dn = lib.osc_density
+    dn.argtypes = [V, I, I, I, ctypes.c_float, V, V, V, V]
+    assert dn(p16, 8, 256, 24, 5.0, p16, p16, p16, None) == -3              # G
+    assert dn(p16, 8, 250, 32, 5.0, p16, p16, p16, None) == -1              # K % G
+    assert dn(p16, 8, 256, 32, 5.0, None, p16, p16, None) == -1             # table required
+    assert dn(V(p16.value + 2), 8, 256, 32, 5.0, p16, p16, p16, None) == -2  # alignment
+    st = lib.osc_select_tier
+    st.argtypes = [V, V, I, V]
+    assert st(None, None, 0, None) == 2 and st(None, None, 3, None) == -1
     lib.osc_set_cta_pair.argtypes = [I]
     assert lib.osc_set_cta_pair(3) == -1
     prev = lib.osc_set_cta_pair(1)

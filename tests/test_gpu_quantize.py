@@ -198,3 +198,45 @@ def test_build_table(oracle, osc, case, G, alpha, min_hits):
     osc.osc_build_table(to_dev(X), G, alpha, min_hits, L)
     torch.cuda.synchronize()
     assert np.array_equal(to_np(L), oracle.build_table(X, G, alpha, min_hits))
+
+
+@pytest.mark.parametrize("case,G", [("qkv", 32), ("w2", 32), ("ffn", 16), ("ffn", 64), ("random", 32)])
+def test_density_and_tier(oracle, osc, case, G):
+    """§2.2 density on the GPU: per-group event and hit counts equal the oracle's, for a table
+    built from calibration tokens and evaluated on other tokens; the tier chosen from the GPU
+    counts is the one chosen from the oracle's."""
+    if case == "qkv":
+        c = I.qkv_case(512)
+        X, L = c.X, oracle.build_table(c.calib, G)
+    elif case == "w2":
+        c = I.w2_case(M=512)
+        X, L = c.X, oracle.build_table(c.calib, G)
+    elif case == "ffn":
+        c = I.ffn_case(G, M=512)
+        X, L = c.X, oracle.build_table(c.calib, G)
+    else:
+        rng = np.random.default_rng(17)
+        X = I.bf16_bits(rng.standard_t(3, size=(600, 1024)))
+        L = rng.integers(-1, G, size=1024 // G).astype(np.int8)
+        L[0], L[1], L[2] = 0, G - 1, -1
+    S, K = X.shape
+    nh = torch.empty(K // G, dtype=torch.int32, device="cuda")
+    nt = torch.empty(K // G, dtype=torch.int32, device="cuda")
+    osc.osc_density(to_dev(X), G, 5.0, to_dev(L), nh, nt)
+    torch.cuda.synchronize()
+    assert osc.osc_status() == (0, 0)
+    rh, rt = oracle.density(X, G, L, 5.0)
+    assert np.array_equal(to_np(nh), rh) and np.array_equal(to_np(nt), rt)
+    assert osc.osc_select_tier(to_np(nh), to_np(nt)) == osc.osc_select_tier(rh, rt)
+
+
+def test_density_bad_table_entry_is_reported(osc):
+    X = to_dev(I.bf16_bits(np.random.default_rng(2).standard_normal((64, 256)) * 3))
+    L = np.full(8, -1, np.int8)
+    L[5] = 33                                   # >= G
+    nh = torch.empty(8, dtype=torch.int32, device="cuda")
+    nt = torch.empty(8, dtype=torch.int32, device="cuda")
+    osc.osc_density(X, 32, 5.0, to_dev(L), nh, nt)
+    torch.cuda.synchronize()
+    assert osc.osc_status() == (-6, 2)
+    assert to_np(nh)[5] == 0

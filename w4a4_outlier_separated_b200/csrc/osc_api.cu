@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 
@@ -249,6 +250,38 @@ int osc_build_table(const uint16_t* Xcal, int S, int K, int G, float alpha, int 
   if (rc != OSC_OK) return rc;
   osc::TableParams p{Xcal, S, K, G, alpha, min_hits, L};
   return launch_result(osc::launch_build_table(p, ds->sms, (cudaStream_t)stream));
+}
+
+int osc_density(const uint16_t* X, int S, int K, int G, float alpha, const int8_t* L, int* n_hit, int* n_total,
+                osc_stream_t stream) {
+  if (!valid_g(G)) return OSC_ERR_G;
+  if (!X || !L || !n_hit || !n_total || S < 0 || K <= 0 || K % G != 0) return OSC_ERR_ARG;
+  if (!a16(X)) return OSC_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != OSC_OK) return rc;
+  osc::DensityParams p{X, S, K, G, alpha, L, n_hit, n_total, ds->status};
+  return launch_result(osc::launch_density(p, (cudaStream_t)stream));
+}
+
+int osc_select_tier(const int* n_hit, const int* n_total, int Kg, double* c_bar) {
+  if (Kg < 0 || (Kg > 0 && (!n_hit || !n_total))) return OSC_ERR_ARG;
+  double sum = 0.0;
+  int groups = 0;
+  for (int k = 0; k < Kg; ++k) {
+    if (n_hit[k] < 0 || n_total[k] < 0 || n_hit[k] > n_total[k]) return OSC_ERR_ARG;
+    if (n_total[k] > 0) {
+      sum += (double)n_hit[k] / (double)n_total[k];
+      ++groups;
+    }
+  }
+  if (groups == 0) {
+    if (c_bar) *c_bar = std::nan("");
+    return OSC_TIER_HIGH;
+  }
+  const double c = sum / groups;
+  if (c_bar) *c_bar = c;
+  return c > 0.60 ? OSC_TIER_HIGH : (c >= 0.35 ? OSC_TIER_MID : OSC_TIER_FP8);
 }
 
 int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int K_L, uint8_t* QX, uint8_t* SX,

@@ -79,4 +79,15 @@ struct TableParams {
 };
 cudaError_t launch_build_table(const TableParams& p, int num_sms, cudaStream_t s);
 
+struct DensityParams {
+  const uint16_t* X;   // S x K bf16
+  int S, K, G;
+  float alpha;
+  const int8_t* L;     // K/G entries
+  int* n_hit;          // K/G
+  int* n_total;        // K/G
+  int* status;
+};
+cudaError_t launch_density(const DensityParams& p, cudaStream_t s);
+
 }  // namespace osc

@@ -11,10 +11,38 @@
 // does not depend on the order in which tokens are visited.
 //
 // One CTA per channel group; threads stride over tokens; a shared histogram of G counters.
+//
+// The clustering density of §2.2 uses the same event: over a set of tokens, N_total(k) counts
+// group k's events and N_hit(k) those whose channel is the table's entry L[k]; the ratio
+// C_k = N_hit / N_total, averaged over the groups with events, selects the tier of §2.3.
 #include "osc_device.cuh"
 #include "osc_internal.h"
 
 namespace osc {
+
+// One token's group of G bf16 values at xg (16-byte aligned): the channel of largest |x|
+// (lowest on ties, compared on the magnitude bits) and whether it is an outlier event.
+template <int G>
+__device__ __forceinline__ bool group_event(const uint16_t* xg, float alpha, int* j_out) {
+  const uint4* src = reinterpret_cast<const uint4*>(xg);
+  float s = 0.0f;
+  uint32_t best = 0;
+  int jb = 0;
+#pragma unroll
+  for (int v = 0; v < G / 8; ++v) {
+    const uint4 r = __ldg(src + v);
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      const uint32_t mag = (h & 1) ? (w[h >> 1] >> 16) & 0x7FFFu : w[h >> 1] & 0x7FFFu;
+      s += __uint_as_float(mag << 16);
+      if (mag > best) { best = mag; jb = v * 8 + h; }
+    }
+  }
+  *j_out = jb;
+  const double amax = (double)__uint_as_float(best << 16);
+  return best != 0u && (double)G * amax >= (double)alpha * (double)s;
+}
 
 template <int G>
 __global__ void __launch_bounds__(256) build_table_kernel(TableParams p) {
@@ -23,23 +51,8 @@ __global__ void __launch_bounds__(256) build_table_kernel(TableParams p) {
   for (int j = threadIdx.x; j < G; j += blockDim.x) hist[j] = 0;
   __syncthreads();
   for (int t = threadIdx.x; t < p.S; t += blockDim.x) {
-    const uint4* src = reinterpret_cast<const uint4*>(p.X + (size_t)t * p.K + (size_t)k * G);
-    float s = 0.0f;
-    uint32_t best = 0;
-    int jb = 0;
-#pragma unroll
-    for (int v = 0; v < G / 8; ++v) {
-      const uint4 r = __ldg(src + v);
-      const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        const uint32_t mag = (h & 1) ? (w[h >> 1] >> 16) & 0x7FFFu : w[h >> 1] & 0x7FFFu;
-        s += __uint_as_float(mag << 16);
-        if (mag > best) { best = mag; jb = v * 8 + h; }
-      }
-    }
-    const double amax = (double)__uint_as_float(best << 16);
-    if (best != 0u && (double)G * amax >= (double)p.alpha * (double)s) atomicAdd(&hist[jb], 1);
+    int jb;
+    if (group_event<G>(p.X + (size_t)t * p.K + (size_t)k * G, p.alpha, &jb)) atomicAdd(&hist[jb], 1);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -48,6 +61,46 @@ __global__ void __launch_bounds__(256) build_table_kernel(TableParams p) {
       if (hist[j] > hist[js]) js = j;
     p.L[k] = (hist[js] > 0 && hist[js] >= p.min_hits) ? (int8_t)js : (int8_t)-1;
   }
+}
+
+// One CTA per group: the group's event and hit counts over the S tokens.
+template <int G>
+__global__ void __launch_bounds__(256) density_kernel(DensityParams p) {
+  __shared__ int cnt[2];
+  const int k = blockIdx.x;
+  if (threadIdx.x < 2) cnt[threadIdx.x] = 0;
+  const int l = p.L[k];
+  if (threadIdx.x == 0 && l >= G) record_status(p.status, DEV_BAD_TABLE);   // never matches a channel
+  __syncthreads();
+  int hit = 0, tot = 0;
+  for (int t = threadIdx.x; t < p.S; t += blockDim.x) {
+    int jb;
+    if (group_event<G>(p.X + (size_t)t * p.K + (size_t)k * G, p.alpha, &jb)) {
+      ++tot;
+      hit += (jb == l);
+    }
+  }
+  if (tot) {
+    atomicAdd(&cnt[0], hit);
+    atomicAdd(&cnt[1], tot);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    p.n_hit[k] = cnt[0];
+    p.n_total[k] = cnt[1];
+  }
+}
+
+cudaError_t launch_density(const DensityParams& p, cudaStream_t s) {
+  const int Kg = p.K / p.G;
+  if (Kg == 0) return cudaSuccess;
+  switch (p.G) {
+    case 16: density_kernel<16><<<Kg, 256, 0, s>>>(p); break;
+    case 32: density_kernel<32><<<Kg, 256, 0, s>>>(p); break;
+    case 64: density_kernel<64><<<Kg, 256, 0, s>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
 }
 
 cudaError_t launch_build_table(const TableParams& p, int num_sms, cudaStream_t s) {

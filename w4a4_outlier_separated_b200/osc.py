@@ -45,6 +45,8 @@ def lib() -> ctypes.CDLL:
             "osc_scale_bytes": ([i32, i32, i32], ctypes.c_size_t),
             "osc_table_kl": ([P, i32], i32),
             "osc_build_table": ([P, i32, i32, i32, f32, i32, P, P], i32),
+            "osc_density": ([P, i32, i32, i32, f32, P, P, P, P], i32),
+            "osc_select_tier": ([P, P, i32, P], i32),
             "osc_quantize": ([P, i32, i32, i32, P, i32, P, P, P, P], i32),
             "osc_prepare_weight": ([P, i32, i32, i32, P, i32, P, P, P, P], i32),
             "osc_linear": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P], i32),
@@ -114,6 +116,31 @@ def osc_set_cta_pair(mode: int) -> int:
 def osc_build_table(Xcal, G: int, alpha: float, min_hits: int, L, stream=None):
     S, K = Xcal.shape
     _check("osc_build_table", lib().osc_build_table(_ptr(Xcal), S, K, G, alpha, min_hits, _ptr(L), _stream(stream)))
+
+
+def osc_density(X, G: int, alpha: float, L, n_hit, n_total, stream=None):
+    """Per-group outlier-event and table-hit counts (int32 CUDA tensors of K/G entries)."""
+    S, K = X.shape
+    _check("osc_density", lib().osc_density(_ptr(X), S, K, G, alpha, _ptr(L), _ptr(n_hit), _ptr(n_total),
+                                            _stream(stream)))
+
+
+TIERS = {0: "fp8_fallback", 1: "mid", 2: "high"}
+
+
+def osc_select_tier(n_hit, n_total):
+    """Host counts (numpy or CPU tensors) -> (tier code, C-bar). The tier codes are those of
+    include/osc.h: 0 = MXFP8 fallback, 1 = mid, 2 = high clustering."""
+    h = torch.as_tensor(n_hit, dtype=torch.int32).contiguous().cpu()
+    t = torch.as_tensor(n_total, dtype=torch.int32).contiguous().cpu()
+    if h.numel() != t.numel():
+        raise ValueError("n_hit and n_total differ in length")
+    c = ctypes.c_double(0.0)
+    rc = lib().osc_select_tier(ctypes.c_void_p(h.data_ptr()), ctypes.c_void_p(t.data_ptr()), h.numel(),
+                               ctypes.byref(c))
+    if rc < 0:
+        _check("osc_select_tier", rc)
+    return int(rc), float(c.value)
 
 
 def osc_quantize(X, G: int, L, K_L: int, QX, SX, B, stream=None):
