@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
   for (; step < cta_end; step += wstride, slot ^= 1) {
     const bool loaded = step * QSTEP < real_items;            // warp-uniform (pad rows are not loaded)
     if (loaded) {
-      // lane 0 waits (bounded) and the warp follows its verdict; __syncwarp then orders the
+      // lane 0 waits (bounded) and the warp follows its result; __syncwarp then orders the
       // other lanes' shared-memory reads after the completed load
       bool ok = true;
       if (lane == 0) ok = mbar_wait(smem_u32(&s_bar[warp][slot]), (phbits >> slot) & 1u, reinterpret_cast<volatile int*>(&s_abort), p.status);
