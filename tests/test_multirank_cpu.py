@@ -90,3 +90,18 @@ def test_reference_arm_runs_on_rank0_only():
     out = subprocess.run([sys.executable, "-c", REF_WORKER], env=env, capture_output=True, text=True, timeout=120)
     assert out.returncode == 0, out.stderr[-2000:]
     assert out.stdout.strip().splitlines()[-1] == "NONE"
+
+
+def test_algorithmic_bytes_and_row_record():
+    """The quantize byte counts behind the HBM fractions: X read (bf16), codes, one E8M0 byte
+    per 32 (or 16) elements, and B, written out for the QKV and W2 shapes."""
+    import bench
+    assert bench.quant_bytes(2048, 4096, 32, 96) == 2048 * 4096 * 2 + 2048 * 2048 + 2048 * 128 + 2048 * 96 * 2
+    assert bench.quant_bytes(2048, 4096, 32, 96) == 21_626_880                  # ~21.6 MB per QKV launch
+    assert bench.quant_bytes(2048, 4096, 16, 96) - bench.quant_bytes(2048, 4096, 32, 96) == 2048 * 128
+    assert bench.quant_bytes(4096, 12288, 32, 0, fp8=True) == 152_567_808       # MXFP8 W2: ~3.03 B/elem
+    peaks = {"hbm_gbs": 6450.0, "bf16_tflops": 1672.7}
+    r = bench._row_record("x", 2048, 4096, 6144, 32, 96, 0.0373, 0.0073, 0.0284, 2.0 * 2048 * 6144 * 4096,
+                          21_626_880, 4 * 1672.7, peaks, 8)
+    assert abs(r["TFLOPs"] - 2764.2) < 1.0 and abs(r["linear_frac"] - 0.5425) < 1e-3
+    assert abs(r["quantize_GBps"] - 2962.6) < 0.5 and abs(r["quantize_hbm_frac"] - 0.459) < 1e-3
