@@ -477,11 +477,26 @@ def _status_ok():
         raise RuntimeError(f"device status {code} ({raw})")
 
 
-def _row_record(name, M, K, N, G, K_L, s_ms, q_ms, l_ms, useful_flops, qbytes, tc_peak, peaks, R):
+def tensor_bytes(*ts) -> int:
+    """Bytes of the given tensors (None entries count 0)."""
+    return int(sum(t.numel() * t.element_size() for t in ts if t is not None))
+
+
+def _row_record(name, M, K, N, G, K_L, s_ms, q_ms, l_ms, useful_flops, qbytes, tc_peak, peaks, R, lbytes, mma_flops=None):
+    """One row's line. The linear kernel is held to the roofline that bounds it: the tensor
+    peak for its MMA flops, or HBM for the bytes it must move (operands, scales, B, W_L read
+    once and Y written once), whichever takes longer."""
+    mma_flops = useful_flops if mma_flops is None else mma_flops
+    t_tensor = mma_flops / (tc_peak * 1e12)
+    t_hbm = lbytes / (peaks["hbm_gbs"] * 1e9)
     return {"workload": name, "M": M, "K": K, "N": N, "G": G, "K_L": K_L, "input_sets": R,
             "ms_per_step": round(s_ms, 5), "TFLOPs": round(useful_flops / (s_ms * 1e-3) / 1e12, 1),
             "linear_ms": round(l_ms, 5),
             "linear_frac": round(useful_flops / (l_ms * 1e-3) / 1e12 / tc_peak, 4),
+            "linear_bytes": lbytes,
+            "linear_GBps": round(lbytes / (l_ms * 1e-3) / 1e9, 1),
+            "linear_bound": "hbm" if t_hbm > t_tensor else "tensor",
+            "linear_roofline_frac": round(max(t_hbm, t_tensor) / (l_ms * 1e-3), 4),
             "quantize_ms": round(q_ms, 5),
             "quantize_GBps": round(qbytes / (q_ms * 1e-3) / 1e9, 1),
             "quantize_hbm_frac": round(qbytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}
@@ -526,8 +541,10 @@ def _osc_dense_row(name, X, W, calib, G, steps, R, peaks):
     torch.cuda.synchronize()
     s_ms, q_ms, l_ms = _timed_graphs([step, quant, lin], steps)
     _status_ok()
+    c = sets[0]
+    lbytes = tensor_bytes(c["QX"], c["SX"], c["B"], c["QW"], c["SW"], c["WL"], c["Y"])
     return _row_record(name, M, K, N, G, K_L, s_ms, q_ms, l_ms, 2.0 * M * N * K, quant_bytes(M, K, G, K_L),
-                       4.0 * peaks["bf16_tflops"], peaks, R)
+                       4.0 * peaks["bf16_tflops"], peaks, R, lbytes)
 
 
 def _fp8_dense_row(name, X, W, steps, R, peaks):
@@ -566,8 +583,10 @@ def _fp8_dense_row(name, X, W, steps, R, peaks):
     torch.cuda.synchronize()
     s_ms, q_ms, l_ms = _timed_graphs([step, quant, lin], steps)
     _status_ok()
+    c = sets[0]
+    lbytes = tensor_bytes(c["QX"], c["SX"], c["QW"], c["SW"], c["Y"])
     return _row_record(name, M, K, N, 32, 0, s_ms, q_ms, l_ms, 2.0 * M * N * K, quant_bytes(M, K, 32, 0, fp8=True),
-                       2.0 * peaks["bf16_tflops"], peaks, R)
+                       2.0 * peaks["bf16_tflops"], peaks, R, lbytes)
 
 
 def _moe_row(which, steps, peaks):
@@ -617,8 +636,10 @@ def _moe_row(which, steps, peaks):
     s_ms, q_ms, l_ms = _timed_graphs([step, quant, lin], steps)
     _status_ok()
     T = int(case.counts.sum())
+    lbytes = tensor_bytes(QX, SX, B, QW, SW, WL, Y)                  # every expert's weights, padded rows
     rec = _row_record(f"moe_{which} E={E} top-8 of 4096 tokens", T, K, N, G, K_L, s_ms, q_ms, l_ms, 2.0 * T * N * K,
-                      quant_bytes(T, K, G, K_L), 4.0 * peaks["bf16_tflops"], peaks, 1)
+                      quant_bytes(T, K, G, K_L), 4.0 * peaks["bf16_tflops"], peaks, 1, lbytes,
+                      mma_flops=2.0 * Mp * N * K)
     rec.update(padded_rows=Mp, experts_with_tokens=int((case.counts > 0).sum()),
                largest_expert=int(case.counts.max()))
     return rec
@@ -691,8 +712,10 @@ def scope_rows(steps: int):
     run("moe_down", lambda: _moe_row("down", steps, peaks))
     out["tiers"] = tiers
     out["how"] = ("per row: K steps (quantize + linear) as one CUDA graph between events, R rotating input sets "
-                  "(each with its own weight copy) so that inputs exceed L2; linear_frac against the FP4 peak "
-                  "(bf16 burst x 4), or the FP8 peak (x 2) for MXFP8; quantize bytes: X + codes + scales + B")
+                  "(each with its own weight copy) so that inputs exceed L2; linear_frac = useful flops against the "
+                  "FP4 peak (bf16 burst x 4), or the FP8 peak (x 2) for MXFP8; linear_roofline_frac = the longer of "
+                  "(MMA flops / tensor peak) and (linear_bytes / HBM) over the measured time, linear_bound names it; "
+                  "quantize bytes: X + codes + scales + B")
     return out
 
 

@@ -101,7 +101,15 @@ def test_algorithmic_bytes_and_row_record():
     assert bench.quant_bytes(2048, 4096, 16, 96) - bench.quant_bytes(2048, 4096, 32, 96) == 2048 * 128
     assert bench.quant_bytes(4096, 12288, 32, 0, fp8=True) == 152_567_808       # MXFP8 W2: ~3.03 B/elem
     peaks = {"hbm_gbs": 6450.0, "bf16_tflops": 1672.7}
+    qkv_lbytes = 4_194_304 + 262_144 + 393_216 + 12_582_912 + 786_432 + 1_179_648 + 25_165_824
     r = bench._row_record("x", 2048, 4096, 6144, 32, 96, 0.0373, 0.0073, 0.0284, 2.0 * 2048 * 6144 * 4096,
-                          21_626_880, 4 * 1672.7, peaks, 8)
+                          21_626_880, 4 * 1672.7, peaks, 8, qkv_lbytes)
     assert abs(r["TFLOPs"] - 2764.2) < 1.0 and abs(r["linear_frac"] - 0.5425) < 1e-3
     assert abs(r["quantize_GBps"] - 2962.6) < 0.5 and abs(r["quantize_hbm_frac"] - 0.459) < 1e-3
+    assert r["linear_bound"] == "tensor" and r["linear_roofline_frac"] == r["linear_frac"]
+    # MoE gate+up: 404 MB to move at 6.45 TB/s (62.6 us) outlasts 253 GFLOP at 6.69 PFLOP/s (37.8 us)
+    moe = bench._row_record("m", 32768, 2048, 1536, 32, 48, 0.174, 0.0759, 0.0998, 2.0 * 32768 * 1536 * 2048,
+                            1, 4 * 1672.7, peaks, 1, 404_000_000, mma_flops=2.0 * 40192 * 1536 * 2048)
+    assert moe["linear_bound"] == "hbm" and abs(moe["linear_roofline_frac"] - 0.6276) < 1e-3
+    import torch
+    assert bench.tensor_bytes(torch.empty(3, 5, dtype=torch.int16), None, torch.empty(7, dtype=torch.uint8)) == 37
