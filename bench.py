@@ -27,7 +27,6 @@ import hashlib
 import json
 import os
 import sys
-import threading
 import time
 
 import numpy as np
@@ -85,14 +84,15 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+    """Samples SM clock and throttle reasons through NVML while the timed work runs: the
+    caller enqueues the timed region, then calls sample_while(end_event), which samples from
+    the host until the event completes (at least once), so every sample falls inside it."""
 
     REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
                "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
     def __init__(self, dev_index: int):
         self.samples, self.reasons, self.max_mhz = [], set(), None
-        self._stop = threading.Event()
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -102,28 +102,24 @@ class ClockSampler:
         except Exception:
             self.nv = None
 
-    def _run(self):
-        while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                r = self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
-                for k, v in self.REASONS.items():
-                    if r & v:
-                        self.reasons.add(k)
-            except Exception:
-                pass
-            time.sleep(0.005)
+    def sample(self):
+        if self.nv is None:
+            return
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            r = self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+            for k, v in self.REASONS.items():
+                if r & v:
+                    self.reasons.add(k)
+        except Exception:
+            pass
 
-    def __enter__(self):
-        if self.nv is not None:
-            self.t = threading.Thread(target=self._run, daemon=True)
-            self.t.start()
-        return self
-
-    def __exit__(self, *a):
-        self._stop.set()
-        if self.nv is not None:
-            self.t.join()
+    def sample_while(self, end_event, period_s: float = 0.0005):
+        while True:
+            self.sample()
+            if end_event.query():
+                break
+            time.sleep(period_s)
 
     def summary(self):
         if not self.samples:
@@ -247,11 +243,12 @@ def run_osc(args):
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(dev_index) as clk:
-        e0.record(stream)
-        g_step.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
+    clk = ClockSampler(dev_index)
+    e0.record(stream)
+    g_step.replay()
+    e1.record(stream)
+    clk.sample_while(e1)                              # host-side samples while the timed steps run
+    torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
     step_ms = e0.elapsed_time(e1) / args.steps

@@ -113,3 +113,37 @@ def test_algorithmic_bytes_and_row_record():
     assert moe["linear_bound"] == "hbm" and abs(moe["linear_roofline_frac"] - 0.6276) < 1e-3
     import torch
     assert bench.tensor_bytes(torch.empty(3, 5, dtype=torch.int16), None, torch.empty(7, dtype=torch.uint8)) == 37
+
+
+def test_clock_sampler_samples_while_the_timed_work_runs():
+    """Samples are taken from the host until the end event of the timed region completes, at
+    least once; throttle reasons are collected by name."""
+    import bench
+
+    class NV:
+        NVML_CLOCK_SM = 0
+
+        @staticmethod
+        def nvmlDeviceGetClockInfo(h, kind):
+            return 1965
+
+        @staticmethod
+        def nvmlDeviceGetCurrentClocksThrottleReasons(h):
+            return 0x4
+
+    class Event:
+        def __init__(self, done_after):
+            self.calls, self.done_after = 0, done_after
+
+        def query(self):
+            self.calls += 1
+            return self.calls >= self.done_after
+
+    c = bench.ClockSampler(0)
+    c.nv, c.h, c.samples, c.reasons = NV, None, [], set()
+    c.sample_while(Event(3), 0.0)
+    assert len(c.samples) == 3
+    assert c.summary() == {"sm_mhz": 1965.0, "sm_max_mhz": c.max_mhz, "reasons": ["sw_power_cap"], "samples": 3}
+    c.samples = []
+    c.sample_while(Event(1), 0.0)                    # work already done: still one sample
+    assert len(c.samples) == 1
