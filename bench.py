@@ -801,9 +801,10 @@ def main():
         return
     res, wl = run_osc(args)
     if res is not None:
+        # the per-row measurements and the oracle's CPU baseline belong to the one-GPU line
         if res["n_gpus"] == 1 and not args.no_rows:
             res["scope_rows"] = scope_rows(min(args.steps, 50))
-        if not args.no_cpu_baseline:
+        if res["n_gpus"] == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(wl["X"], wl["W"], wl["calib"], args.cpu_seconds)
         print(json.dumps(res), flush=True)
 
