@@ -110,6 +110,16 @@ def test_argument_limits_of_every_entry_point(lib):
     assert q(p16, 1 << 30, 256, 32, None, 0, p16, p16, None, None) == -1   # (M + 127) * K / 32 >= 2^31
     assert q(p16, 4, 256, 32, p16, 16, p16, p16, None, None) == -1         # K_L > 0 needs B
     assert q(p16, 0, 256, 32, None, 0, None, None, None, None) == 0        # M = 0: no-op, NULLs allowed
+    li = lib.osc_linear
+    li.argtypes = [V] * 6 + [I] * 5 + [V, V, V]
+    assert li(None, None, None, None, None, None, 0, 128, 256, 32, 0, None, None, None) == 0   # M = 0: no-op
+    assert li(None, None, None, None, None, None, 0, 128, 256, 24, 0, None, None, None) == -3  # G still checked
+    q8 = lib.osc_quantize_fp8
+    q8.argtypes = [V, I, I, V, V, V]
+    assert q8(None, 0, 256, None, None, None) == 0                          # M = 0: no-op
+    l8 = lib.osc_linear_fp8_fallback
+    l8.argtypes = [V, V, V, V, I, I, I, V, V, V]
+    assert l8(None, None, None, None, 0, 64, 256, None, None, None) == 0  # M = 0: no-op
     w = lib.osc_prepare_weight
     w.argtypes = [V, I, I, I, V, I, V, V, V, V]
     assert w(p16, 4, 256, 48, None, 0, p16, p16, None, None) == -3         # G
