@@ -62,6 +62,15 @@ def test_qkv(oracle, osc, M):
     _run_osc(oracle, osc, c.X, c.W, 32, L, rows=rows)
 
 
+@pytest.mark.parametrize("G", [16, 64])
+def test_qkv_group_sizes_full_size(oracle, osc, G):
+    """The QKV shape at G = 16 and 64 in the launch configuration the bench times (automatic
+    tile and CTA grouping), table by Algorithm 1 for that G."""
+    c = I.qkv_case(2048)
+    L = oracle.build_table(c.calib, G)
+    _run_osc(oracle, osc, c.X, c.W, G, L, rows=I.sample_rows(2048, 16, seed=G + 1))
+
+
 def test_qkv_tile_shapes(oracle, osc):
     """128- and 256-wide single-CTA tiles and the 2-CTA 256 x 256 pair tile."""
     c = I.qkv_case(2048)
