@@ -667,7 +667,8 @@ def scope_rows(steps: int):
     graphs for the rooflines. FFN up/gate at G = 16 / 32 / 64; W2 (K = 12288) as OSC and as the
     MXFP8 fallback; the grouped MoE expert layers; and the W8A8 comparator of the page's
     Table 2 at the QKV shape beside OSC at G = 16 / 32 / 64 (step-time ratio). "tiers" holds
-    the automatic tier of each dense module input (density on the GPU, rule on the host)."""
+    the automatic tier of each dense module input at each group size (density on the GPU,
+    rule on the host)."""
     import torch
     from w4a4_outlier_separated_b200 import inputs as I
     peaks, _ = measured_peaks()
@@ -691,19 +692,22 @@ def scope_rows(steps: int):
         out["table2_osc_speedup_over_w8a8"] = {
             f"G{G}": round(w8["ms_per_step"] / out[f"qkv_g{G}"]["ms_per_step"], 3)
             for G in (16, 32, 64) if "ms_per_step" in out.get(f"qkv_g{G}", {})}
-    run("qkv_g32", lambda: _tier(q.X, q.calib, 32), tiers)
+    for G in (16, 32, 64):
+        run(f"qkv_g{G}", lambda G=G: _tier(q.X, q.calib, G), tiers)
     del q
     f = I.ffn_case(32)
     for G in (16, 32, 64):
         run(f"ffn_g{G}", lambda G=G: _osc_dense_row(f"ffn_up M=4096 K=4096 N=24576 G={G}", f.X, f.W, f.calib, G,
                                                     steps, 2, peaks))
-    run("ffn_g32", lambda: _tier(f.X, f.calib, 32), tiers)
+    for G in (16, 32, 64):
+        run(f"ffn_g{G}", lambda G=G: _tier(f.X, f.calib, G), tiers)
     del f
     w = I.w2_case()
     run("w2_osc_g32", lambda: _osc_dense_row("w2_down M=4096 K=12288 N=4096 G=32", w.X, w.W, w.calib, 32, steps, 2, peaks))
     run("w2_fp8_fallback", lambda: _fp8_dense_row("w2_down M=4096 K=12288 N=4096 MXFP8 fallback", w.X, w.W, steps, 2,
                                                   peaks))
-    run("w2_g32", lambda: _tier(w.X, w.calib, 32), tiers)
+    for G in (16, 32, 64):
+        run(f"w2_g{G}", lambda G=G: _tier(w.X, w.calib, G), tiers)
     del w
     run("moe_gateup", lambda: _moe_row("gateup", steps, peaks))
     run("moe_down", lambda: _moe_row("down", steps, peaks))
