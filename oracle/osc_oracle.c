@@ -93,8 +93,9 @@ static int all_finite_bf16(const uint16_t* x, int64_t n)
  * fp64, so both sides of any parity test take the same decision.
  * The channel with the most events wins (lowest j on ties) if it has at least
  * min_hits events; otherwise the group has no consistent outlier (-1).
- * j* = 0 is a valid channel (the page's "j_star if j_star else -1" would drop
- * it, which reads as a shorthand for "found", not as a rule).
+ * j* = 0 is a valid channel: the printed algorithm keeps the found channel only
+ * when its index is nonzero, which reads as a shorthand for "a channel was
+ * found", not as a rule.
  */
 static int group_event(const uint16_t* xg, int G, float alpha, int* j_out)
 {
