@@ -221,10 +221,11 @@ int orc_gather_wl(const uint16_t* W, int N, int K, int G, const int8_t* L,
     return 0;
 }
 
-/* ---- Microscaling (§3.2 "dynamic-range compression") ------------------------
+/* ---- Microscaling (§3.2, the dynamic-range step) ------------------------------
  *
- * The page computes "a tighter scale on the zeroed tensor" and quantizes it to
- * 4 bits; the element and scale formats are the OCP MX ones: E2M1 elements
+ * After the table channels are zeroed the page rescales each group with its
+ * now smaller range and quantizes it to 4 bits; the element and scale formats
+ * are the OCP MX ones: E2M1 elements
  * with one shared E8M0 power-of-two scale per block (E4M3 elements for the
  * FP8 fallback of §4).
  *   shared exponent   e = floor(log2(amax)) - emax_elem, emax_elem = 2 (E2M1)
