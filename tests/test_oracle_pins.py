@@ -116,6 +116,27 @@ def test_e4m3_decode_definition(oracle):
     assert vals.max() == 448.0 and np.isnan(oracle.decode_e4m3(0x7F))
 
 
+def test_e4m3_spec_points(oracle):
+    """The E4M3 decoder against the format's stated characteristic values (golden file), and
+    the quantizer at the saturation and subnormal boundaries those values define."""
+    rows = _read_table("e4m3_spec_points.txt")
+    assert len(rows) == 10
+    for r in rows:
+        code, want = int(r[0], 16), float(r[1])
+        got = oracle.decode_e4m3(code)
+        if np.isnan(want):
+            assert np.isnan(got)
+        else:
+            assert got == want and np.signbit(got) == np.signbit(want), (r, got)
+    # with e = 0 (block max 480: floor(log2 480) - 8 = 0): 448 stays, 470 saturates to 448,
+    # 2^-9 stays, 2^-10 is a tie with 0 (to the even code 0), 3 * 2^-11 rounds up to 2^-9
+    v = np.array([480.0, 448.0, 470.0, 2.0 ** -9, 2.0 ** -10, 3 * 2.0 ** -11, -(2.0 ** -10)])
+    X = I.bf16_bits(np.concatenate([v, np.zeros(32 - len(v))]))[None, :]
+    codes, exps = oracle.mx_quantize(X, 32, oracle.FMT_E4M3)
+    assert exps[0, 0] == 0
+    assert list(codes[0, :7]) == [0x7E, 0x7E, 0x7E, 0x01, 0x00, 0x01, 0x80]
+
+
 @pytest.mark.parametrize("shift", [0, 7, -50])
 def test_e4m3_rounding_matches_bruteforce(oracle, shift):
     anchor = I.bf16_bits(np.array([480.0 * 2.0 ** shift]))[0]      # floor(log2 480) - 8 = 0
