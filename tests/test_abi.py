@@ -159,3 +159,17 @@ def test_argument_limits_of_every_entry_point(lib):
     assert lib.osc_set_cta_pair(3) == -1
     prev = lib.osc_set_cta_pair(1)
     assert lib.osc_set_cta_pair(prev) == 1
+
+
+def test_scale_layout_fills_the_buffer_exactly(lib):
+    """The documented scale layout maps every (row, slot) of the padded rows to a distinct byte,
+    and together they cover the buffer osc_scale_bytes sizes, with no gap or overlap."""
+    from tests._layout import scale_offsets
+    f = lib.osc_scale_bytes
+    f.restype = ctypes.c_size_t
+    for rows, K, G in ((128, 256, 32), (256, 4096, 32), (384, 512, 16), (128, 1024, 64), (130, 768, 32)):
+        V = 16 if G == 16 else 32
+        mpad = (rows + 127) // 128 * 128
+        offs = scale_offsets(mpad, K, V).reshape(-1)
+        size = f(rows, K, G)
+        assert np.array_equal(np.sort(offs), np.arange(size)), (rows, K, G)
