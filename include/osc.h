@@ -189,6 +189,12 @@ OSC_API int osc_linear_grouped(const uint8_t* QX, const uint8_t* SX, const uint1
  * OSC_OK, OSC_ERR_TIMEOUT or OSC_ERR_TABLE; *raw (may be NULL) gets the raw device code. */
 OSC_API int osc_status(int* raw, osc_stream_t stream);
 
+/* Failure-detection self-test (not part of the OSC method): launches one kernel whose bounded
+ * wait on a barrier that nothing signals runs out after limit_us microseconds (1 .. 1000000).
+ * The timeout is recorded in the status word exactly as a stalled kernel pipeline records it,
+ * so the next osc_status returns OSC_ERR_TIMEOUT. No fault, trap or unbounded wait. */
+OSC_API int osc_selftest_timeout(int limit_us, osc_stream_t stream);
+
 /* Tile width of the tensor-core kernels: 0 = automatic (default), 128 or 256. Applies to
  * calls made afterwards from any thread. Returns the previous value, or OSC_ERR_ARG. */
 OSC_API int osc_set_tile_n(int bn);

@@ -155,6 +155,9 @@ def test_argument_limits_of_every_entry_point(lib):
     st = lib.osc_select_tier
     st.argtypes = [V, V, I, V]
     assert st(None, None, 0, None) == 2 and st(None, None, 3, None) == -1
+    stt = lib.osc_selftest_timeout
+    stt.argtypes = [I, V]
+    assert stt(0, None) == -1 and stt(2_000_000, None) == -1                # limit out of range
     lib.osc_set_cta_pair.argtypes = [I]
     assert lib.osc_set_cta_pair(3) == -1
     prev = lib.osc_set_cta_pair(1)

@@ -429,6 +429,15 @@ int osc_linear_grouped(const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
                   (cudaStream_t)stream);
 }
 
+int osc_selftest_timeout(int limit_us, osc_stream_t stream) {
+  if (limit_us < 1 || limit_us > 1000000) return OSC_ERR_ARG;
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != OSC_OK) return rc;
+  return launch_result(osc::launch_selftest_wait(ds->status, 1000ull * (unsigned long long)limit_us,
+                                                 (cudaStream_t)stream));
+}
+
 int osc_status(int* raw, osc_stream_t stream) {
   DeviceState* ds = nullptr;
   int rc = device_state(&ds);

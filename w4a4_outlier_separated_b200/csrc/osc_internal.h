@@ -90,4 +90,7 @@ struct DensityParams {
 };
 cudaError_t launch_density(const DensityParams& p, cudaStream_t s);
 
+// one bounded wait on a barrier nothing signals: records a timeout in `status`
+cudaError_t launch_selftest_wait(int* status, unsigned long long limit_ns, cudaStream_t s);
+
 }  // namespace osc

@@ -56,6 +56,7 @@ def lib() -> ctypes.CDLL:
             "osc_quantize_grouped": ([P, i32, P, P, P, i32, i32, i32, P, i32, P, P, P, P], i32),
             "osc_linear_grouped": ([P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P], i32),
             "osc_status": ([P, P], i32),
+            "osc_selftest_timeout": ([i32, P], i32),
             "osc_set_tile_n": ([i32], i32),
             "osc_set_cta_pair": ([i32], i32),
         }
@@ -202,6 +203,11 @@ def osc_linear_grouped(QX, SX, B, QW, SW, WL, mblock_expert, kl, E: int, Mp: int
                                                           _ptr(SW), _ptr(WL) if K_L else None, _ptr(mblock_expert),
                                                           _ptr(kl), E, Mp, N, K, G, K_L, _ptr(Y), _ptr(Yf32),
                                                           _stream(stream)))
+
+
+def osc_selftest_timeout(limit_us: int = 10000, stream=None):
+    """Launch the failure-detection self-test: a bounded wait that runs out after limit_us."""
+    _check("osc_selftest_timeout", lib().osc_selftest_timeout(limit_us, _stream(stream)))
 
 
 def osc_status(stream=None):
