@@ -23,7 +23,12 @@
  *     A call with zero rows (M = 0) does nothing and returns OSC_OK; its pointers may be NULL.
  *     Errors found by a kernel while it runs (a table entry >= G, more entries than K_L,
  *     a bounded wait that ran out) are recorded in a per-device status word that
- *     osc_status() reads and clears.
+ *     osc_status() reads and clears. The word is shared by every stream and host thread
+ *     using the device in this process; it keeps the first error recorded since it was last
+ *     cleared. After OSC_ERR_TIMEOUT, every output written since the last clean osc_status
+ *     is undefined (the kernel that ran out stopped part way and returned).
+ *   - osc_set_tile_n and osc_set_cta_pair change process-wide launch choices; they are
+ *     tuning and test knobs, not meant to be flipped while other threads issue calls.
  *
  * Shapes: X is M x K bf16 row-major (tokens x input channels); W is N x K bf16 row-major
  * (output x input channels, the layout of a PyTorch Linear weight); Y is M x N bf16.
@@ -185,8 +190,10 @@ OSC_API int osc_linear_grouped(const uint8_t* QX, const uint8_t* SX, const uint1
                        const int* mblock_expert, const int* kl, int E, int Mp, int N, int K,
                        int G, int K_L, uint16_t* Y, float* Yf32, osc_stream_t stream);
 
-/* Reads and clears the current device's status word (synchronizes `stream`). Returns
- * OSC_OK, OSC_ERR_TIMEOUT or OSC_ERR_TABLE; *raw (may be NULL) gets the raw device code. */
+/* Reads and clears the current device's status word in one atomic exchange on `stream`, then
+ * synchronizes `stream`. Returns OSC_OK, OSC_ERR_TIMEOUT or OSC_ERR_TABLE; *raw (may be NULL)
+ * gets the raw device code. An error that a kernel on another stream records while this call
+ * runs is either returned by it or kept for the next call. */
 OSC_API int osc_status(int* raw, osc_stream_t stream);
 
 /* Failure-detection self-test (not part of the OSC method): launches one kernel whose bounded

@@ -16,6 +16,9 @@ def _layer(G=32, K=512, N=48, K_L=16, seed=0):
     from w4a4_outlier_separated_b200 import osc
     rng = np.random.default_rng(seed)
     L = torch.from_numpy(rng.integers(-1, G, size=K // G).astype(np.int8))
+    if K_L == 0:
+        L[:] = -1                                             # no compensation columns, no entries
+    assert osc.osc_table_kl(L.numpy()) <= K_L
     QW = torch.from_numpy(rng.integers(0, 256, size=(N, K // 2)).astype(np.uint8))
     SW = torch.from_numpy(rng.integers(0, 256, size=osc.osc_scale_bytes(N, K, G)).astype(np.uint8))
     WL = torch.from_numpy(rng.integers(-30000, 30000, size=(N, K_L)).astype(np.int16)) if K_L else None
@@ -68,3 +71,32 @@ def test_damaged_or_mismatched_files_are_rejected(tmp_path):
         A.load_layer(str(bad), device="cpu")
     with pytest.raises(ValueError, match="QW"):
         A.save_layer(p, d["L"], d["QW"][:10], d["SW"], d["WL"], G=32, K=512, N=48, K_L=16)
+
+
+def test_tables_that_do_not_fit_the_layer_are_rejected(tmp_path):
+    """Entries outside [-1, G) or more entries than K_L columns hold: refused on save, and on
+    load of a file whose table bytes were changed after saving."""
+    d = _layer()
+    p = str(tmp_path / "layer.osc")
+    bad_entry = d["L"].clone()
+    bad_entry[3] = 32                                         # channel >= G
+    with pytest.raises(ValueError, match="entries must lie"):
+        A.save_layer(p, bad_entry, d["QW"], d["SW"], d["WL"], G=32, K=512, N=48, K_L=16)
+    many = torch.arange(16, dtype=torch.int8)                 # 16 entries need K_L = 16 ...
+    few = _layer(G=32, K_L=0)                                 # ... but this layer has K_L = 0
+    with pytest.raises(ValueError, match="more than K_L"):
+        A.save_layer(p, many, few["QW"], few["SW"], None, G=32, K=512, N=48, K_L=0)
+    A.save_layer(p, d["L"], d["QW"], d["SW"], d["WL"], G=32, K=512, N=48, K_L=16)
+    raw = bytearray(open(p, "rb").read())
+    raw[72 + 2] = 0x7F                                         # entry 127 >= G in the stored table
+    bad = tmp_path / "bad.osc"
+    bad.write_bytes(bytes(raw))
+    with pytest.raises(ValueError, match="entries must lie"):
+        A.load_layer(str(bad), device="cpu")
+    d0 = _layer(G=32, K_L=0)
+    A.save_layer(p, d0["L"], d0["QW"], d0["SW"], None, G=32, K=512, N=48, K_L=0)
+    raw = bytearray(open(p, "rb").read())
+    raw[72] = 5                                               # one entry, but K_L = 0 in the header
+    bad.write_bytes(bytes(raw))
+    with pytest.raises(ValueError, match="more than K_L"):
+        A.load_layer(str(bad), device="cpu")

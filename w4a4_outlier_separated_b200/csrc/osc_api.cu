@@ -18,6 +18,11 @@ std::atomic<int> g_tile_n{0};
 std::atomic<int> g_pair{-1};   // -1 automatic, 1 single CTAs, 2 CTA pairs
 
 __device__ int g_status_word;   // per-device error word written by the kernels
+__device__ int g_status_taken;  // where osc_status's exchange leaves the word's old value
+
+// Reads and clears the status word in one atomic step, so an error recorded by a kernel on
+// another stream is either returned now or left for the next read, never lost in between.
+__global__ void status_take_kernel() { g_status_taken = atomicExch(&g_status_word, 0); }
 
 constexpr int kMaxDevices = 64;
 
@@ -26,6 +31,8 @@ struct DeviceState {
   bool sm100 = false;
   int sms = 0;
   int* status = nullptr;
+  int* taken = nullptr;   // device address of g_status_taken
+  std::mutex status_mu;   // one osc_status at a time per device in this process
 };
 
 int fail_cuda(cudaError_t e) {
@@ -48,10 +55,13 @@ int device_state(DeviceState** out) {
     if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return fail_cuda(e);
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return fail_cuda(e);
     void* addr = nullptr;
+    void* taken = nullptr;
     if ((e = cudaGetSymbolAddress(&addr, g_status_word)) != cudaSuccess) return fail_cuda(e);
+    if ((e = cudaGetSymbolAddress(&taken, g_status_taken)) != cudaSuccess) return fail_cuda(e);
     s.sm100 = (major == 10);
     s.sms = sms;
     s.status = static_cast<int*>(addr);
+    s.taken = static_cast<int*>(taken);
     s.ready = true;
   }
   if (!s.sm100) return OSC_ERR_DEVICE;
@@ -401,7 +411,7 @@ int osc_quantize_grouped(const uint16_t* X, int E, const int* off, const int* po
   if ((long long)(Mp + 127) * (K / 32) >= (1LL << 31)) return OSC_ERR_ARG;
   if (!a16(X) || !a16(QX) || !a16(SX) || (B && !a16(B))) return OSC_ERR_ALIGN;
   if (K % 256 != 0 || K_L % 16 != 0 || Mp % 128 != 0) return OSC_ERR_ALIGN;
-  if (osc::grouped_quant_smem(E, K / G) > 200 * 1024) return OSC_ERR_ARG;   // E x K/G table entries
+  if (osc::grouped_quant_smem(E, K / G) > (size_t)osc::GROUPED_QUANT_SMEM_MAX) return OSC_ERR_ARG;   // E x K/G table entries
   DeviceState* ds = nullptr;
   int rc = device_state(&ds);
   if (rc != OSC_OK) return rc;
@@ -443,9 +453,10 @@ int osc_status(int* raw, osc_stream_t stream) {
   int rc = device_state(&ds);
   if (rc != OSC_OK) return rc;
   int v = 0;
-  cudaError_t e = cudaMemcpyAsync(&v, ds->status, sizeof(int), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
-  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
-  if (e == cudaSuccess) e = cudaMemsetAsync(ds->status, 0, sizeof(int), (cudaStream_t)stream);
+  std::lock_guard<std::mutex> lock(ds->status_mu);
+  status_take_kernel<<<1, 1, 0, (cudaStream_t)stream>>>();
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&v, ds->taken, sizeof(int), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return fail_cuda(e);
   if (raw) *raw = v;

@@ -143,26 +143,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 // ---- tcgen05 --------------------------------------------------------------------------------
 
-__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(dst_smem), "r"(ncols));
-}
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols));
-}
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// Arrive on an mbarrier once every tcgen05 op issued so far by this thread has completed.
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
-}
-
 // Shared-memory matrix descriptor (tcgen05 format): start>>4 in [0,14), leading byte
 // offset>>4 in [16,30), stride byte offset>>4 in [32,46), version 1 at bit 46, layout type
 // in [61,64) (0 = no swizzle, 2 = 128-byte swizzle).
@@ -176,54 +162,6 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t addr) { return sm
 // 32 rows x 16 bytes, contiguous, no swizzle: the source of a 32x128b scale copy.
 __device__ __forceinline__ uint64_t desc_scale_atom(uint32_t addr) { return smem_desc(addr, 0, 128, 0); }
 
-// Copy one 512-byte scale atom (32 rows x 16 bytes) into 4 TMEM columns, replicated to all
-// four 32-lane quadrants.
-__device__ __forceinline__ void tc_cp_scale_atom(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
-}
-
-// D(tmem) (+)= A(smem) * B(smem)^T with per-32 (block32) E8M0 scales from TMEM, E2M1 operands.
-__device__ __forceinline__ void tc_mma_mxf4_b32(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                                uint32_t sfa, uint32_t sfb, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-      :: "r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb) : "memory");
-}
-// Same with per-16 scales (block16).
-__device__ __forceinline__ void tc_mma_mxf4_b16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                                uint32_t sfa, uint32_t sfb, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-      :: "r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb) : "memory");
-}
-// E4M3 x E4M3 with per-32 E8M0 scales.
-__device__ __forceinline__ void tc_mma_mxf8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                            uint32_t sfa, uint32_t sfb, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-      :: "r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb) : "memory");
-}
-// BF16 x BF16 -> F32 (the compensation path).
-__device__ __forceinline__ void tc_mma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      :: "r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
-}
-
-// Instruction descriptors (M = 128, K-major A and B).
-// Block-scaled kinds: b_sf_id [4,6), a/b format [7,10)/[10,13), N>>3 [17,23), scale format
-// [23] (1 = E8M0), M>>4 [24,29), a_sf_id [29,31).
-__host__ __device__ constexpr uint32_t idesc_block_scaled(uint32_t fmt, uint32_t n, uint32_t sfa_id, uint32_t sfb_id) {
-  return (sfb_id << 4) | (fmt << 7) | (fmt << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24) | (sfa_id << 29);
-}
-// kind::f16 with BF16 inputs and F32 accumulate: c format [4,6) = 1, a/b format = 1.
-__host__ __device__ constexpr uint32_t idesc_bf16(uint32_t n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
-}
 constexpr uint32_t FMT_MXF4_E2M1 = 1;   // E2M1 in the mxf4 / mxf4nvf4 kinds
 constexpr uint32_t FMT_F8_E4M3 = 0;     // E4M3 in the mxf8f6f4 kind
 

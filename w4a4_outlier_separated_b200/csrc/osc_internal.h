@@ -4,8 +4,27 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <algorithm>
+#include <mutex>
 
 namespace osc {
+
+// One-time, per-device set-up (a kernel attribute) that any number of host threads may reach
+// at once: `f` runs once for each device, with that device current, and every caller on that
+// device gets the first run's result.
+struct PerDeviceOnce {
+  static constexpr int kMaxDevices = 64;
+  std::once_flag flag[kMaxDevices];
+  cudaError_t result[kMaxDevices] = {};
+  template <class F>
+  cudaError_t run(F f) {
+    int dev = 0;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::call_once(flag[dev], [&] { result[dev] = f(); });
+    return result[dev];
+  }
+};
 
 struct QuantParams {
   const uint16_t* X;   // M x K bf16
@@ -39,8 +58,9 @@ struct GroupedQuantParams {
   int* status;
 };
 cudaError_t launch_quantize_grouped(const GroupedQuantParams& p, int num_sms, cudaStream_t s);
-// shared memory the grouped quantize needs to stage every expert's table
+// shared memory the grouped quantize needs to stage every expert's table, and its limit
 size_t grouped_quant_smem(int E, int Kg);
+constexpr int GROUPED_QUANT_SMEM_MAX = 200 * 1024;
 cudaError_t launch_gather_wl(const uint16_t* W, int N, int K, int G, const int8_t* L, int K_L, uint16_t* WL,
                              int* status, int num_sms, cudaStream_t s);
 

@@ -11,7 +11,7 @@
 // The same kernel serves the MXFP8 fallback of §4 (E4M3 x E4M3, per-32 E8M0) and the
 // per-expert grouped form for MoE layers.
 //
-// Structure: persistent CTAs (one per SM), 8 warps.
+// Structure: persistent CTAs (one per SM), 12 warps.
 //   warp 0 (one lane)   TMA producer: operand tiles (128B swizzle) and scale atoms
 //   warp 1 (one lane)   MMA issuer: tcgen05.mma, tcgen05.commit
 //   warp 2              TMEM allocator, then (one lane) scale copier of odd stages
@@ -395,16 +395,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 template <int BN, int KIND, int CG>
 static cudaError_t launch_one(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t s) {
   using C = GemmCfg<BN, KIND, CG>;
-  static int attr_done[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, KIND, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_TOTAL);
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = 1;
-  }
+  static PerDeviceOnce smem_attr;
+  const cudaError_t ae = smem_attr.run([] {
+    return cudaFuncSetAttribute(gemm_kernel<BN, KIND, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_TOTAL);
+  });
+  if (ae != cudaSuccess) return ae;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(GEMM_THREADS, 1, 1);

@@ -456,14 +456,11 @@ constexpr int QSMEM = QWARPS * 2 * QSTEP * 64 + 1024;
 
 template <int G, bool FP8, bool TABLE>
 static cudaError_t launch_quant(const CUtensorMap& tmX, const QuantParams& p, int grid, cudaStream_t s) {
-  static int attr_done[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(quantize_tma_kernel<G, FP8, TABLE>, cudaFuncAttributeMaxDynamicSharedMemorySize, QSMEM);
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = 1;
-  }
+  static PerDeviceOnce smem_attr;
+  const cudaError_t ae = smem_attr.run([] {
+    return cudaFuncSetAttribute(quantize_tma_kernel<G, FP8, TABLE>, cudaFuncAttributeMaxDynamicSharedMemorySize, QSMEM);
+  });
+  if (ae != cudaSuccess) return ae;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(256, 1, 1);
@@ -508,18 +505,25 @@ size_t grouped_quant_smem(int E, int Kg) {
 cudaError_t launch_quantize_grouped(const GroupedQuantParams& p, int num_sms, cudaStream_t s) {
   if (p.Mp == 0) return cudaSuccess;
   const size_t smem = grouped_quant_smem(p.E, p.Kg);
-  if (smem > 200 * 1024) return cudaErrorInvalidValue;
+  if (smem > GROUPED_QUANT_SMEM_MAX) return cudaErrorInvalidValue;
   const long long items = (long long)p.Mp * (p.K / 32);
   const int grid = (int)std::max<long long>(1, std::min<long long>((items + 255) / 256, (long long)num_sms * 4));
+  // the attribute is raised once per device to the largest table size the entry point accepts,
+  // so no later call with more experts needs a new setting
+  static PerDeviceOnce attr[3];
+  auto raise = [](auto kern) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GROUPED_QUANT_SMEM_MAX);
+  };
+  cudaError_t e;
   switch (p.G) {
     case 16:
-      if (smem > 48 * 1024) cudaFuncSetAttribute(quantize_grouped_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if ((e = attr[0].run([&] { return raise(quantize_grouped_kernel<16>); })) != cudaSuccess) return e;
       quantize_grouped_kernel<16><<<grid, 256, smem, s>>>(p); break;
     case 32:
-      if (smem > 48 * 1024) cudaFuncSetAttribute(quantize_grouped_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if ((e = attr[1].run([&] { return raise(quantize_grouped_kernel<32>); })) != cudaSuccess) return e;
       quantize_grouped_kernel<32><<<grid, 256, smem, s>>>(p); break;
     case 64:
-      if (smem > 48 * 1024) cudaFuncSetAttribute(quantize_grouped_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if ((e = attr[2].run([&] { return raise(quantize_grouped_kernel<64>); })) != cudaSuccess) return e;
       quantize_grouped_kernel<64><<<grid, 256, smem, s>>>(p); break;
     default: return cudaErrorInvalidValue;
   }
