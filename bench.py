@@ -810,7 +810,40 @@ def main():
             res["scope_rows"] = scope_rows(min(args.steps, 50))
         if res["n_gpus"] == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(wl["X"], wl["W"], wl["calib"], args.cpu_seconds)
-        print(json.dumps(res), flush=True)
+        print(json.dumps(tail_order(res)), flush=True)
+
+
+def rows_brief(rows: dict) -> dict:
+    """One short list per measured row, [step us, linear fraction of its roofline, quantize
+    fraction of HBM], plus the Table 2 ratios: the per-row figures in a form that fits the end
+    of the line."""
+    out = {}
+    for k, r in rows.items():
+        if isinstance(r, dict) and "ms_per_step" in r:
+            out[k] = [round(r["ms_per_step"] * 1e3, 1), r["linear_roofline_frac"], r["quantize_hbm_frac"]]
+        elif isinstance(r, dict) and "error" in r:
+            out[k] = "error"
+    if "table2_osc_speedup_over_w8a8" in rows:
+        out["table2"] = rows["table2_osc_speedup_over_w8a8"]
+    return out
+
+
+def tail_order(res: dict) -> dict:
+    """The same line with the per-kernel figures moved to its end: the long per-row detail
+    and the CPU baseline come first, then a compact per-row summary, the headline kernels'
+    own numbers and the weight-bound lines, so that a reader of the line's last ~1.5 kB
+    (a log tail) still sees every kernel's throughput."""
+    out = {k: v for k, v in res.items() if k not in ("kernels", "weight_bound")}
+    if "scope_rows" in res:
+        out["rows_brief"] = rows_brief(res["scope_rows"])
+    if "kernels" in res:
+        out["kernels"] = res["kernels"]
+    if "weight_bound" in res:
+        wb = res["weight_bound"]
+        out["weight_bound"] = {"unit": wb["unit"], "peak": wb["peak"],
+                               "lines": [[d["M"], d["us"], d["GBps"], d["frac"]] for d in wb["lines"]],
+                               "columns": ["M", "us", "GB/s", "frac"], "what": wb["what"]}
+    return out
 
 
 if __name__ == "__main__":

@@ -91,3 +91,13 @@ def test_same_seed_same_arrays():
     a, b = I.qkv_case(64), I.qkv_case(64)
     assert np.array_equal(a.X, b.X) and np.array_equal(a.W, b.W) and np.array_equal(a.calib, b.calib)
     assert not np.array_equal(I.gen_weights(8, 256, seed=1), I.gen_weights(8, 256, seed=2))
+
+
+def test_block_rows_reach_every_block_edge():
+    """The parity row sampler covers the first and last row of every 128-row block (ragged
+    tail included), and nothing outside [0, M)."""
+    for M in (1, 127, 128, 129, 300, 3712):
+        r = I.block_rows(M, seed=M)
+        assert r.min() >= 0 and r.max() < M and np.all(np.diff(r) > 0)
+        for b0 in range(0, M, 128):
+            assert b0 in r and min(M, b0 + 128) - 1 in r

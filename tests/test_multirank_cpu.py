@@ -147,3 +147,25 @@ def test_clock_sampler_samples_while_the_timed_work_runs():
     c.samples = []
     c.sample_while(Event(1), 0.0)                    # work already done: still one sample
     assert len(c.samples) == 1
+
+
+def test_line_ends_with_the_kernel_figures():
+    """The printed line keeps every required key and ends with the compact per-row summary,
+    the headline kernels' figures and the weight-bound lines, so they fit a 1.5 kB log tail
+    even after a long per-row section."""
+    import json
+    import bench
+    row = {"ms_per_step": 0.0373, "linear_roofline_frac": 0.54, "quantize_hbm_frac": 0.46, "detail": "x" * 400}
+    res = {"metric": "m", "value": 1.0, "kernels": {"osc_quantize_GBps": 2950.0, "osc_quantize_hbm_frac": 0.46},
+           "weight_bound": {"unit": "GB/s", "peak": 6450.0, "what": "w",
+                            "lines": [{"M": m, "us": 9.9, "GBps": 1490.0, "frac": 0.23} for m in (1, 16, 128)]},
+           "roofline": {"frac": 0.5},
+           "scope_rows": {f"row{i}": dict(row) for i in range(12)} | {"table2_osc_speedup_over_w8a8": {"G32": 1.35}},
+           "cpu_baseline": {"value": 0.0035}}
+    out = bench.tail_order(res)
+    assert list(out)[-3:] == ["rows_brief", "kernels", "weight_bound"]
+    assert out["rows_brief"]["row3"] == [37.3, 0.54, 0.46] and out["rows_brief"]["table2"] == {"G32": 1.35}
+    line = json.dumps(out)
+    tail = line[-1500:]
+    assert '"osc_quantize_GBps": 2950.0' in tail and "[16, 9.9, 1490.0, 0.23]" in tail and '"row11"' in tail
+    assert {"metric", "value", "roofline", "scope_rows", "cpu_baseline"} <= set(out)

@@ -114,14 +114,16 @@ def pad16(n: int) -> int:
     return (n + 15) // 16 * 16
 
 
-def sample_rows(M: int, n: int, seed: int) -> np.ndarray:
-    """Sorted row sample for parity checks: first, last, tail rows and a seeded draw."""
-    if M <= n:
-        return np.arange(M, dtype=np.int32)
+def block_rows(M: int, seed: int, block: int = 128) -> np.ndarray:
+    """Sorted rows for parity checks that reach every `block`-row block of M rows: each
+    block's first and last row and one seeded row inside it (so every output tile row block,
+    and both CTAs of a 256-row CTA-pair tile, is checked at its edges)."""
     rng = np.random.default_rng(seed)
-    pick = {0, M - 1, (M // 128) * 128 - 1 if M >= 128 else 0, M - 2}
-    pick.update(int(v) for v in rng.choice(M, size=n, replace=False))
-    return np.array(sorted(p for p in pick if 0 <= p < M)[: max(n, 4)], dtype=np.int32)
+    pick = set()
+    for b0 in range(0, M, block):
+        b1 = min(M, b0 + block) - 1
+        pick.update((b0, b1, int(rng.integers(b0, b1 + 1))))
+    return np.array(sorted(pick), dtype=np.int32)
 
 
 # ---- the named workloads ------------------------------------------------------
