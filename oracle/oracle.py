@@ -60,6 +60,9 @@ def lib():
         L.orc_bf16_to_double.restype = ctypes.c_double
         L.orc_double_to_bf16.argtypes = [ctypes.c_double]
         L.orc_double_to_bf16.restype = ctypes.c_uint16
+        L.orc_row_sumsq.argtypes = [P, i32]
+        L.orc_row_sumsq.restype = ctypes.c_float
+        L.orc_rmsnorm.argtypes = [P, i32, i32, P, f32, P, P]
         _ = (i64,)
         _lib = L
     return _lib
@@ -200,6 +203,24 @@ def to_bf16_array(Y: np.ndarray) -> np.ndarray:
     return out
 
 
+def row_sumsq(x: np.ndarray) -> float:
+    """fp32 sum of squares of one bf16 row, in the order the RMSNorm reading fixes."""
+    x = np.ascontiguousarray(x, dtype=np.uint16).reshape(-1)
+    return float(lib().orc_row_sumsq(_p(x), x.size))
+
+
+def rmsnorm(X: np.ndarray, gamma: np.ndarray, eps: float = 1e-6):
+    """RMSNorm of each row (the producer step before the quantize): returns (Y bf16 bits,
+    inv_rms fp32 per row)."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    gamma = np.ascontiguousarray(gamma, dtype=np.uint16).reshape(-1)
+    M, K = X.shape
+    Y = np.empty_like(X)
+    inv = np.empty(M, dtype=np.float32)
+    _chk(lib().orc_rmsnorm(_p(X), M, K, _p(gamma), float(eps), _p(Y), _p(inv)), "rmsnorm")
+    return Y, inv
+
+
 # ---- the whole OSC layer, step by step -----------------------------------------
 
 def osc_prepare_weight(W: np.ndarray, G: int, L: np.ndarray, K_L: int):
@@ -216,6 +237,15 @@ def osc_forward(X: np.ndarray, G: int, L: np.ndarray, K_L: int, cw, ew, WL, rows
     cx, ex = mx_quantize(Xz, G, FMT_E2M1)
     Y = linear(cx, ex, cw, ew, B if K_L else None, WL if K_L else None, FMT_E2M1, rows)
     return dict(Xz=Xz, B=B, cx=cx, ex=ex, Y=Y)
+
+
+def rmsnorm_osc_forward(X: np.ndarray, gamma: np.ndarray, eps: float, G: int, L: np.ndarray, K_L: int,
+                        cw, ew, WL, rows=None):
+    """The producer-fused input side: RMSNorm, then the online OSC path on its output."""
+    Yn, _ = rmsnorm(X, gamma, eps)
+    out = osc_forward(Yn, G, L, K_L, cw, ew, WL, rows)
+    out["Xn"] = Yn
+    return out
 
 
 def fp8_forward(X: np.ndarray, W: np.ndarray, rows=None):

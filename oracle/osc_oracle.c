@@ -221,6 +221,76 @@ int orc_gather_wl(const uint16_t* W, int N, int K, int G, const int8_t* L,
     return 0;
 }
 
+/* ---- The producer step before the quantize: RMSNorm --------------------------
+ *
+ * Figure 2 (§3.2) places extraction and microscaling directly before the GEMM; in
+ * the Qwen3 layers the page measures (§1, §5.2) the activations that reach the QKV
+ * and FFN up/gate projections come straight out of an RMSNorm. The page does not
+ * describe that step; READING (the usual RMSNorm, with its order of operations fixed
+ * so that both sides reach the same bits), for one row x of K bf16 values, weight
+ * gamma (K bf16 values) and eps, all in fp32 with every operation rounded to
+ * nearest even:
+ *   s_b    = x_{32b}^2 + x_{32b+1}^2 + ... + x_{32b+31}^2, added in ascending
+ *            order, one sum per 32-channel block b = 0 .. K/32 - 1;
+ *   total  the block sums padded with zeros to a power of two P and combined
+ *            pairwise: for h = P/2, P/4, ..., 1: s_b <- s_b + s_{b+h} (b < h);
+ *            total = s_0;
+ *   inv    = 1 / sqrt(total / K + eps);
+ *   y_j    = bf16( (x_j * inv) * gamma_j ).
+ * The normalized row y then goes through extraction and microscaling unchanged.
+ */
+static float f32_of_bf16(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Sum of squares of one row in the stated order. */
+float orc_row_sumsq(const uint16_t* x, int K)
+{
+    int nb = K / 32, P = 1;
+    while (P < nb) P *= 2;
+    float* s = (float*)calloc((size_t)P, sizeof(float));
+    if (!s) return NAN;
+    for (int b = 0; b < nb; ++b) {
+        float acc = 0.0f;
+        for (int j = 0; j < 32; ++j) {
+            float v = f32_of_bf16(x[b * 32 + j]);
+            float sq = v * v;
+            acc = acc + sq;
+        }
+        s[b] = acc;
+    }
+    for (int h = P / 2; h >= 1; h /= 2)
+        for (int b = 0; b < h; ++b) s[b] = s[b] + s[b + h];
+    float total = s[0];
+    free(s);
+    return total;
+}
+
+int orc_rmsnorm(const uint16_t* X, int M, int K, const uint16_t* gamma, float eps,
+                uint16_t* Y, float* inv_out)
+{
+    if (!X || !gamma || !Y || M < 0 || K <= 0 || K % 32 != 0 || !(eps >= 0.0f)) return -1;
+    if (!all_finite_bf16(X, (int64_t)M * K) || !all_finite_bf16(gamma, K)) return -1;
+    for (int t = 0; t < M; ++t) {
+        const uint16_t* x = X + (int64_t)t * K;
+        float total = orc_row_sumsq(x, K);
+        float mean = total / (float)K;
+        float root = sqrtf(mean + eps);
+        float inv = 1.0f / root;
+        if (inv_out) inv_out[t] = inv;
+        for (int j = 0; j < K; ++j) {
+            float a = f32_of_bf16(x[j]) * inv;
+            float b = a * f32_of_bf16(gamma[j]);
+            Y[(int64_t)t * K + j] = orc_double_to_bf16((double)b);
+        }
+    }
+    return 0;
+}
+
 /* ---- Microscaling (§3.2, the dynamic-range step) ------------------------------
  *
  * After the table channels are zeroed the page rescales each group with its

@@ -136,6 +136,28 @@ MUTANTS = [
     ("weights_decoded_as_e2m1", "c",
      "qw[k] = (fmt == ORC_FMT_E2M1) ? orc_decode_e2m1(c) : orc_decode_e4m3(c);",
      "qw[k] = orc_decode_e2m1(c);"),
+    # the RMSNorm step before the quantize (its order of operations is a stated reading)
+    ("rms_sum_left_to_right_over_blocks", "c",
+     "for (int h = P / 2; h >= 1; h /= 2)\n        for (int b = 0; b < h; ++b) s[b] = s[b] + s[b + h];",
+     "for (int b = 1; b < P; ++b) s[0] = s[0] + s[b];"),
+    ("rms_block_summed_descending", "c",
+     "float v = f32_of_bf16(x[b * 32 + j]);",
+     "float v = f32_of_bf16(x[b * 32 + 31 - j]);"),
+    ("rms_mean_over_blocks", "c",
+     "float mean = total / (float)K;",
+     "float mean = total / (float)(K / 32);"),
+    ("rms_eps_outside_sqrt", "c",
+     "float root = sqrtf(mean + eps);",
+     "float root = sqrtf(mean) + eps;"),
+    ("rms_gamma_dropped", "c",
+     "float b = a * f32_of_bf16(gamma[j]);",
+     "float b = a;"),
+    ("rms_gamma_reversed", "c",
+     "float b = a * f32_of_bf16(gamma[j]);",
+     "float b = a * f32_of_bf16(gamma[K - 1 - j]);"),
+    ("rms_quantizes_raw_rows", "py",
+     "out = osc_forward(Yn, G, L, K_L, cw, ew, WL, rows)",
+     "out = osc_forward(X, G, L, K_L, cw, ew, WL, rows)"),
     # the step order of the layer (oracle.py)
     ("quantize_before_extraction", "py",
      "cx, ex = mx_quantize(Xz, G, FMT_E2M1)",

@@ -465,3 +465,105 @@ def test_group_size_sweep_roundtrip(oracle):
         cw0, ew0, _ = oracle.osc_prepare_weight(Wsmall, G, L0, 0)
         r0 = oracle.osc_forward(c.X, G, L0, 0, cw0, ew0, None)
         assert np.abs(r["Y"] - ref).mean() < 0.8 * np.abs(r0["Y"] - ref).mean()
+
+
+# ---- the producer step before the quantize (RMSNorm; the reading fixes its order) ----------
+
+def _bf16_row(vals):
+    return I.bf16_bits(np.asarray(vals, dtype=np.float64))
+
+
+def test_rmsnorm_sum_order_closed_forms(oracle):
+    """Totals worked out by hand in fp32 (ties to even; the spacing of fp32 at 2^24 is 2).
+    Row A: 4096 then 31 ones in block 0, then seven blocks of 32 ones: in ascending order
+    every 1 added to 2^24 is a tie that rounds back to 2^24, so block 0 sums to 2^24, the
+    other blocks to 32 each, and the pairwise combination gives 2^24 + 224 exactly (a plain
+    left-to-right sum over the row would lose every 1 and give 2^24; block 0 summed in
+    descending order would give 2^24 + 32 for that block).
+    Row B: 4096 alone in block 0, a single 1 in each of blocks 1..7: pairwise, 2^24 + 1 ties
+    back to 2^24, then 2^24 + 2 and 2^24 + 6 are exact; left to right over the block sums
+    every 1 ties back to 2^24."""
+    a = np.ones(256)
+    a[0] = 4096.0
+    assert oracle.row_sumsq(_bf16_row(a)) == 16777216.0 + 224.0
+    b = np.zeros(256)
+    b[0] = 4096.0
+    b[32::32] = 1.0
+    assert oracle.row_sumsq(_bf16_row(b)) == 16777216.0 + 6.0
+
+
+@pytest.mark.parametrize("K", [256, 768, 4096])
+def test_rmsnorm_sum_within_fp32_bound(oracle, K):
+    """On random rows (K/32 not always a power of two) the fp32 total stays within the error
+    bound of its additions, (31 + log2 P) * 2^-24 relative, of the exact sum of squares."""
+    import math
+    rng = np.random.default_rng(K)
+    for scale in (1.0, 1e-3, 300.0):
+        x = I.bf16_bits(rng.standard_normal(K) * scale)
+        v = I.bf16_to_f32(x).astype(np.float64)
+        exact = math.fsum(float(t) * float(t) for t in v)      # each square is exact in fp64
+        depth = 31 + math.ceil(math.log2(K // 32))
+        assert abs(oracle.row_sumsq(x) - exact) <= depth * 2.0 ** -24 * exact
+
+
+def test_rmsnorm_constant_rows_give_unit_output(oracle):
+    """A row of one repeated value c (gamma = 1, eps = 0) normalizes to sign(c) * 1 exactly
+    in bf16: its root mean square is |c|."""
+    rng = np.random.default_rng(11)
+    c = rng.choice([-1, 1], 40) * np.exp2(rng.uniform(-30, 30, 40))
+    X = I.bf16_bits(np.repeat(c[:, None], 512, axis=1))
+    Y, _ = oracle.rmsnorm(X, np.full(512, 0x3F80, np.uint16), 0.0)
+    assert np.array_equal(Y, np.where(c[:, None] < 0, 0xBF80, 0x3F80).astype(np.uint16) * np.ones((1, 512), np.uint16))
+
+
+def test_rmsnorm_scale_invariance(oracle):
+    """Scaling a row by 2^k scales every square and sum exactly and the root by 2^k, so with
+    eps = 0 the normalized row is bit-identical and the inverse root scales by 2^-k."""
+    c = I.qkv_case(8)
+    X = c.X[:, :1024]
+    gamma = I.bf16_bits(1.0 + 0.1 * np.random.default_rng(2).standard_normal(1024))
+    Y0, inv0 = oracle.rmsnorm(X, gamma, 0.0)
+    for k in (-20, -3, 5, 17):
+        Xk = I.bf16_bits(I.bf16_to_f32(X).astype(np.float64) * 2.0 ** k)
+        Yk, invk = oracle.rmsnorm(Xk, gamma, 0.0)
+        assert np.array_equal(Yk, Y0), k
+        assert np.array_equal(invk.astype(np.float64), inv0.astype(np.float64) * 2.0 ** -k), k
+
+
+def test_rmsnorm_matches_the_fp64_definition(oracle):
+    """Against x / sqrt(mean(x^2) + eps) * gamma computed in fp64 from the same bf16 inputs:
+    within one bf16 ulp (the fp32 steps add a few fp32 ulps before the final rounding). A row of
+    tiny values, where eps dominates the mean, pins where eps enters."""
+    from tests._layout import bf16_ulp
+    rng = np.random.default_rng(5)
+    c = I.qkv_case(16)
+    X = np.concatenate([c.X, I.bf16_bits(rng.standard_normal((2, 4096)) * 1e-4)], axis=0)
+    gamma = I.bf16_bits(1.0 + 0.2 * rng.standard_normal(4096))
+    for eps in (1e-6, 1e-2):
+        Y, _ = oracle.rmsnorm(X, gamma, eps)
+        x = I.bf16_to_f32(X).astype(np.float64)
+        g = I.bf16_to_f32(gamma).astype(np.float64)
+        ref = x / np.sqrt((x * x).mean(axis=1, keepdims=True) + np.float64(np.float32(eps))) * g
+        y = I.bf16_to_f32(Y).astype(np.float64)
+        assert np.all(np.abs(y - ref) <= bf16_ulp(ref) + 1e-30), eps
+
+
+def test_rmsnorm_then_osc_is_osc_of_the_normalized_rows(oracle):
+    """The fused input side quantizes the normalized rows: rows that RMSNorm leaves unchanged
+    (every value +-1, gamma = 1, eps = 0) give exactly the plain OSC outputs, and scaling them
+    by 2^k changes nothing (the raw rows would get other scale exponents)."""
+    rng = np.random.default_rng(9)
+    K, G = 512, 32
+    X = I.bf16_bits(rng.choice([-1.0, 1.0], (6, K)))
+    W = I.gen_weights(64, K, seed=4)
+    L = np.full(K // G, -1, np.int8)
+    L[[1, 5, 9]] = [3, 0, 31]
+    K_L = 16
+    ones = np.full(K, 0x3F80, np.uint16)
+    cw, ew, WL = oracle.osc_prepare_weight(W, G, L, K_L)
+    plain = oracle.osc_forward(X, G, L, K_L, cw, ew, WL)
+    Xk = I.bf16_bits(I.bf16_to_f32(X).astype(np.float64) * 2.0 ** 9)
+    fused = oracle.rmsnorm_osc_forward(Xk, ones, 0.0, G, L, K_L, cw, ew, WL)
+    for key in ("cx", "ex", "B"):
+        assert np.array_equal(fused[key], plain[key]), key
+    assert np.array_equal(fused["Y"], plain["Y"])
