@@ -134,6 +134,18 @@ OSC_API int osc_select_tier(const int* n_hit, const int* n_total, int Kg, double
 OSC_API int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int K_L,
                  uint8_t* QX, uint8_t* SX, uint16_t* B, osc_stream_t stream);
 
+/* Figure 2 (§3.2) with the step that produces the projection's input: RMSNorm of each row,
+ * then the osc_quantize of the normalized row, in one pass over X (the normalized rows are
+ * never written out). X: M x K bf16 activations, gamma: K bf16 weights, eps >= 0. Per row, in
+ * fp32 with every operation rounded to nearest even: the squares of each 32-channel block
+ * summed in ascending order; the block sums padded with zeros to a power of two and combined
+ * pairwise (s_b += s_{b+h}, h = P/2 .. 1); inv = 1 / sqrt(sum / K + eps); the normalized value
+ * bf16((x * inv) * gamma). Outputs and table arguments as osc_quantize (the table comes from
+ * calibration rows that were normalized the same way). K must be at most 6144. */
+OSC_API int osc_rmsnorm_quantize(const uint16_t* X, const uint16_t* gamma, float eps, int M, int K, int G,
+                                 const int8_t* L, int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B,
+                                 osc_stream_t stream);
+
 /* §3.3 weight side (offline): W (N x K bf16) -> QW (N x K/2), SW (osc_scale_bytes(N, K, G))
  * quantized with no table (its outlier columns meet zeroed activations), and
  * W_L (N x K_L bf16) gathered through L (device; may be NULL when K_L == 0). */

@@ -241,3 +241,91 @@ def test_density_bad_table_entry_is_reported(osc):
     torch.cuda.synchronize()
     assert osc.osc_status() == (-6, 2)
     assert to_np(nh)[5] == 0
+
+
+def _gamma(K, seed):
+    return I.bf16_bits(1.0 + 0.1 * np.random.default_rng(seed).standard_normal(K))
+
+
+def _check_rmsnorm_quant(oracle, osc, X, gamma, eps, G, L, K_L):
+    """osc_rmsnorm_quantize against the oracle's RMSNorm followed by extraction and
+    microscaling: codes, scales (pad rows zero) and B bit for bit, every row."""
+    M, K = X.shape
+    Ld = to_dev(L) if L is not None else None
+    QX, SX, B = osc.rmsnorm_quantize(to_dev(X), to_dev(gamma), eps, G, Ld, K_L)
+    torch.cuda.synchronize()
+    assert osc.osc_status() == (0, 0)
+    Xn, _ = oracle.rmsnorm(X, gamma, eps)
+    V = 16 if G == 16 else 32
+    SXn = to_np(SX)
+    assert pad_rows_zero(SXn, M, K, V)
+    if L is not None:
+        Xz, Bref = oracle.extract(Xn, G, L, K_L)
+        if K_L:
+            assert np.array_equal(to_np(B), Bref)
+    else:
+        Xz = Xn
+    cref, eref = oracle.mx_quantize(Xz, G)
+    codes = unpack_e2m1(to_np(QX), K)
+    bad = np.argwhere(codes != cref)
+    assert bad.size == 0, f"{len(bad)} code mismatches, first {bad[:4]}"
+    assert np.array_equal(unswizzle_scales(SXn, M, K, V), eref)
+
+
+@pytest.mark.parametrize("M", [1, 16, 130, 2048])
+def test_rmsnorm_quantize_qkv(oracle, osc, M):
+    """The fused input side at the QKV shape (K = 4096, G = 32), table by Algorithm 1 on
+    calibration rows normalized the same way."""
+    c = I.qkv_case(M)
+    gamma = _gamma(4096, 1)
+    L = oracle.build_table(oracle.rmsnorm(c.calib, gamma, 1e-6)[0], 32)
+    K_L = I.pad16(oracle.table_count(L))
+    _check_rmsnorm_quant(oracle, osc, c.X, gamma, 1e-6, 32, L, K_L)
+
+
+@pytest.mark.parametrize("G", [16, 64])
+def test_rmsnorm_quantize_group_sizes(oracle, osc, G):
+    c = I.qkv_case(256)
+    gamma = _gamma(4096, G)
+    L = oracle.build_table(oracle.rmsnorm(c.calib[:512], gamma, 1e-6)[0], G)
+    _check_rmsnorm_quant(oracle, osc, c.X, gamma, 1e-6, G, L, I.pad16(oracle.table_count(L)))
+
+
+@pytest.mark.parametrize("K", [256, 768, 1280, 2048, 6144])
+def test_rmsnorm_quantize_row_lengths(oracle, osc, K):
+    """Rows of 8 to 192 blocks: fewer blocks than lanes (K = 256, 768), a block count that is
+    not a power of two (1280, 6144: partial last pass of the lanes), and the largest K."""
+    rng = np.random.default_rng(K)
+    M, G = 130, 32
+    x = rng.standard_normal((M, K)) * np.exp2(rng.integers(-8, 8, (M, 1)))
+    L = np.full(K // G, -1, np.int8)
+    idx = rng.permutation(K // G)[: max(1, K // G // 2)]
+    L[idx] = rng.integers(0, G, idx.size)
+    for k, j in enumerate(L):
+        if j >= 0:
+            x[:, k * G + int(j)] *= 40.0
+    X = I.bf16_bits(x)
+    _check_rmsnorm_quant(oracle, osc, X, _gamma(K, K + 1), 1e-5, G, L, I.pad16(oracle.table_count(L)))
+
+
+def test_rmsnorm_quantize_edge_rows(oracle, osc):
+    """All-zero and negative-zero rows (eps > 0 keeps their scale finite), a constant row, rows
+    whose squares overflow or underflow fp32 (both sides follow IEEE fp32: an infinite sum
+    gives inv = 0), a negative and a zero gamma entry; with and without a table."""
+    rng = np.random.default_rng(8)
+    M, K = 9, 512
+    x = rng.standard_normal((M, K))
+    x[0] = 0.0
+    x[1] = -0.0
+    x[2] = 3.0
+    x[3] *= 2.0 ** 100                                        # squares overflow fp32: inv = 0
+    x[4] *= 2.0 ** -100                                       # squares underflow: eps decides
+    x[5] *= 2.0 ** 50
+    X = I.bf16_bits(x)
+    gamma = _gamma(K, 3)
+    gamma[7] = I.bf16_bits(np.array([-1.5]))[0]
+    gamma[9] = 0
+    _check_rmsnorm_quant(oracle, osc, X, gamma, 1e-6, 32, None, 0)
+    L = np.full(K // 32, -1, np.int8)
+    L[[0, 7, 15]] = [0, 31, 9]
+    _check_rmsnorm_quant(oracle, osc, X, gamma, 1e-6, 32, L, 16)

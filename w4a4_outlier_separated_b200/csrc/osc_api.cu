@@ -105,6 +105,12 @@ int make_block_map(CUtensorMap* m, const uint16_t* X, int rows, int K) {
   uint32_t box[2] = {32, (uint32_t)osc::QUANT_STEP_ITEMS};
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, d, st, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
+// The same view with one whole row per box (box {32, K/32}): the fused RMSNorm form.
+int make_row_map(CUtensorMap* m, const uint16_t* X, int rows, int K) {
+  uint64_t d[2] = {32, (uint64_t)rows * (uint64_t)(K / 32)}, st[1] = {64};
+  uint32_t box[2] = {32, (uint32_t)(K / 32)};
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, d, st, box, CU_TENSOR_MAP_SWIZZLE_64B);
+}
 inline bool valid_g(int G) { return G == 16 || G == 32 || G == 64; }
 
 int launch_result(cudaError_t e) { return e == cudaSuccess ? OSC_OK : fail_cuda(e); }
@@ -313,6 +319,28 @@ int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int K_
   CUtensorMap tm;
   if ((rc = make_block_map(&tm, X, M, K))) return rc;
   return launch_result(osc::launch_quantize(tm, p, false, ds->sms, (cudaStream_t)stream));
+}
+
+int osc_rmsnorm_quantize(const uint16_t* X, const uint16_t* gamma, float eps, int M, int K, int G, const int8_t* L,
+                         int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B, osc_stream_t stream) {
+  if (!valid_g(G)) return OSC_ERR_G;
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return OSC_ERR_ARG;
+  if (M == 0 && K > 0 && K_L >= 0) return OSC_OK;          // nothing to read or write
+  if (!X || !gamma || !QX || !SX || M < 0 || K <= 0 || K_L < 0) return OSC_ERR_ARG;
+  if (K > osc::NQ_MAX_K) return OSC_ERR_ARG;
+  if ((long long)(M + 127) * (K / 32) >= (1LL << 31)) return OSC_ERR_ARG;
+  if (L == nullptr && K_L != 0) return OSC_ERR_ARG;
+  if (L != nullptr && K_L > 0 && !B) return OSC_ERR_ARG;
+  if (K_L > 32767) return OSC_ERR_ARG;
+  if (!a16(X) || !a16(gamma) || !a16(QX) || !a16(SX) || (B && !a16(B))) return OSC_ERR_ALIGN;
+  if (K % 256 != 0 || K_L % 16 != 0) return OSC_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != OSC_OK) return rc;
+  osc::NormQuantParams p{X, gamma, eps, M, K, G, K / G, L, K_L, QX, SX, B, ds->status};
+  CUtensorMap tm;
+  if ((rc = make_row_map(&tm, X, M, K))) return rc;
+  return launch_result(osc::launch_rmsnorm_quantize(tm, p, ds->sms, (cudaStream_t)stream));
 }
 
 int osc_prepare_weight(const uint16_t* W, int N, int K, int G, const int8_t* L, int K_L, uint8_t* QW, uint8_t* SW,

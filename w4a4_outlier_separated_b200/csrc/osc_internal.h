@@ -44,6 +44,24 @@ constexpr int QUANT_STEP_ITEMS = 64;
 // (see make_block_map)
 cudaError_t launch_quantize(const CUtensorMap& tmX, const QuantParams& p, bool fp8, int num_sms, cudaStream_t s);
 
+// Producer-fused quantize: RMSNorm of each row, then the OSC quantize of the normalized row.
+struct NormQuantParams {
+  const uint16_t* X;       // M x K bf16
+  const uint16_t* gamma;   // K bf16
+  float eps;
+  int M, K, G, Kg;
+  const int8_t* L;         // Kg entries (device) or nullptr
+  int K_L;
+  uint8_t* Q;
+  uint8_t* S;
+  uint16_t* B;
+  int* status;
+};
+// largest K of the fused form: two row buffers per warp (2 K bytes each) and gamma in shared memory
+constexpr int NQ_MAX_K = 6144;
+// tmX: X as (32-channel blocks) x 64 bytes, box {32, K/32} (one row per box), 64-byte swizzle
+cudaError_t launch_rmsnorm_quantize(const CUtensorMap& tmX, const NormQuantParams& p, int num_sms, cudaStream_t s);
+
 struct GroupedQuantParams {
   const uint16_t* X;          // off[E] x K bf16, expert-sorted
   const int* off;             // E+1 (device)

@@ -212,11 +212,14 @@ __device__ int stage_table(const int8_t* __restrict__ L, int Kg, int K_L, int* t
 // One item = one 32-channel block of one row: extraction, amax, exponent(s), codes, scales.
 // All 32 lanes of a warp call it together (for G = 64 the two blocks of a group sit on
 // neighbouring lanes and meet by a shuffle); lanes hold consecutive blocks of a row.
+// `valid` false: the lane holds no block (a row with fewer blocks than the warp has lanes);
+// it still takes part in the G = 64 shuffle but writes nothing.
 template <int G, bool FP8, bool TABLE>
 __device__ __forceinline__ void quant_block(uint32_t (&w)[16], int row, int blk, bool live, const BlockTable& t,
                                             int count, int K, int K_L, uint16_t* __restrict__ B,
-                                            uint8_t* __restrict__ Q, uint8_t* __restrict__ S) {
+                                            uint8_t* __restrict__ Q, uint8_t* __restrict__ S, bool valid = true) {
   const int lane = threadIdx.x & 31;
+  live = live && valid;
   if constexpr (TABLE) {
     if (t.lw0 >= 0) {
       const uint16_t v = take_channel(w, t.lw0);
@@ -244,7 +247,7 @@ __device__ __forceinline__ void quant_block(uint32_t (&w)[16], int row, int blk,
       dst[0] = make_uint4(c[0], c[1], c[2], c[3]);
       dst[1] = make_uint4(c[4], c[5], c[6], c[7]);
     }
-    S[scale_byte_offset(row, blk, nblk / 4)] = (uint8_t)(e + 127);
+    if (valid) S[scale_byte_offset(row, blk, nblk / 4)] = (uint8_t)(e + 127);
   } else if constexpr (G == 16) {
     const int e0 = shared_exp<2>(block_amax<0, 8>(w));
     const int e1 = shared_exp<2>(block_amax<8, 8>(w));
@@ -252,8 +255,9 @@ __device__ __forceinline__ void quant_block(uint32_t (&w)[16], int row, int blk,
     const uint2 q1 = codes16<8>(w, pow2_neg_x2(e1));
     if (live) *reinterpret_cast<uint4*>(Q + (size_t)row * (K / 2) + (size_t)blk * 16) = make_uint4(q0.x, q0.y, q1.x, q1.y);
     // slots 2*blk and 2*blk + 1: two neighbouring bytes of one scale word
-    *reinterpret_cast<uint16_t*>(S + scale_byte_offset(row, 2 * blk, nblk / 2)) =
-        (uint16_t)((uint32_t)(e0 + 127) | ((uint32_t)(e1 + 127) << 8));
+    if (valid)
+      *reinterpret_cast<uint16_t*>(S + scale_byte_offset(row, 2 * blk, nblk / 2)) =
+          (uint16_t)((uint32_t)(e0 + 127) | ((uint32_t)(e1 + 127) << 8));
   } else {
     uint32_t am = block_amax<0, 16>(w);
     if constexpr (G == 64) am = max(am, __shfl_xor_sync(0xffffffffu, am, 1));
@@ -262,7 +266,7 @@ __device__ __forceinline__ void quant_block(uint32_t (&w)[16], int row, int blk,
     const uint2 q0 = codes16<0>(w, f2);
     const uint2 q1 = codes16<8>(w, f2);
     if (live) *reinterpret_cast<uint4*>(Q + (size_t)row * (K / 2) + (size_t)blk * 16) = make_uint4(q0.x, q0.y, q1.x, q1.y);
-    S[scale_byte_offset(row, blk, nblk / 4)] = (uint8_t)(e + 127);
+    if (valid) S[scale_byte_offset(row, blk, nblk / 4)] = (uint8_t)(e + 127);
   }
   (void)lane;
 }
@@ -412,6 +416,187 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
     }
     __syncwarp();                                             // every lane is done with this slot
     if (step + 2 * wstride < cta_end) { fence_proxy_async_smem(); issue(step + 2 * wstride, slot); }
+  }
+}
+
+// Producer-fused form: RMSNorm of each row, then extraction and MX quantization of the
+// normalized row, in one pass over X (Figure 2 of the OSC page puts extraction and
+// microscaling right before the GEMM; the RMSNorm that produces the projection's input is
+// the step before them). A warp owns a row: the row's sum of squares must be complete before
+// any block can be scaled. Rows arrive by one TMA box each ({32 channels, K/32 blocks}, the
+// 64-byte swizzle of the dense kernel) into a per-warp double buffer; gamma is staged once per
+// CTA in the same swizzle. Arithmetic, every step rounded to nearest even in fp32 with no
+// fused multiply-add: s_b = x_0^2 + ... + x_31^2 per 32-channel block in ascending order; the
+// block sums, padded with zeros to a power of two, combined pairwise (s_b += s_{b+h} for
+// h = P/2 .. 1); inv = 1 / sqrt(total / K + eps); y = bf16((x * inv) * gamma).
+constexpr int NQ_WARPS = 8;
+constexpr int NQ_PARTS = 8;                      // block sums per lane: a power of two >= NQ_MAX_K / 1024
+static_assert(NQ_PARTS * 1024 >= NQ_MAX_K && (NQ_PARTS & (NQ_PARTS - 1)) == 0, "block sums per lane");
+
+template <int G, bool TABLE>
+__global__ void __launch_bounds__(256, 1) rmsnorm_quantize_kernel(const __grid_constant__ CUtensorMap tmX, NormQuantParams p) {
+  extern __shared__ uint8_t nq_dyn[];
+  uint8_t* base = nq_dyn + ((1024u - (smem_u32(nq_dyn) & 1023u)) & 1023u);
+  const int nb = p.K / 32;                                   // 32-channel blocks per row
+  const uint32_t row_bytes = (uint32_t)p.K * 2u;
+  const uint32_t slot_bytes = (row_bytes + 1023u) & ~1023u;
+  uint8_t* gam = base;
+  auto row_buf = [&](int wp, int sl) { return base + slot_bytes * (1u + (uint32_t)(wp * 2 + sl)); };
+  __shared__ __align__(8) uint64_t s_bar[NQ_WARPS][2];
+  __shared__ __align__(8) int s_tab[TABLE ? MAX_KG : 2];
+  __shared__ int s_warp[8];
+  __shared__ int s_abort;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t mpad = (uint32_t)(p.M + 127) / 128u * 128u;
+  // CTA b takes a contiguous run of rows (one more for the first mpad % grid CTAs); its warps
+  // take the run's rows round robin
+  const uint32_t per = mpad / gridDim.x, extra = mpad % gridDim.x;
+  const uint32_t first = blockIdx.x * per + min(blockIdx.x, extra);
+  const uint32_t end = first + per + (blockIdx.x < extra ? 1u : 0u);
+  uint32_t row = first + warp;
+  if (threadIdx.x == 0) s_abort = 0;
+  if (lane == 0) { mbar_init(smem_u32(&s_bar[warp][0]), 1); mbar_init(smem_u32(&s_bar[warp][1]), 1); }
+  fence_barrier_init();
+  __syncwarp();
+  grid_dep_wait();                                           // X, gamma and L are free of the previous kernel
+  auto issue = [&](uint32_t r, int slot) {
+    if (lane == 0 && r < (uint32_t)p.M) {
+      const uint32_t bar = smem_u32(&s_bar[warp][slot]);
+      mbar_arrive_expect_tx(bar, row_bytes);
+      tma_load_2d(smem_u32(row_buf(warp, slot)), &tmX, 0, (int)(r * (uint32_t)nb), bar);
+    }
+  };
+  if (row < end) issue(row, 0);
+  if (row + NQ_WARPS < end) issue(row + NQ_WARPS, 1);
+  for (int i = threadIdx.x; i < nb * 4; i += blockDim.x) {  // gamma, 16-byte chunks, swizzled
+    const int b = i >> 2, c = i & 3;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.gamma) + i);
+    *reinterpret_cast<uint4*>(gam + b * 64 + ((c ^ ((b >> 1) & 3)) * 16)) = v;
+  }
+  int count = 0;
+  if constexpr (TABLE) count = stage_table<G>(p.L, p.Kg, p.K_L, s_tab, s_warp, p.status);
+  else __syncthreads();
+  const int iters = (nb + 31) / 32;                          // blocks per lane (<= NQ_PARTS)
+  uint32_t phbits = 0;
+  int slot = 0;
+  for (; row < end; row += NQ_WARPS, slot ^= 1) {
+    const bool loaded = row < (uint32_t)p.M;                 // warp-uniform (pad rows are not loaded)
+    if (loaded) {
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(smem_u32(&s_bar[warp][slot]), (phbits >> slot) & 1u, reinterpret_cast<volatile int*>(&s_abort), p.status);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      __syncwarp();
+      if (!ok) {
+        if (lane == 0 && row + NQ_WARPS < end && row + NQ_WARPS < (uint32_t)p.M) {
+          volatile int never = 0;
+          mbar_wait(smem_u32(&s_bar[warp][slot ^ 1]), (phbits >> (slot ^ 1)) & 1u, &never, nullptr, 100000000ull);
+        }
+        break;
+      }
+      phbits ^= 1u << slot;
+    }
+    const uint8_t* buf = row_buf(warp, slot);
+    float inv = 0.0f;
+    if (loaded) {
+      float part[NQ_PARTS];
+#pragma unroll
+      for (int i = 0; i < NQ_PARTS; ++i) {
+        part[i] = 0.0f;
+        const int blk = lane + 32 * i;
+        if (i < iters && blk < nb) {
+          uint32_t w[16];
+          load_block_smem(buf, blk, w);
+          float acc = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float lo = lo_f(w[j]), hi = hi_f(w[j]);
+            acc = __fadd_rn(acc, __fmul_rn(lo, lo));
+            acc = __fadd_rn(acc, __fmul_rn(hi, hi));
+          }
+          part[i] = acc;
+        }
+      }
+      // pairwise over the blocks: first the levels whose partners sit in the same lane
+      // (h = 32 hh blocks apart), then across lanes; levels above the row's own power of two
+      // only add zeros, which changes nothing
+#pragma unroll
+      for (int hh = NQ_PARTS / 2; hh >= 1; hh >>= 1)
+#pragma unroll
+        for (int i = 0; i < hh; ++i) part[i] = __fadd_rn(part[i], part[i + hh]);
+      float v = part[0];
+#pragma unroll
+      for (int h = 16; h >= 1; h >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, h));
+      const float total = __shfl_sync(0xffffffffu, v, 0);
+      const float root = __fsqrt_rn(__fadd_rn(__fdiv_rn(total, (float)p.K), p.eps));
+      inv = __fdiv_rn(1.0f, root);
+    }
+    for (int i = 0; i < iters; ++i) {
+      const int blk = lane + 32 * i;
+      const bool valid = blk < nb;
+      uint32_t w[16];
+      if (loaded && valid) {
+        uint32_t x[16], g[16];
+        load_block_smem(buf, blk, x);
+        load_block_smem(gam, blk, g);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float ylo = __fmul_rn(__fmul_rn(lo_f(x[j]), inv), lo_f(g[j]));
+          const float yhi = __fmul_rn(__fmul_rn(hi_f(x[j]), inv), hi_f(g[j]));
+          w[j] = pack_bf16x2(ylo, yhi);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) w[j] = 0u;
+      }
+      BlockTable t{-1, 0, -1, 0};
+      if constexpr (TABLE) t = block_table_packed<G>(valid ? blk : 0, s_tab);
+      quant_block<G, false, TABLE>(w, (int)row, blk, loaded, t, count, p.K, p.K_L, p.B, p.Q, p.S, valid);
+    }
+    __syncwarp();                                             // every lane is done with this slot
+    if (row + 2 * NQ_WARPS < end) { fence_proxy_async_smem(); issue(row + 2 * NQ_WARPS, slot); }
+  }
+}
+
+size_t rmsnorm_quant_smem(int K) {
+  const size_t slot = ((size_t)K * 2 + 1023) & ~(size_t)1023;
+  return slot * (1 + 2 * NQ_WARPS) + 1024;
+}
+
+template <int G, bool TABLE>
+static cudaError_t launch_nq(const CUtensorMap& tmX, const NormQuantParams& p, int grid, size_t smem, cudaStream_t s) {
+  static PerDeviceOnce smem_attr;
+  const cudaError_t ae = smem_attr.run([] {
+    return cudaFuncSetAttribute(rmsnorm_quantize_kernel<G, TABLE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)rmsnorm_quant_smem(NQ_MAX_K));
+  });
+  if (ae != cudaSuccess) return ae;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, rmsnorm_quantize_kernel<G, TABLE>, tmX, p);
+}
+
+cudaError_t launch_rmsnorm_quantize(const CUtensorMap& tmX, const NormQuantParams& p, int num_sms, cudaStream_t s) {
+  if (p.K % 256 != 0 || p.K > NQ_MAX_K) return cudaErrorInvalidValue;
+  const bool table = p.L != nullptr;
+  if (table && p.Kg > MAX_KG) return cudaErrorInvalidValue;
+  const size_t smem = rmsnorm_quant_smem(p.K);
+  const long long rows = (long long)(p.M + 127) / 128 * 128;
+  // CTAs per SM: shared memory allows (227 KB / smem), registers (about 124 a thread) two
+  const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(2, (size_t)(227 * 1024) / smem));
+  const int grid = (int)std::max<long long>(1, std::min<long long>((rows + NQ_WARPS - 1) / NQ_WARPS, (long long)num_sms * per_sm));
+  switch (p.G) {
+    case 16: return table ? launch_nq<16, true>(tmX, p, grid, smem, s) : launch_nq<16, false>(tmX, p, grid, smem, s);
+    case 32: return table ? launch_nq<32, true>(tmX, p, grid, smem, s) : launch_nq<32, false>(tmX, p, grid, smem, s);
+    case 64: return table ? launch_nq<64, true>(tmX, p, grid, smem, s) : launch_nq<64, false>(tmX, p, grid, smem, s);
+    default: return cudaErrorInvalidValue;
   }
 }
 

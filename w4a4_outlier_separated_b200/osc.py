@@ -48,6 +48,7 @@ def lib() -> ctypes.CDLL:
             "osc_density": ([P, i32, i32, i32, f32, P, P, P, P], i32),
             "osc_select_tier": ([P, P, i32, P], i32),
             "osc_quantize": ([P, i32, i32, i32, P, i32, P, P, P, P], i32),
+            "osc_rmsnorm_quantize": ([P, P, f32, i32, i32, i32, P, i32, P, P, P, P], i32),
             "osc_prepare_weight": ([P, i32, i32, i32, P, i32, P, P, P, P], i32),
             "osc_linear": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P], i32),
             "osc_quantize_fp8": ([P, i32, i32, P, P, P], i32),
@@ -150,6 +151,13 @@ def osc_quantize(X, G: int, L, K_L: int, QX, SX, B, stream=None):
                                               _ptr(B) if K_L else None, _stream(stream)))
 
 
+def osc_rmsnorm_quantize(X, gamma, eps: float, G: int, L, K_L: int, QX, SX, B, stream=None):
+    M, K = X.shape
+    _check("osc_rmsnorm_quantize", lib().osc_rmsnorm_quantize(_ptr(X), _ptr(gamma), eps, M, K, G, _ptr(L), K_L,
+                                                              _ptr(QX), _ptr(SX), _ptr(B) if K_L else None,
+                                                              _stream(stream)))
+
+
 def osc_prepare_weight(W, G: int, L, K_L: int, QW, SW, WL, stream=None):
     N, K = W.shape
     _check("osc_prepare_weight", lib().osc_prepare_weight(_ptr(W), N, K, G, _ptr(L), K_L, _ptr(QW), _ptr(SW),
@@ -232,6 +240,14 @@ def quantize(X, G: int, L=None, K_L: int = 0, stream=None):
     M, K = X.shape
     QX, SX, B = alloc_quantize_outputs(M, K, G, K_L, X.device)
     osc_quantize(X, G, L, K_L, QX, SX, B, stream)
+    return QX, SX, B
+
+
+def rmsnorm_quantize(X, gamma, eps: float, G: int, L=None, K_L: int = 0, stream=None):
+    """X (M x K) and gamma (K) -> (QX, SX, B) of the normalized rows."""
+    M, K = X.shape
+    QX, SX, B = alloc_quantize_outputs(M, K, G, K_L, X.device)
+    osc_rmsnorm_quantize(X, gamma, eps, G, L, K_L, QX, SX, B, stream)
     return QX, SX, B
 
 
