@@ -544,6 +544,68 @@ def _osc_dense_row(name, X, W, calib, G, steps, R, peaks):
                        4.0 * peaks["bf16_tflops"], peaks, R, lbytes)
 
 
+def _rmsnorm_fused_row(name, X, W, calib, G, steps, R, peaks):
+    """The producer-fused input side: osc_rmsnorm_quantize (RMSNorm + extraction + MX
+    quantization, one read of X) + osc_linear, beside the unfused sequence in which a library
+    RMSNorm (torch.nn.functional.rms_norm, a comparator only) writes the normalized rows and
+    osc_quantize reads them back. Table by Algorithm 1 on calibration rows normalized the same
+    way."""
+    import torch
+    from w4a4_outlier_separated_b200 import osc
+    M, K = X.shape
+    N = W.shape[0]
+    eps = 1e-6
+    gamma_h = (1.0 + 0.1 * np.random.default_rng(1).standard_normal(K))
+    gamma = torch.from_numpy(gamma_h).to(torch.bfloat16).cuda()
+    gbits = gamma.view(torch.int16)
+    Cd = _to_dev(calib).view(torch.bfloat16)
+    Cn = torch.nn.functional.rms_norm(Cd.float(), (K,), gamma.float(), eps).to(torch.bfloat16)
+    Ld = torch.empty(K // G, dtype=torch.int8, device="cuda")
+    osc.osc_build_table(Cn.view(torch.int16), G, 5.0, 5, Ld)
+    K_L = osc.osc_table_kl(Ld.cpu().numpy())
+    QW, SW, WL = osc.prepare_weight(_to_dev(W), G, Ld, K_L)
+    Xd = _to_dev(X)
+    sets = []
+    for i in range(R):
+        QX, SX, B = osc.alloc_quantize_outputs(M, K, G, K_L, "cuda")
+        sets.append(dict(X=Xd if i == 0 else Xd.clone(), QW=QW if i == 0 else QW.clone(), SW=SW if i == 0 else SW.clone(),
+                         WL=(WL if i == 0 else WL.clone()) if K_L else None, QX=QX, SX=SX, B=B,
+                         Y=torch.empty((M, N), dtype=torch.bfloat16, device="cuda")))
+
+    def fused(i):
+        c = sets[i % R]
+        osc.osc_rmsnorm_quantize(c["X"], gbits, eps, G, Ld, K_L, c["QX"], c["SX"], c["B"])
+
+    def unfused(i):
+        c = sets[i % R]
+        Xn = torch.nn.functional.rms_norm(c["X"].view(torch.bfloat16), (K,), gamma, eps)
+        osc.osc_quantize(Xn.view(torch.int16), G, Ld, K_L, c["QX"], c["SX"], c["B"])
+
+    def lin(i):
+        c = sets[i % R]
+        osc.osc_linear(c["QX"], c["SX"], c["B"], c["QW"], c["SW"], c["WL"], M, N, K, G, K_L, c["Y"])
+
+    def step(i):
+        fused(i)
+        lin(i)
+
+    for i in range(max(3, R)):
+        step(i)
+        unfused(i)
+    torch.cuda.synchronize()
+    s_ms, f_ms, u_ms = _timed_graphs([step, fused, unfused], steps)
+    _status_ok()
+    qb = quant_bytes(M, K, G, K_L) + K * 2
+    return {"workload": name, "M": M, "K": K, "N": N, "G": G, "K_L": K_L, "input_sets": R,
+            "ms_per_step": round(s_ms, 5), "TFLOPs": round(2.0 * M * N * K / (s_ms * 1e-3) / 1e12, 1),
+            "fused_quantize_ms": round(f_ms, 5), "fused_quantize_GBps": round(qb / (f_ms * 1e-3) / 1e9, 1),
+            "fused_quantize_hbm_frac": round(qb / (f_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+            "unfused_norm_then_quantize_ms": round(u_ms, 5),
+            "bytes_saved_per_step": 2 * M * K * 2,
+            "how": "fused = osc_rmsnorm_quantize; unfused = torch rms_norm (bf16 out, library kernel) then "
+                   "osc_quantize; the fused kernel neither writes nor re-reads the normalized rows"}
+
+
 def _fp8_dense_row(name, X, W, steps, R, peaks):
     """MXFP8 (E4M3, per-32 E8M0) on one dense layer: the fallback of the OSC page's §4, and the
     W8A8 comparator of its Table 2. Each step osc_quantize_fp8 + osc_linear_fp8_fallback."""
@@ -687,6 +749,8 @@ def scope_rows(steps: int):
     for G in (16, 32, 64):
         run(f"qkv_g{G}", lambda G=G: _osc_dense_row(f"qkv_proj G={G}", q.X, q.W, q.calib, G, steps, 4, peaks))
     run("qkv_w8a8", lambda: _fp8_dense_row("qkv_proj W8A8 (MXFP8)", q.X, q.W, steps, 4, peaks))
+    run("qkv_rmsnorm_fused", lambda: _rmsnorm_fused_row("qkv_proj RMSNorm-fused quantize G=32", q.X, q.W, q.calib,
+                                                         32, steps, 8, peaks))
     w8 = out.get("qkv_w8a8", {})
     if "ms_per_step" in w8:
         out["table2_osc_speedup_over_w8a8"] = {
@@ -819,8 +883,11 @@ def rows_brief(rows: dict) -> dict:
     of the line."""
     out = {}
     for k, r in rows.items():
-        if isinstance(r, dict) and "ms_per_step" in r:
+        if isinstance(r, dict) and "linear_roofline_frac" in r:
             out[k] = [round(r["ms_per_step"] * 1e3, 1), r["linear_roofline_frac"], r["quantize_hbm_frac"]]
+        elif isinstance(r, dict) and "fused_quantize_hbm_frac" in r:
+            out[k] = [round(r["ms_per_step"] * 1e3, 1), round(r["fused_quantize_ms"] * 1e3, 2),
+                      round(r["unfused_norm_then_quantize_ms"] * 1e3, 2), r["fused_quantize_hbm_frac"]]
         elif isinstance(r, dict) and "error" in r:
             out[k] = "error"
     if "table2_osc_speedup_over_w8a8" in rows:
