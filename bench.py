@@ -268,9 +268,9 @@ def run_osc(args):
     del g_step, g_q, g_l
 
     wb = weight_bound(wl, args.steps)
-    wb_us = max_over_ranks([d["us"] for d in wb], "cuda")
-    for d, us in zip(wb, wb_us):
-        d["us"] = us
+    wb_us = max_over_ranks([d["us"] for d in wb] + [d["us_one_part"] for d in wb], "cuda")
+    for i, d in enumerate(wb):
+        d["us"], d["us_one_part"] = wb_us[i], wb_us[len(wb) + i]
 
     # End to end through the public API with host buffers: each step copies its X in from pinned
     # host memory and its Y out to pinned host memory. Three streams overlap step i's kernels
@@ -359,12 +359,17 @@ def run_osc(args):
                            "copy of step i+1 and the output copy of step i-1 overlap step i's kernels on "
                            "separate streams (double-buffered device X and Y)"},
             "weight_bound": {
-                "what": "osc_linear alone at few token rows (QKV K=4096 N=6144): bytes of Q_W, S_W, W_L, "
-                        "Q_X, S_X, B and Y per launch over its duration; launches rotate over 10 weight "
-                        "copies (~146 MB > L2)",
+                "what": "the product alone at few token rows (QKV K=4096 N=6144): bytes of Q_W, S_W, W_L, "
+                        "Q_X, S_X, B and Y per launch over its duration, for osc_linear_splitk (K split over "
+                        "several SMs, fp32 partials in a workspace, chained reduction; 'us') and osc_linear "
+                        "(one part per weight tile; 'us_one_part'); launches rotate over 10 weight copies "
+                        "(~146 MB > L2)",
                 "unit": "GB/s", "peak": peaks["hbm_gbs"],
                 "lines": [{"M": d["M"], "us": round(d["us"], 2), "GBps": round(d["bytes"] / (d["us"] * 1e-6) / 1e9, 1),
-                           "frac": round(d["bytes"] / (d["us"] * 1e-6) / 1e9 / peaks["hbm_gbs"], 3)} for d in wb]},
+                           "frac": round(d["bytes"] / (d["us"] * 1e-6) / 1e9 / peaks["hbm_gbs"], 3),
+                           "us_one_part": round(d["us_one_part"], 2),
+                           "frac_one_part": round(d["bytes"] / (d["us_one_part"] * 1e-6) / 1e9 / peaks["hbm_gbs"], 3)}
+                          for d in wb]},
             "gpu_launches": 2 * args.steps,
             "clocks": clk.summary(),
         }
@@ -388,35 +393,27 @@ def weight_bound(wl, steps: int):
         QX, SX, B = osc.alloc_quantize_outputs(M, K_, G_, K_L, "cuda")
         osc.osc_quantize(wl["Xd"][:M].contiguous(), G_, wl["Ld"], K_L, QX, SX, B)
         Y = torch.empty((M, N_), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(max(1, osc.osc_linear_workspace_bytes(M, N_, K_, K_L) // 4), dtype=torch.float32,
+                         device="cuda")
 
         def lin(i):
             QW, SW, WL = wsets[i % R]
             osc.osc_linear(QX, SX, B, QW, SW, WL, M, N_, K_, G_, K_L, Y)
 
+        def lin_split(i):
+            QW, SW, WL = wsets[i % R]
+            osc.osc_linear_splitk(QX, SX, B, QW, SW, WL, M, N_, K_, G_, K_L, Y, ws)
+
         for i in range(R):
             lin(i)
+            lin_split(i)
         torch.cuda.synchronize()
-        gs = torch.cuda.Stream()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(gs):
-            lin(0)
-            gs.synchronize()
-            with torch.cuda.graph(g, stream=gs):
-                for i in range(steps):
-                    lin(i)
-        torch.cuda.synchronize()
-        g.replay()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        g.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / steps
+        us_plain, us_split = (t * 1e3 for t in _timed_graphs([lin, lin_split], steps))
+        _status_ok()
         nbytes = (wl["QW"].numel() + wl["SW"].numel() + wl["WL"].numel() * 2 + QX.numel() + SX.numel()
                   + (B.numel() * 2 if B is not None else 0) + Y.numel() * 2)
-        out.append({"M": M, "us": us, "bytes": nbytes})
-        del g
+        out.append({"M": M, "us": us_split, "us_one_part": us_plain, "bytes": nbytes,
+                    "workspace_bytes": ws.numel() * 4})
     return out
 
 
@@ -908,8 +905,10 @@ def tail_order(res: dict) -> dict:
     if "weight_bound" in res:
         wb = res["weight_bound"]
         out["weight_bound"] = {"unit": wb["unit"], "peak": wb["peak"],
-                               "lines": [[d["M"], d["us"], d["GBps"], d["frac"]] for d in wb["lines"]],
-                               "columns": ["M", "us", "GB/s", "frac"], "what": wb["what"]}
+                               "lines": [[d["M"], d["us"], d["GBps"], d["frac"], d.get("us_one_part"),
+                                          d.get("frac_one_part")] for d in wb["lines"]],
+                               "columns": ["M", "us", "GB/s", "frac", "us_one_part", "frac_one_part"],
+                               "what": wb["what"]}
     return out
 
 

@@ -161,6 +161,23 @@ OSC_API int osc_linear(const uint8_t* QX, const uint8_t* SX, const uint16_t* B,
                int M, int N, int K, int G, int K_L, uint16_t* Y, float* Yf32,
                osc_stream_t stream);
 
+/* The product of osc_linear for few token rows, with the weight stream split over more SMs.
+ * For M <= 128 the product is weight-bound: every call reads all of QW, SW and W_L. osc_linear
+ * already computes it transposed (the weight tile as the 128-row tensor-core operand, the M
+ * token rows as its narrow side), one 128-row weight tile per SM. osc_linear_splitk also
+ * splits each tile's K range over S SMs: each part writes its fp32 partial product (M x N) into
+ * `workspace`, and a second kernel on the same stream adds the S partials in a fixed order
+ * (part 0 first) and rounds to bf16, so Y does not depend on timing. Arguments as osc_linear,
+ * plus workspace: caller-allocated device memory of workspace_bytes bytes (16-byte aligned).
+ * Its contents need no initial value and are left undefined; calls that share a workspace
+ * must not overlap on the GPU. When workspace_bytes < osc_linear_workspace_bytes(M, N, K, K_L)
+ * (or M > 128) the call runs exactly as osc_linear. */
+OSC_API size_t osc_linear_workspace_bytes(int M, int N, int K, int K_L);
+OSC_API int osc_linear_splitk(const uint8_t* QX, const uint8_t* SX, const uint16_t* B,
+                              const uint8_t* QW, const uint8_t* SW, const uint16_t* WL,
+                              int M, int N, int K, int G, int K_L, uint16_t* Y, float* Yf32,
+                              float* workspace, size_t workspace_bytes, osc_stream_t stream);
+
 /* §4 FP8 fallback, quantize side: X (M x K bf16) -> QX8 (M x K E4M3 codes),
  * SX (osc_scale_bytes(M, K, 0)); per-32 E8M0 scales, no separation. Also used for the
  * weights of the fallback. */

@@ -158,6 +158,25 @@ def test_argument_limits_of_every_entry_point(lib):
     stt = lib.osc_selftest_timeout
     stt.argtypes = [I, V]
     assert stt(0, None) == -1 and stt(2_000_000, None) == -1                # limit out of range
+    rq = lib.osc_rmsnorm_quantize
+    rq.argtypes = [V, V, ctypes.c_float, I, I, I, V, I, V, V, V, V]
+    assert rq(p16, p16, -1.0, 4, 256, 32, None, 0, p16, p16, None, None) == -1       # eps < 0
+    assert rq(p16, p16, float("nan"), 4, 256, 32, None, 0, p16, p16, None, None) == -1
+    assert rq(p16, p16, 1e-6, 4, 8192, 32, None, 0, p16, p16, None, None) == -1       # K above 6144
+    assert rq(p16, None, 1e-6, 4, 256, 32, None, 0, p16, p16, None, None) == -1       # gamma required
+    assert rq(p16, V(p16.value + 2), 1e-6, 4, 256, 32, None, 0, p16, p16, None, None) == -2  # gamma alignment
+    assert rq(p16, p16, 1e-6, 4, 256, 24, None, 0, p16, p16, None, None) == -3        # G
+    assert rq(None, None, 1e-6, 0, 256, 32, None, 0, None, None, None, None) == 0     # M = 0: no-op
+    sk = lib.osc_linear_splitk
+    sk.argtypes = [V] * 6 + [I] * 5 + [V, V, V, ctypes.c_size_t, V]
+    assert sk(p16, p16, None, p16, p16, None, 4, 128, 256, 32, 0, p16, None, None, 64, None) == -1   # bytes, no buffer
+    assert sk(p16, p16, None, p16, p16, None, 4, 128, 256, 32, 0, p16, None, V(p16.value + 4), 64, None) == -2
+    assert sk(p16, p16, None, p16, p16, None, 4, 100, 256, 32, 0, p16, None, p16, 64, None) == -2    # N % 16
+    assert sk(None, None, None, None, None, None, 0, 128, 256, 32, 0, None, None, None, 0, None) == 0  # M = 0
+    wb = lib.osc_linear_workspace_bytes
+    wb.argtypes = [I, I, I, I]
+    wb.restype = ctypes.c_size_t
+    assert wb(129, 6144, 4096, 96) == 0 and wb(16, 6144, 4000, 96) == 0                # M > 128, K % 256
     lib.osc_set_cta_pair.argtypes = [I]
     assert lib.osc_set_cta_pair(3) == -1
     prev = lib.osc_set_cta_pair(1)

@@ -239,3 +239,99 @@ def test_moe_grouped_full_size_gateup(oracle, osc):
 
 def test_moe_grouped_full_size_down(oracle, osc):
     _moe(oracle, osc, None, "down", block_sample=True)
+
+
+def _prep(osc, X, W, G, L, K_L):
+    Ld = to_dev(L) if L is not None else None
+    QW, SW, WL = osc.prepare_weight(to_dev(W), G, Ld, K_L)
+    QX, SX, B = osc.quantize(to_dev(X), G, Ld, K_L)
+    return QX, SX, B, QW, SW, WL
+
+
+def _split_and_plain(oracle, osc, X, W, G, L, K_L):
+    """osc_linear_splitk with its workspace (K split over several SMs, partials added by the
+    chained reduction) and osc_linear (one part per weight tile), each launched with and without
+    the fp32 output; both against the oracle on every row and column."""
+    M, K = X.shape
+    N = W.shape[0]
+    QX, SX, B, QW, SW, WL = _prep(osc, X, W, G, L, K_L)
+    nbytes = osc.osc_linear_workspace_bytes(M, N, K, K_L)
+    assert nbytes > 0 and nbytes % (4 * M * N) == 0                # S >= 2 parts of M x N fp32
+    ws = torch.empty(nbytes // 4, dtype=torch.float32, device="cuda")
+    Y = [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _ in range(4)]
+    Yf = [torch.empty((M, N), dtype=torch.float32, device="cuda") for _ in range(2)]
+    osc.osc_linear_splitk(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y[0], ws, Yf[0])
+    osc.osc_linear_splitk(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y[1], ws)
+    osc.osc_linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y[2], Yf[1])
+    osc.osc_linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y[3])
+    torch.cuda.synchronize()
+    assert osc.osc_status() == (0, 0)
+    assert torch.equal(Y[1].view(torch.int16), Y[0].view(torch.int16))
+    assert torch.equal(Y[3].view(torch.int16), Y[2].view(torch.int16))
+    Lo = L if L is not None else np.full(K // G, -1, np.int8)
+    cw, ew, WLr = oracle.osc_prepare_weight(W, G, Lo, K_L)
+    ref = oracle.osc_forward(X, G, Lo, K_L, cw, ew, WLr)["Y"]
+    _compare(to_np(Y[0]), to_np(Yf[0]), ref)
+    _compare(to_np(Y[2]), to_np(Yf[1]), ref)
+    return QX, SX, B, QW, SW, WL
+
+
+@pytest.mark.parametrize("M", [1, 5, 16, 33, 64, 100, 128])
+def test_few_rows_qkv(oracle, osc, M):
+    """Few token rows at the QKV shape: token tiles of 16, 32, 64 and 128 (ragged M inside each),
+    K split over several SMs, the compensation stages dealt out with the FP4 ones."""
+    c = I.qkv_case(M)
+    L = oracle.build_table(c.calib, 32)
+    _split_and_plain(oracle, osc, c.X, c.W, 32, L, I.pad16(oracle.table_count(L)))
+
+
+@pytest.mark.parametrize("G", [16, 64])
+def test_few_rows_group_sizes(oracle, osc, G):
+    c = I.qkv_case(16)
+    L = oracle.build_table(c.calib, G)
+    _split_and_plain(oracle, osc, c.X, c.W, G, L, I.pad16(oracle.table_count(L)))
+
+
+def test_few_rows_ragged_and_small_workspace(oracle, osc):
+    """A partial last weight tile (N = 400), two compensation stages with a partial one
+    (K_L = 80), table channels 0 and G-1; then a workspace one byte too small, which must give
+    the one-part result bit for bit."""
+    rng = np.random.default_rng(31)
+    M, K, N, G = 7, 2304, 400, 32
+    x = rng.standard_normal((M, K))
+    L = np.full(K // G, -1, np.int8)
+    idx = rng.permutation(K // G)[:70]
+    L[idx] = rng.integers(0, G, size=70)
+    L[idx[0]], L[idx[1]] = 0, G - 1
+    for k, j in enumerate(L):
+        if j >= 0:
+            x[:, k * G + int(j)] = rng.choice([-1, 1], M) * rng.uniform(20, 80, M)
+    X = I.bf16_bits(x)
+    W = I.gen_weights(N, K, seed=3)
+    K_L = 80
+    QX, SX, B, QW, SW, WL = _split_and_plain(oracle, osc, X, W, G, L, K_L)
+    nbytes = osc.osc_linear_workspace_bytes(M, N, K, K_L)
+    small = torch.empty(nbytes - 1, dtype=torch.uint8, device="cuda")
+    Ya = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    Yb = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    osc.osc_linear_splitk(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Ya, small)
+    osc.osc_linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Yb)
+    torch.cuda.synchronize()
+    assert torch.equal(Ya.view(torch.int16), Yb.view(torch.int16))
+
+
+def test_few_rows_fp8_fallback(oracle, osc):
+    """The MXFP8 product at few token rows takes the same transposed path (K = 12288, the W2
+    shape, 16 rows)."""
+    c = I.w2_case(M=16)
+    M, K, N = 16, 12288, 4096
+    QX, SX, _ = osc.alloc_quantize_outputs(M, K, 32, 0, fp8=True)
+    QW, SW, _ = osc.alloc_quantize_outputs(N, K, 32, 0, fp8=True)
+    osc.osc_quantize_fp8(to_dev(c.X), QX, SX)
+    osc.osc_quantize_fp8(to_dev(c.W), QW, SW)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    Yf = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    osc.osc_linear_fp8_fallback(QX, SX, QW, SW, M, N, K, Y, Yf)
+    torch.cuda.synchronize()
+    assert osc.osc_status() == (0, 0)
+    _compare(to_np(Y), to_np(Yf), oracle.fp8_forward(c.X, c.W)["Y"])

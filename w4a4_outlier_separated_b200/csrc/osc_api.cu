@@ -119,10 +119,78 @@ int launch_result(cudaError_t e) { return e == cudaSuccess ? OSC_OK : fail_cuda(
 
 namespace {
 
+// The split plan of the few-row product: S parts of K per 128-row weight tile, so that
+// tiles x S CTAs (at most one per SM) stream the weights; S = 1 when there is no room for a
+// split or no workspace for its partials.
+struct SmallPlan {
+  int S, n_tiles;
+  size_t partial_bytes;
+};
+SmallPlan small_plan(int kind, int M, int N, int K, int K_L, int sms, bool with_workspace) {
+  SmallPlan pl;
+  pl.n_tiles = (N + 127) / 128;
+  const int T = K / (kind == osc::KIND_MXF8_B32 ? 128 : 256) + (K_L + 63) / 64;
+  int S = with_workspace ? sms / std::max(1, pl.n_tiles) : 1;
+  S = std::max(1, std::min(S, std::min(8, T / 2)));
+  pl.S = S;
+  pl.partial_bytes = S > 1 ? (size_t)S * (size_t)M * (size_t)N * sizeof(float) : 0;
+  return pl;
+}
+
+// Few-row product (M <= 128, dense calls): see osc_linear_small.cu.
+int run_gemm_small(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const uint8_t* QW,
+                   const uint8_t* SW, const uint16_t* WL, int M, int N, int K, int K_L, uint16_t* Y, float* Yf32,
+                   float* workspace, size_t workspace_bytes, const DeviceState* ds, cudaStream_t stream) {
+  const bool fp8 = kind == osc::KIND_MXF8_B32;
+  const int V = kind == osc::KIND_MXF4_B16 ? 16 : 32;
+  SmallPlan pl = small_plan(kind, M, N, K, K_L, ds->sms, workspace != nullptr);
+  if (pl.S > 1 && workspace_bytes < pl.partial_bytes) pl = small_plan(kind, M, N, K, K_L, ds->sms, false);
+  const int nt = osc::small_token_tile(M);
+  const uint64_t kb = fp8 ? (uint64_t)K : (uint64_t)K / 2;
+  const int nslot4 = K / V / 4;
+  const uint32_t aps = fp8 ? 1u : (V == 16 ? 4u : 2u);
+  osc::SmallMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  int rc;
+  {
+    uint64_t d[2] = {kb, (uint64_t)N}, st[1] = {kb};
+    uint32_t box[2] = {128, 128};
+    if ((rc = make_map(&maps.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, QW, d, st, box, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+    uint64_t dx[2] = {kb, (uint64_t)M};
+    uint32_t boxx[2] = {128, (uint32_t)nt};
+    if ((rc = make_map(&maps.x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, QX, dx, st, boxx, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+  }
+  {
+    uint64_t d[3] = {128, (uint64_t)nslot4, (uint64_t)((N + 127) / 128)}, st[2] = {512, (uint64_t)nslot4 * 512};
+    uint32_t box[3] = {128, aps, 1};
+    if ((rc = make_map(&maps.sw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, SW, d, st, box, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
+    uint64_t dx[3] = {128, (uint64_t)nslot4, 1};
+    if ((rc = make_map(&maps.sx, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, SX, dx, st, box, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
+  }
+  if (K_L > 0) {
+    uint64_t d[2] = {(uint64_t)K_L, (uint64_t)N}, st[1] = {(uint64_t)K_L * 2};
+    uint32_t box[2] = {64, 128};
+    if ((rc = make_map(&maps.wl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, WL, d, st, box, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+    uint64_t db[2] = {(uint64_t)K_L, (uint64_t)M};
+    uint32_t boxb[2] = {64, (uint32_t)nt};
+    if ((rc = make_map(&maps.b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, db, st, boxb, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+  }
+  osc::SmallParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = M; p.N = N; p.K = K; p.K_L = K_L;
+  p.S = pl.S; p.n_tiles = pl.n_tiles; p.num_sms = ds->sms;
+  p.Y = Y; p.Yf32 = Yf32; p.partial = pl.S > 1 ? workspace : nullptr;
+  p.status = ds->status;
+  const int units = pl.n_tiles * pl.S;
+  const int grid = units < ds->sms ? units : ds->sms;
+  return launch_result(osc::launch_gemm_small(kind, maps, p, grid, stream));
+}
+
 // Shared launch path of the dense, fallback and grouped products.
 int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const uint8_t* QW,
              const uint8_t* SW, const uint16_t* WL, int M, int N, int K, int K_L, int E,
-             const int* mblock_expert, const int* kl, uint16_t* Y, float* Yf32, cudaStream_t stream) {
+             const int* mblock_expert, const int* kl, uint16_t* Y, float* Yf32, cudaStream_t stream,
+             float* workspace = nullptr, size_t workspace_bytes = 0) {
   DeviceState* ds = nullptr;
   int rc = device_state(&ds);
   if (rc != OSC_OK) return rc;
@@ -131,6 +199,10 @@ int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
   int bn = g_tile_n.load();
   int cg = g_pair.load();
   const bool grouped = mblock_expert != nullptr;
+  // few token rows: the transposed product whose tensor work scales with the real row count,
+  // unless a tile shape was forced (the tests use that to reach the general kernel at small M)
+  if (!grouped && M <= 128 && bn == 0 && cg < 0)
+    return run_gemm_small(kind, QX, SX, B, QW, SW, WL, M, N, K, K_L, Y, Yf32, workspace, workspace_bytes, ds, stream);
   if (bn == 0) bn = (N >= 256 && (long long)((M + 127) / 128) * ((N + 255) / 256) >= ds->sms) ? 256 : 128;
   // the CTA pair needs 256-wide tiles, whole 256-row tiles of work and a per-128-row expert map
   // it cannot honour, so grouped calls stay on single CTAs
@@ -377,6 +449,32 @@ int osc_linear(const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const ui
   if ((rc = device_state(&ds)) != OSC_OK) return rc;
   const int kind = G == 16 ? osc::KIND_MXF4_B16 : osc::KIND_MXF4_B32;
   return run_gemm(kind, QX, SX, B, QW, SW, WL, M, N, K, K_L, 1, nullptr, nullptr, Y, Yf32, (cudaStream_t)stream);
+}
+
+size_t osc_linear_workspace_bytes(int M, int N, int K, int K_L) {
+  if (M <= 0 || M > 128 || N <= 0 || K <= 0 || K_L < 0 || K % 256 != 0 || N % 16 != 0 || K_L % 16 != 0) return 0;
+  DeviceState* ds = nullptr;
+  if (device_state(&ds) != OSC_OK) return 0;
+  return small_plan(osc::KIND_MXF4_B32, M, N, K, K_L, ds->sms, true).partial_bytes;
+}
+
+int osc_linear_splitk(const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const uint8_t* QW, const uint8_t* SW,
+                      const uint16_t* WL, int M, int N, int K, int G, int K_L, uint16_t* Y, float* Yf32,
+                      float* workspace, size_t workspace_bytes, osc_stream_t stream) {
+  if (!valid_g(G)) return OSC_ERR_G;
+  if (M == 0 && N > 0 && K > 0 && K_L >= 0) return OSC_OK;  // nothing to read or write
+  int rc = check_linear_common(QX, SX, QW, SW, M, N, K, Y, Yf32);
+  if (rc != OSC_OK) return rc;
+  if (K_L < 0 || K_L % 16 != 0) return K_L < 0 ? OSC_ERR_ARG : OSC_ERR_ALIGN;
+  if (K_L > 0 && (!B || !WL)) return OSC_ERR_ARG;
+  if (K_L > 0 && (!a16(B) || !a16(WL))) return OSC_ERR_ALIGN;
+  if (workspace_bytes > 0 && !workspace) return OSC_ERR_ARG;
+  if (workspace && !a16(workspace)) return OSC_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(&ds)) != OSC_OK) return rc;
+  const int kind = G == 16 ? osc::KIND_MXF4_B16 : osc::KIND_MXF4_B32;
+  return run_gemm(kind, QX, SX, B, QW, SW, WL, M, N, K, K_L, 1, nullptr, nullptr, Y, Yf32, (cudaStream_t)stream,
+                  workspace, workspace_bytes);
 }
 
 int osc_quantize_fp8(const uint16_t* X, int M, int K, uint8_t* QX8, uint8_t* SX, osc_stream_t stream) {

@@ -108,6 +108,23 @@ struct GemmMaps {
 // grid is a multiple of cg; m_tiles in p counts (128 * cg)-row tiles.
 cudaError_t launch_gemm(int kind, int bn, int cg, const GemmMaps& maps, const GemmParams& p, int grid, cudaStream_t s);
 
+// Few token rows (M <= 128): the transposed product with the weight tile as the 128-row MMA
+// operand, split over K into S parts (S > 1: fp32 partials in `partial`, S x M x N, added by a
+// chained reduction kernel).
+struct SmallParams {
+  int M, N, K, K_L;
+  int S, n_tiles, num_sms;
+  uint16_t* Y;
+  float* Yf32;
+  float* partial;
+  int* status;
+};
+struct SmallMaps {
+  CUtensorMap w, x, sw, sx, wl, b;
+};
+int small_token_tile(int M);   // MMA N for M token rows: 16, 32, 64 or 128
+cudaError_t launch_gemm_small(int kind, const SmallMaps& maps, const SmallParams& p, int grid, cudaStream_t s);
+
 struct TableParams {
   const uint16_t* X;   // S x K bf16
   int S, K, G;

@@ -176,10 +176,10 @@ __device__ __forceinline__ BlockTable block_table_packed(int blk, const int* tab
 // Stage one table (Kg entries) in shared memory, packed with each entry's B column; returns
 // the number of entries (at most K_L). Entries >= G or beyond K_L columns are reported and
 // dropped.
-template <int G>
+template <int G, int NTHREADS = 256>
 __device__ int stage_table(const int8_t* __restrict__ L, int Kg, int K_L, int* tab, int* s_warp, int* status) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int per = (Kg + 255) / 256;
+  const int per = (Kg + NTHREADS - 1) / NTHREADS;
   const int i0 = threadIdx.x * per, i1 = min(Kg, i0 + per);
   int local = 0;
   for (int i = i0; i < i1; ++i) {
@@ -197,7 +197,7 @@ __device__ int stage_table(const int8_t* __restrict__ L, int Kg, int K_L, int* t
   if (lane == 31) s_warp[warp] = incl;
   __syncthreads();
   int run = incl - local, count = 0;
-  for (int w = 0; w < 8; ++w) { if (w < warp) run += s_warp[w]; count += s_warp[w]; }
+  for (int w = 0; w < NTHREADS / 32; ++w) { if (w < warp) run += s_warp[w]; count += s_warp[w]; }
   for (int i = i0; i < i1; ++i) {
     const int v = tab[i];
     if (v < 0) { tab[i] = 0xFF; continue; }
@@ -429,57 +429,64 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
 // fused multiply-add: s_b = x_0^2 + ... + x_31^2 per 32-channel block in ascending order; the
 // block sums, padded with zeros to a power of two, combined pairwise (s_b += s_{b+h} for
 // h = P/2 .. 1); inv = 1 / sqrt(total / K + eps); y = bf16((x * inv) * gamma).
-constexpr int NQ_WARPS = 8;
+constexpr int NQ_WARPS = 16;
+constexpr int NQ_THREADS = NQ_WARPS * 32;
 constexpr int NQ_PARTS = 8;                      // block sums per lane: a power of two >= NQ_MAX_K / 1024
 static_assert(NQ_PARTS * 1024 >= NQ_MAX_K && (NQ_PARTS & (NQ_PARTS - 1)) == 0, "block sums per lane");
 
+// Row buffers per warp: two (the next row loads while this one is computed) when they fit in
+// shared memory beside gamma, else one.
+__host__ __device__ constexpr int nq_slots(int K) {
+  return (size_t)(((size_t)K * 2 + 1023) & ~(size_t)1023) * (1 + 2 * NQ_WARPS) + 1024 <= 227 * 1024 ? 2 : 1;
+}
+
 template <int G, bool TABLE>
-__global__ void __launch_bounds__(256, 1) rmsnorm_quantize_kernel(const __grid_constant__ CUtensorMap tmX, NormQuantParams p) {
+__global__ void __launch_bounds__(NQ_THREADS, 1) rmsnorm_quantize_kernel(const __grid_constant__ CUtensorMap tmX, NormQuantParams p) {
   extern __shared__ uint8_t nq_dyn[];
   uint8_t* base = nq_dyn + ((1024u - (smem_u32(nq_dyn) & 1023u)) & 1023u);
   const int nb = p.K / 32;                                   // 32-channel blocks per row
+  const int nslots = nq_slots(p.K);
   const uint32_t row_bytes = (uint32_t)p.K * 2u;
   const uint32_t slot_bytes = (row_bytes + 1023u) & ~1023u;
   uint8_t* gam = base;
-  auto row_buf = [&](int wp, int sl) { return base + slot_bytes * (1u + (uint32_t)(wp * 2 + sl)); };
+  auto row_buf = [&](int wp, int sl) { return base + slot_bytes * (1u + (uint32_t)(wp * nslots + sl)); };
   __shared__ __align__(8) uint64_t s_bar[NQ_WARPS][2];
   __shared__ __align__(8) int s_tab[TABLE ? MAX_KG : 2];
-  __shared__ int s_warp[8];
+  __shared__ int s_warp[NQ_WARPS];
   __shared__ int s_abort;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t mpad = (uint32_t)(p.M + 127) / 128u * 128u;
   // CTA b takes a contiguous run of rows (one more for the first mpad % grid CTAs); its warps
-  // take the run's rows round robin
+  // take the run's rows round robin; the warp's j-th row uses buffer j % nslots
   const uint32_t per = mpad / gridDim.x, extra = mpad % gridDim.x;
   const uint32_t first = blockIdx.x * per + min(blockIdx.x, extra);
   const uint32_t end = first + per + (blockIdx.x < extra ? 1u : 0u);
-  uint32_t row = first + warp;
   if (threadIdx.x == 0) s_abort = 0;
   if (lane == 0) { mbar_init(smem_u32(&s_bar[warp][0]), 1); mbar_init(smem_u32(&s_bar[warp][1]), 1); }
   fence_barrier_init();
   __syncwarp();
   grid_dep_wait();                                           // X, gamma and L are free of the previous kernel
   auto issue = [&](uint32_t r, int slot) {
-    if (lane == 0 && r < (uint32_t)p.M) {
+    if (lane == 0 && r < end && r < (uint32_t)p.M) {
       const uint32_t bar = smem_u32(&s_bar[warp][slot]);
       mbar_arrive_expect_tx(bar, row_bytes);
       tma_load_2d(smem_u32(row_buf(warp, slot)), &tmX, 0, (int)(r * (uint32_t)nb), bar);
     }
   };
-  if (row < end) issue(row, 0);
-  if (row + NQ_WARPS < end) issue(row + NQ_WARPS, 1);
+  const uint32_t row0 = first + warp;
+  for (int sl = 0; sl < nslots; ++sl) issue(row0 + (uint32_t)sl * NQ_WARPS, sl);
   for (int i = threadIdx.x; i < nb * 4; i += blockDim.x) {  // gamma, 16-byte chunks, swizzled
     const int b = i >> 2, c = i & 3;
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.gamma) + i);
     *reinterpret_cast<uint4*>(gam + b * 64 + ((c ^ ((b >> 1) & 3)) * 16)) = v;
   }
   int count = 0;
-  if constexpr (TABLE) count = stage_table<G>(p.L, p.Kg, p.K_L, s_tab, s_warp, p.status);
+  if constexpr (TABLE) count = stage_table<G, NQ_THREADS>(p.L, p.Kg, p.K_L, s_tab, s_warp, p.status);
   else __syncthreads();
   const int iters = (nb + 31) / 32;                          // blocks per lane (<= NQ_PARTS)
   uint32_t phbits = 0;
   int slot = 0;
-  for (; row < end; row += NQ_WARPS, slot ^= 1) {
+  for (uint32_t row = row0; row < end; row += NQ_WARPS, slot = (slot + 1 == nslots) ? 0 : slot + 1) {
     const bool loaded = row < (uint32_t)p.M;                 // warp-uniform (pad rows are not loaded)
     if (loaded) {
       bool ok = true;
@@ -487,9 +494,12 @@ __global__ void __launch_bounds__(256, 1) rmsnorm_quantize_kernel(const __grid_c
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       __syncwarp();
       if (!ok) {
-        if (lane == 0 && row + NQ_WARPS < end && row + NQ_WARPS < (uint32_t)p.M) {
+        // let the other buffer's load (if one was issued) land before leaving
+        const uint32_t nxt = row + NQ_WARPS;
+        if (lane == 0 && nslots == 2 && nxt < end && nxt < (uint32_t)p.M) {
+          const int o = slot ^ 1;
           volatile int never = 0;
-          mbar_wait(smem_u32(&s_bar[warp][slot ^ 1]), (phbits >> (slot ^ 1)) & 1u, &never, nullptr, 100000000ull);
+          mbar_wait(smem_u32(&s_bar[warp][o]), (phbits >> o) & 1u, &never, nullptr, 100000000ull);
         }
         break;
       }
@@ -552,14 +562,15 @@ __global__ void __launch_bounds__(256, 1) rmsnorm_quantize_kernel(const __grid_c
       if constexpr (TABLE) t = block_table_packed<G>(valid ? blk : 0, s_tab);
       quant_block<G, false, TABLE>(w, (int)row, blk, loaded, t, count, p.K, p.K_L, p.B, p.Q, p.S, valid);
     }
-    __syncwarp();                                             // every lane is done with this slot
-    if (row + 2 * NQ_WARPS < end) { fence_proxy_async_smem(); issue(row + 2 * NQ_WARPS, slot); }
+    __syncwarp();                                             // every lane is done with this buffer
+    const uint32_t nxt = row + (uint32_t)nslots * NQ_WARPS;
+    if (nxt < end) { fence_proxy_async_smem(); issue(nxt, slot); }
   }
 }
 
 size_t rmsnorm_quant_smem(int K) {
   const size_t slot = ((size_t)K * 2 + 1023) & ~(size_t)1023;
-  return slot * (1 + 2 * NQ_WARPS) + 1024;
+  return slot * (1 + (size_t)nq_slots(K) * NQ_WARPS) + 1024;
 }
 
 template <int G, bool TABLE>
@@ -567,12 +578,12 @@ static cudaError_t launch_nq(const CUtensorMap& tmX, const NormQuantParams& p, i
   static PerDeviceOnce smem_attr;
   const cudaError_t ae = smem_attr.run([] {
     return cudaFuncSetAttribute(rmsnorm_quantize_kernel<G, TABLE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)rmsnorm_quant_smem(NQ_MAX_K));
+                                (int)rmsnorm_quant_smem(NQ_MAX_K));   // the largest K needs the most
   });
   if (ae != cudaSuccess) return ae;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(256, 1, 1);
+  cfg.blockDim = dim3(NQ_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -589,9 +600,8 @@ cudaError_t launch_rmsnorm_quantize(const CUtensorMap& tmX, const NormQuantParam
   if (table && p.Kg > MAX_KG) return cudaErrorInvalidValue;
   const size_t smem = rmsnorm_quant_smem(p.K);
   const long long rows = (long long)(p.M + 127) / 128 * 128;
-  // CTAs per SM: shared memory allows (227 KB / smem), registers (about 124 a thread) two
-  const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(2, (size_t)(227 * 1024) / smem));
-  const int grid = (int)std::max<long long>(1, std::min<long long>((rows + NQ_WARPS - 1) / NQ_WARPS, (long long)num_sms * per_sm));
+  // one CTA of 16 warps per SM (its registers, up to 128 a thread, fill the SM's file)
+  const int grid = (int)std::max<long long>(1, std::min<long long>((rows + NQ_WARPS - 1) / NQ_WARPS, (long long)num_sms));
   switch (p.G) {
     case 16: return table ? launch_nq<16, true>(tmX, p, grid, smem, s) : launch_nq<16, false>(tmX, p, grid, smem, s);
     case 32: return table ? launch_nq<32, true>(tmX, p, grid, smem, s) : launch_nq<32, false>(tmX, p, grid, smem, s);

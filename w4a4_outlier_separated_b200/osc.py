@@ -51,6 +51,8 @@ def lib() -> ctypes.CDLL:
             "osc_rmsnorm_quantize": ([P, P, f32, i32, i32, i32, P, i32, P, P, P, P], i32),
             "osc_prepare_weight": ([P, i32, i32, i32, P, i32, P, P, P, P], i32),
             "osc_linear": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P], i32),
+            "osc_linear_workspace_bytes": ([i32, i32, i32, i32], ctypes.c_size_t),
+            "osc_linear_splitk": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P, ctypes.c_size_t, P], i32),
             "osc_quantize_fp8": ([P, i32, i32, P, P, P], i32),
             "osc_linear_fp8_fallback": ([P, P, P, P, i32, i32, i32, P, P, P], i32),
             "osc_grouped_plan": ([P, i32, P, P, P, i32], i32),
@@ -168,6 +170,22 @@ def osc_linear(QX, SX, B, QW, SW, WL, M: int, N: int, K: int, G: int, K_L: int, 
     _check("osc_linear", lib().osc_linear(_ptr(QX), _ptr(SX), _ptr(B) if K_L else None, _ptr(QW), _ptr(SW),
                                           _ptr(WL) if K_L else None, M, N, K, G, K_L, _ptr(Y), _ptr(Yf32),
                                           _stream(stream)))
+
+
+def osc_linear_workspace_bytes(M: int, N: int, K: int, K_L: int) -> int:
+    """Bytes of fp32 partials osc_linear_splitk needs on the current device (0: no split)."""
+    return int(lib().osc_linear_workspace_bytes(M, N, K, K_L))
+
+
+def osc_linear_splitk(QX, SX, B, QW, SW, WL, M: int, N: int, K: int, G: int, K_L: int, Y, workspace, Yf32=None,
+                      stream=None):
+    """osc_linear for few token rows with the K range of each weight tile split over several SMs;
+    `workspace` is a CUDA tensor (any dtype) whose bytes hold the fp32 partials."""
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("osc_linear_splitk", lib().osc_linear_splitk(_ptr(QX), _ptr(SX), _ptr(B) if K_L else None, _ptr(QW),
+                                                        _ptr(SW), _ptr(WL) if K_L else None, M, N, K, G, K_L,
+                                                        _ptr(Y), _ptr(Yf32), _ptr(workspace), nbytes,
+                                                        _stream(stream)))
 
 
 def osc_quantize_fp8(X, QX8, SX, stream=None):
