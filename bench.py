@@ -727,7 +727,7 @@ def scope_rows(steps: int):
     MXFP8 fallback; the grouped MoE expert layers; and the W8A8 comparator of the page's
     Table 2 at the QKV shape beside OSC at G = 16 / 32 / 64 (step-time ratio). "tiers" holds
     the automatic tier of each dense module input at each group size (density on the GPU,
-    rule on the host)."""
+    rule on the host) and the group size the per-layer rule picks from them."""
     import torch
     from w4a4_outlier_separated_b200 import inputs as I
     peaks, _ = measured_peaks()
@@ -772,6 +772,13 @@ def scope_rows(steps: int):
     del w
     run("moe_gateup", lambda: _moe_row("gateup", steps, peaks))
     run("moe_down", lambda: _moe_row("down", steps, peaks))
+    from w4a4_outlier_separated_b200 import osc
+    for mod in ("qkv", "ffn", "w2"):
+        cs = [tiers.get(f"{mod}_g{G}", {}).get("C_bar") for G in (16, 32, 64)]
+        if all(c is not None for c in cs):
+            g, t = osc.osc_select_group_size(*cs)
+            tiers[f"{mod}_choice"] = {"G": g, "tier": osc.TIERS[t],
+                                      "path": "MXFP8 fallback" if g == 0 else f"OSC W4A4 G={g}"}
     out["tiers"] = tiers
     out["how"] = ("per row: K steps (quantize + linear) as one CUDA graph between events, R rotating input sets "
                   "(each with its own weight copy) so that inputs exceed L2; linear_frac = useful flops against the "

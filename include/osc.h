@@ -127,6 +127,17 @@ enum {
  * (nothing escapes the table; with an empty table OSC is plain MXFP4). */
 OSC_API int osc_select_tier(const int* n_hit, const int* n_total, int Kg, double* c_bar);
 
+/* §6 "dynamic group size" (HOST logic): the group size of one module from its clustering
+ * density measured with tables built at G = 16, 32 and 64, c_bar[0..2] in that order (NaN
+ * where a G saw no events, as osc_select_tier reports it). The page names the idea without a
+ * rule; this one keeps the page's tiers at its default G = 32 and moves G only where static
+ * protection holds at the high tier: the largest G whose C is above 60 % (fewer scales and
+ * table entries, the fastest product in Table 2); if no G is that high, G = 32 with its own
+ * tier. Returns 16, 32 or 64, or 0 when the module takes the MXFP8 fallback (G = 32 in the
+ * fallback tier); *tier (may be NULL) receives the tier of the choice. OSC_ERR_ARG if
+ * c_bar is NULL. */
+OSC_API int osc_select_group_size(const double* c_bar, int* tier);
+
 /* §3.2, Figure 2 (online): extraction + zeroing through the table, then MXFP4 quantization
  * of the zeroed tensor. X (M x K bf16) -> QX (M x K/2), SX (osc_scale_bytes(M, K, G)),
  * B (M x K_L bf16). L may be NULL (no table: plain MXFP4; then K_L must be 0 and B may be
@@ -201,12 +212,13 @@ OSC_API int osc_linear_fp8_fallback(const uint8_t* QX8, const uint8_t* SX, const
 OSC_API int osc_grouped_plan(const int* counts, int E, int* off, int* poff, int* mblock_expert,
                      int mblock_capacity);
 
-/* Per-expert extraction + MXFP4 quantization. X: off[E] x K bf16 (device). off, poff,
+/* Per-expert extraction + MXFP4 quantization. X: T x K bf16 (device), T = off[E] the routed
+ * rows (the value of off[E] on the host, passed so that the call needs no copy back). off, poff,
  * mblock_expert: device copies of the plan. L: E x K/G (device), expert e's table at e*K/G.
  * Outputs over the padded rows: QX (Mp x K/2), SX (osc_scale_bytes(Mp, K, G)),
  * B (Mp x K_L bf16, K_L a common width >= every expert's entry count); pad rows are 0.
  * E x K/G may be at most about 68000 table entries (they are staged in shared memory). */
-OSC_API int osc_quantize_grouped(const uint16_t* X, int E, const int* off, const int* poff,
+OSC_API int osc_quantize_grouped(const uint16_t* X, int T, int E, const int* off, const int* poff,
                          const int* mblock_expert, int Mp, int K, int G, const int8_t* L,
                          int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B, osc_stream_t stream);
 

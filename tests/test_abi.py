@@ -138,10 +138,12 @@ def test_argument_limits_of_every_entry_point(lib):
     assert bt(p16, 8, 250, 32, 5.0, 5, p16, None) == -1                    # K % G
     assert bt(p16, 8, 256, 8, 5.0, 5, p16, None) == -3                     # G
     qg = lib.osc_quantize_grouped
-    qg.argtypes = [V, I, V, V, V, I, I, I, V, I, V, V, V, V]
-    assert qg(p16, 2, p16, p16, p16, 200, 256, 32, p16, 0, p16, p16, None, None) == -2   # Mp % 128
-    assert qg(p16, 2, p16, p16, p16, 256, 256, 32, None, 0, p16, p16, None, None) == -1  # tables required
-    assert qg(p16, 2, p16, p16, p16, 1 << 30, 256, 32, p16, 0, p16, p16, None, None) == -1  # scale index overflow
+    qg.argtypes = [V, I, I, V, V, V, I, I, I, V, I, V, V, V, V]
+    assert qg(p16, 100, 2, p16, p16, p16, 200, 256, 32, p16, 0, p16, p16, None, None) == -2   # Mp % 128
+    assert qg(p16, 100, 2, p16, p16, p16, 256, 256, 32, None, 0, p16, p16, None, None) == -1  # tables required
+    assert qg(p16, 100, 2, p16, p16, p16, 1 << 30, 256, 32, p16, 0, p16, p16, None, None) == -1  # scale index overflow
+    assert qg(p16, 300, 2, p16, p16, p16, 256, 256, 32, p16, 0, p16, p16, None, None) == -1   # T > Mp
+    assert qg(p16, -1, 2, p16, p16, p16, 256, 256, 32, p16, 0, p16, p16, None, None) == -1    # T < 0
     lg = lib.osc_linear_grouped
     lg.argtypes = [V, V, V, V, V, V, V, V, I, I, I, I, I, I, V, V, V]
     assert lg(p16, p16, None, p16, p16, None, p16, None, 2, 200, 256, 256, 32, 0, p16, None, None) == -2  # Mp % 128

@@ -77,3 +77,33 @@ def test_module_inputs_land_in_the_page_tiers(osc, oracle):
     tier, c = osc.osc_select_tier(nh, nt)
     lo, hi = _bands()["w2"]
     assert tier == 0 and lo <= c <= hi
+
+
+def test_group_size_rule(osc):
+    """The per-layer group size (§6, dynamic group size; the rule is a stated reading): the
+    largest G whose density is above 60 %, else G = 32 with its own tier, 0 for the MXFP8
+    fallback. Boundaries of the tiers apply as in osc_select_tier (60 % itself is not high)."""
+    nan = float("nan")
+    assert osc.osc_select_group_size(0.36, 0.703, 0.726) == (64, 2)      # QKV-like: high at 32 and 64
+    assert osc.osc_select_group_size(0.90, 0.70, 0.50) == (32, 2)        # high at 16 and 32 only
+    assert osc.osc_select_group_size(0.65, 0.50, 0.40) == (16, 2)        # high only at the finest G
+    assert osc.osc_select_group_size(0.40, 0.60, 0.45) == (32, 1)        # nothing high: G = 32, mid tier
+    assert osc.osc_select_group_size(0.17, 0.27, 0.37) == (0, 0)         # W2-like: G = 32 falls back to MXFP8
+    assert osc.osc_select_group_size(0.20, 0.3499, 0.5999) == (0, 0)
+    assert osc.osc_select_group_size(0.20, 0.35, 0.30) == (32, 1)        # 35 % is the middle tier
+    assert osc.osc_select_group_size(nan, nan, nan) == (64, 2)           # no events anywhere
+    assert osc.osc_select_group_size(0.5, 0.5, 0.6000001) == (64, 2)
+
+
+def test_group_size_on_the_oracle_densities(osc, oracle):
+    """On the synthetic module inputs the rule picks G = 64 for the attention input (its
+    density stays above 60 % at G = 32 and 64) and the MXFP8 fallback for W2 (every G below
+    60 %, and G = 32 in the fallback tier), computed from the oracle's own counts."""
+    def cbar(case, G):
+        L = oracle.build_table(case.calib, G)
+        nh, nt = oracle.density(case.X, G, L)
+        return osc.osc_select_tier(nh.astype(np.int32), nt.astype(np.int32))[1]
+    q = I.qkv_case(256, calib_tokens=512)
+    assert osc.osc_select_group_size(*(cbar(q, G) for G in (16, 32, 64)))[0] == 64
+    w = I.w2_case(M=256, calib_tokens=512)
+    assert osc.osc_select_group_size(*(cbar(w, G) for G in (16, 32, 64))) == (0, 0)

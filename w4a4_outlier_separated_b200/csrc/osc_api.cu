@@ -352,6 +352,29 @@ int osc_density(const uint16_t* X, int S, int K, int G, float alpha, const int8_
   return launch_result(osc::launch_density(p, (cudaStream_t)stream));
 }
 
+namespace {
+// The tier of §2.3 for a clustering density C (NaN: no events, nothing escapes the table).
+int tier_of(double c) {
+  if (std::isnan(c)) return OSC_TIER_HIGH;
+  return c > 0.60 ? OSC_TIER_HIGH : (c >= 0.35 ? OSC_TIER_MID : OSC_TIER_FP8);
+}
+}  // namespace
+
+int osc_select_group_size(const double* c_bar, int* tier) {
+  if (!c_bar) return OSC_ERR_ARG;
+  static const int kG[3] = {16, 32, 64};
+  int best = 0;
+  for (int i = 0; i < 3; ++i)
+    if (tier_of(c_bar[i]) == OSC_TIER_HIGH) best = kG[i];
+  if (best != 0) {
+    if (tier) *tier = OSC_TIER_HIGH;
+    return best;
+  }
+  const int t = tier_of(c_bar[1]);
+  if (tier) *tier = t;
+  return t == OSC_TIER_FP8 ? 0 : 32;
+}
+
 int osc_select_tier(const int* n_hit, const int* n_total, int Kg, double* c_bar) {
   if (Kg < 0 || (Kg > 0 && (!n_hit || !n_total))) return OSC_ERR_ARG;
   double sum = 0.0;
@@ -369,7 +392,7 @@ int osc_select_tier(const int* n_hit, const int* n_total, int Kg, double* c_bar)
   }
   const double c = sum / groups;
   if (c_bar) *c_bar = c;
-  return c > 0.60 ? OSC_TIER_HIGH : (c >= 0.35 ? OSC_TIER_MID : OSC_TIER_FP8);
+  return tier_of(c);
 }
 
 int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int K_L, uint8_t* QX, uint8_t* SX,
@@ -526,12 +549,13 @@ int osc_grouped_plan(const int* counts, int E, int* off, int* poff, int* mblock_
   return (int)po;
 }
 
-int osc_quantize_grouped(const uint16_t* X, int E, const int* off, const int* poff, const int* mblock_expert, int Mp,
-                         int K, int G, const int8_t* L, int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B,
+int osc_quantize_grouped(const uint16_t* X, int T, int E, const int* off, const int* poff, const int* mblock_expert,
+                         int Mp, int K, int G, const int8_t* L, int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B,
                          osc_stream_t stream) {
   if (!valid_g(G)) return OSC_ERR_G;
   if (!X || !off || !poff || !mblock_expert || !L || !QX || !SX || E <= 0 || Mp < 0 || K <= 0 || K_L < 0)
     return OSC_ERR_ARG;
+  if (T < 0 || T > Mp) return OSC_ERR_ARG;
   if (K_L > 0 && !B) return OSC_ERR_ARG;
   if (K_L > 32767) return OSC_ERR_ARG;
   if ((long long)(Mp + 127) * (K / 32) >= (1LL << 31)) return OSC_ERR_ARG;
@@ -543,6 +567,11 @@ int osc_quantize_grouped(const uint16_t* X, int E, const int* off, const int* po
   if (rc != OSC_OK) return rc;
   if (Mp == 0) return OSC_OK;
   osc::GroupedQuantParams p{X, off, poff, mblock_expert, E, Mp, K, G, K / G, L, K_L, QX, SX, B, ds->status};
+  if (T > 0 && osc::grouped_tma_smem(E, K / G) <= (size_t)osc::GROUPED_TMA_SMEM_MAX) {
+    CUtensorMap tm;
+    if ((rc = make_block_map(&tm, X, T, K))) return rc;
+    return launch_result(osc::launch_quantize_grouped_tma(tm, p, T, ds->sms, (cudaStream_t)stream));
+  }
   return launch_result(osc::launch_quantize_grouped(p, ds->sms, (cudaStream_t)stream));
 }
 

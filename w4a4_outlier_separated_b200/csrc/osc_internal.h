@@ -76,6 +76,11 @@ struct GroupedQuantParams {
   int* status;
 };
 cudaError_t launch_quantize_grouped(const GroupedQuantParams& p, int num_sms, cudaStream_t s);
+// TMA form over the T = off[E] routed rows (tmX: the dense kernel's block view of those rows)
+cudaError_t launch_quantize_grouped_tma(const CUtensorMap& tmX, const GroupedQuantParams& p, int T, int num_sms,
+                                        cudaStream_t s);
+size_t grouped_tma_smem(int E, int Kg);
+constexpr int GROUPED_TMA_SMEM_MAX = 200 * 1024;
 // shared memory the grouped quantize needs to stage every expert's table, and its limit
 size_t grouped_quant_smem(int E, int Kg);
 constexpr int GROUPED_QUANT_SMEM_MAX = 200 * 1024;

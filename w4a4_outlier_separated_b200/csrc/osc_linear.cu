@@ -74,10 +74,18 @@ struct TileInfo {
   int m0, n0, e, kl;   // m0: this CTA's first row
 };
 
+// Tile order: dense products walk the row blocks fastest (CTAs running together share a
+// weight tile; at these sizes every operand fits L2 anyway). Grouped products walk the column
+// blocks fastest: CTAs running together then work on one expert's row block (sharing its
+// activation tile), and an expert's next row block follows right after, while its weights are
+// still in L2; row blocks fastest would spread concurrent CTAs over many experts and evict
+// each expert's weights between its row blocks.
 template <int CG>
 __device__ __forceinline__ TileInfo tile_info(int t, const GemmParams& p, int bn, int rank) {
   TileInfo ti;
-  const int mb = t % p.m_tiles, nb = t / p.m_tiles;     // m_tiles counts (128 * CG)-row tiles
+  const bool by_row = p.num_groups != 0;
+  const int mb = by_row ? t / p.n_tiles : t % p.m_tiles;   // m_tiles counts (128 * CG)-row tiles
+  const int nb = by_row ? t % p.n_tiles : t / p.m_tiles;
   ti.m0 = mb * 128 * CG + 128 * rank;
   ti.n0 = nb * bn;
   if (p.num_groups == 0) {

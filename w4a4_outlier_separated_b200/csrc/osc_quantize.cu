@@ -610,7 +610,194 @@ cudaError_t launch_rmsnorm_quantize(const CUtensorMap& tmX, const NormQuantParam
   }
 }
 
-// Grouped (MoE) form over the padded row space: a row's expert comes from its 128-row block;
+// Grouped (MoE) form on the TMA design of the dense kernel. The T routed rows of X are dense
+// and sorted by expert; steps of QSTEP items run over them exactly as in the dense kernel, and
+// each item's output row is its row in the padded space, poff[e] + t - off[e] for the expert
+// e that owns dense row t. The padded space's other rows take zero codes, scales and B in a
+// tail phase: pad row p (0 <= p < Mp - T) belongs to the expert e with
+// poff[e] - off[e] <= p < poff[e+1] - off[e+1] and sits at row off[e+1] + p.
+// Shared memory after the boxes: every expert's packed table (E x Kg words), off, poff (E+1
+// each) and the experts' entry counts (E).
+__device__ __forceinline__ int last_le(const int* a, int n, int v) {   // largest i < n with a[i] <= v (a[0] <= v)
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a[mid] <= v) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+size_t grouped_tma_smem(int E, int Kg) {
+  return (size_t)QWARPS * 2 * QSTEP * 64 + 1024 + 4 * ((size_t)E * Kg + 2 * ((size_t)E + 1) + (size_t)E);
+}
+
+template <int G>
+__global__ void __launch_bounds__(256) quantize_grouped_tma_kernel(const __grid_constant__ CUtensorMap tmX,
+                                                                    GroupedQuantParams p, int T) {
+  extern __shared__ uint8_t q_dyn[];
+  uint8_t* boxes = q_dyn + ((1024u - (smem_u32(q_dyn) & 1023u)) & 1023u);
+  auto box_at = [&](int wp, int sl) { return boxes + (wp * 2 + sl) * (QSTEP * 64); };
+  int* s_tab = reinterpret_cast<int*>(boxes + QWARPS * 2 * QSTEP * 64);
+  int* s_off = s_tab + p.E * p.Kg;
+  int* s_poff = s_off + (p.E + 1);
+  int* s_cnt = s_poff + (p.E + 1);
+  __shared__ __align__(8) uint64_t s_bar[QWARPS][2];
+  __shared__ int s_abort;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nblk = p.K / 32;
+  const uint32_t real_items = (uint32_t)T * (uint32_t)nblk;
+  const uint32_t nsteps = (real_items + QSTEP - 1) / QSTEP;
+  const uint32_t wstride = QWARPS;
+  const uint32_t per = nsteps / gridDim.x, extra = nsteps % gridDim.x;
+  const uint32_t cta_first = blockIdx.x * per + min(blockIdx.x, extra);
+  const uint32_t cta_end = cta_first + per + (blockIdx.x < extra ? 1u : 0u);
+  uint32_t step = cta_first + warp;
+  if (threadIdx.x == 0) s_abort = 0;
+  if (lane == 0) { mbar_init(smem_u32(&s_bar[warp][0]), 1); mbar_init(smem_u32(&s_bar[warp][1]), 1); }
+  fence_barrier_init();
+  __syncwarp();
+  grid_dep_wait();
+  auto issue = [&](uint32_t st, int slot) {
+    if (lane == 0) {
+      const uint32_t bar = smem_u32(&s_bar[warp][slot]);
+      mbar_arrive_expect_tx(bar, QSTEP * 64);                  // a box past the last item is zero-filled
+      tma_load_2d(smem_u32(box_at(warp, slot)), &tmX, 0, (int)(st * QSTEP), bar);
+    }
+  };
+  if (step < cta_end) issue(step, 0);
+  if (step + wstride < cta_end) issue(step + wstride, 1);
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) { s_off[i] = p.off[i]; s_poff[i] = p.poff[i]; }
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x) {     // one thread per expert table
+    int run = 0;
+    for (int g = 0; g < p.Kg; ++g) {
+      int v = p.L[(size_t)e * p.Kg + g];
+      if (v >= G || (v >= 0 && run >= p.K_L)) { record_status(p.status, DEV_BAD_TABLE); v = -1; }
+      s_tab[e * p.Kg + g] = v < 0 ? 0xFF : ((run++ << 8) | v);
+    }
+    s_cnt[e] = run;
+  }
+  __syncthreads();
+  uint32_t phbits = 0;
+  int slot = 0;
+  for (; step < cta_end; step += wstride, slot ^= 1) {
+    bool ok = true;
+    if (lane == 0) ok = mbar_wait(smem_u32(&s_bar[warp][slot]), (phbits >> slot) & 1u, reinterpret_cast<volatile int*>(&s_abort), p.status);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();
+    if (!ok) {
+      if (lane == 0 && step + wstride < cta_end) {
+        volatile int never = 0;
+        mbar_wait(smem_u32(&s_bar[warp][slot ^ 1]), (phbits >> (slot ^ 1)) & 1u, &never, nullptr, 100000000ull);
+      }
+      break;
+    }
+    phbits ^= 1u << slot;
+    uint8_t* box = box_at(warp, slot);
+    const uint32_t it0 = step * QSTEP;
+    int ta = (int)(it0 / (uint32_t)nblk);                     // dense row and block of item `lane`
+    int blka = (int)(it0 - (uint32_t)ta * nblk) + lane;
+    while (blka >= nblk) { blka -= nblk; ++ta; }
+    int e_row = -1, e = 0, dest0 = 0;                         // expert lookup cached per dense row
+#pragma unroll
+    for (int h = 0; h < QSTEP / 32; ++h) {
+      const int r = lane + 32 * h;
+      int t = ta, blk = blka + 32 * h;
+      while (blk >= nblk) { blk -= nblk; ++t; }
+      const bool live = t < T;
+      if (live && t != e_row) {
+        e = last_le(s_off, p.E + 1, t);                       // the non-empty expert holding row t
+        dest0 = s_poff[e] - s_off[e];
+        e_row = t;
+      }
+      const int row = live ? dest0 + t : 0;
+      uint8_t* item = box + r * 64;
+      const int swz = (r >> 1) & 3;
+      const BlockTable tb = live ? block_table_packed<G>(blk, s_tab + e * p.Kg) : BlockTable{-1, 0, -1, 0};
+      if (tb.lw0 >= 0) {
+        uint16_t* pv = reinterpret_cast<uint16_t*>(item + (((tb.lw0 >> 3) ^ swz) * 16) + (tb.lw0 & 7) * 2);
+        p.B[(size_t)row * p.K_L + tb.pos0] = *pv;
+        *pv = 0;
+      }
+      if (G == 16 && tb.lw1 >= 0) {
+        uint16_t* pv = reinterpret_cast<uint16_t*>(item + (((tb.lw1 >> 3) ^ swz) * 16) + (tb.lw1 & 7) * 2);
+        p.B[(size_t)row * p.K_L + tb.pos1] = *pv;
+        *pv = 0;
+      }
+      if (live && blk == 0)
+        for (int i = s_cnt[e]; i < p.K_L; ++i) p.B[(size_t)row * p.K_L + i] = 0;
+      uint32_t w[16];
+      load_block_smem(box, r, w);
+      const BlockTable none{-1, 0, -1, 0};
+      quant_block<G, false, false>(w, row, blk, live, none, 0, p.K, p.K_L, p.B, p.Q, p.S, live);
+    }
+    __syncwarp();
+    if (step + 2 * wstride < cta_end) { fence_proxy_async_smem(); issue(step + 2 * wstride, slot); }
+  }
+  // tail: the padded space's rows past each expert's tokens get zero codes, scales and B
+  const uint32_t pad_items = (uint32_t)(p.Mp - T) * (uint32_t)nblk;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < pad_items; i += gridDim.x * blockDim.x) {
+    const int pr = (int)(i / (uint32_t)nblk), blk = (int)(i - (uint32_t)pr * nblk);
+    int lo = 0, hi = p.E - 1;                                 // largest e with poff[e] - off[e] <= pr
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_poff[mid] - s_off[mid] <= pr) lo = mid; else hi = mid - 1;
+    }
+    const int row = s_off[lo + 1] + pr;
+    *reinterpret_cast<uint4*>(p.Q + (size_t)row * (p.K / 2) + (size_t)blk * 16) = make_uint4(0u, 0u, 0u, 0u);
+    if (G == 16) *reinterpret_cast<uint16_t*>(p.S + scale_byte_offset(row, 2 * blk, nblk / 2)) = 0;
+    else p.S[scale_byte_offset(row, blk, nblk / 4)] = 0;
+    if (blk == 0)
+      for (int c = 0; c < p.K_L; ++c) p.B[(size_t)row * p.K_L + c] = 0;
+  }
+}
+
+template <int G>
+static cudaError_t launch_grouped_tma_g(const CUtensorMap& tmX, const GroupedQuantParams& p, int T, int grid,
+                                        size_t smem, cudaStream_t s) {
+  static PerDeviceOnce smem_attr;
+  const cudaError_t ae = smem_attr.run([] {
+    return cudaFuncSetAttribute(quantize_grouped_tma_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                GROUPED_TMA_SMEM_MAX);
+  });
+  if (ae != cudaSuccess) return ae;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_grouped_tma_kernel<G>, tmX, p, T);
+}
+
+// T = off[E], the routed rows of X (the tensor map covers exactly these rows).
+cudaError_t launch_quantize_grouped_tma(const CUtensorMap& tmX, const GroupedQuantParams& p, int T, int num_sms,
+                                        cudaStream_t s) {
+  if (p.Mp == 0) return cudaSuccess;
+  const size_t smem = grouped_tma_smem(p.E, p.Kg);
+  if (smem > (size_t)GROUPED_TMA_SMEM_MAX) return cudaErrorInvalidValue;
+  const int per_sm = std::max(1, std::min(QMAXK, (int)(227 * 1024 / (smem + 1024))));
+  const long long steps = std::max<long long>(1, ((long long)T * (p.K / 32) + QSTEP - 1) / QSTEP);
+  int grid = 1;
+  long long best = -1;
+  for (int k = 1; k <= per_sm; ++k) {
+    const long long ctas = std::max<long long>(1, std::min<long long>((steps + QWARPS - 1) / QWARPS, (long long)num_sms * k));
+    const long long busiest = ((steps + ctas - 1) / ctas + QWARPS - 1) / QWARPS;
+    if (best < 0 || busiest <= best) { best = busiest; grid = (int)ctas; }
+  }
+  switch (p.G) {
+    case 16: return launch_grouped_tma_g<16>(tmX, p, T, grid, smem, s);
+    case 32: return launch_grouped_tma_g<32>(tmX, p, T, grid, smem, s);
+    case 64: return launch_grouped_tma_g<64>(tmX, p, T, grid, smem, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// Grouped (MoE) form, one lane per block with plain loads: the fallback for tables too large
+// to stage beside the TMA boxes. Over the padded row space: a row's expert comes from its 128-row block;
 // rows past the expert's token count are padding and come out as zeros. The CTA stages every
 // expert's table (E x Kg entries) with per-expert B columns.
 template <int G>

@@ -47,6 +47,7 @@ def lib() -> ctypes.CDLL:
             "osc_build_table": ([P, i32, i32, i32, f32, i32, P, P], i32),
             "osc_density": ([P, i32, i32, i32, f32, P, P, P, P], i32),
             "osc_select_tier": ([P, P, i32, P], i32),
+            "osc_select_group_size": ([P, P], i32),
             "osc_quantize": ([P, i32, i32, i32, P, i32, P, P, P, P], i32),
             "osc_rmsnorm_quantize": ([P, P, f32, i32, i32, i32, P, i32, P, P, P, P], i32),
             "osc_prepare_weight": ([P, i32, i32, i32, P, i32, P, P, P, P], i32),
@@ -56,7 +57,7 @@ def lib() -> ctypes.CDLL:
             "osc_quantize_fp8": ([P, i32, i32, P, P, P], i32),
             "osc_linear_fp8_fallback": ([P, P, P, P, i32, i32, i32, P, P, P], i32),
             "osc_grouped_plan": ([P, i32, P, P, P, i32], i32),
-            "osc_quantize_grouped": ([P, i32, P, P, P, i32, i32, i32, P, i32, P, P, P, P], i32),
+            "osc_quantize_grouped": ([P, i32, i32, P, P, P, i32, i32, i32, P, i32, P, P, P, P], i32),
             "osc_linear_grouped": ([P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P], i32),
             "osc_status": ([P, P], i32),
             "osc_selftest_timeout": ([i32, P], i32),
@@ -147,6 +148,17 @@ def osc_select_tier(n_hit, n_total):
     return int(rc), float(c.value)
 
 
+def osc_select_group_size(c_bar16: float, c_bar32: float, c_bar64: float):
+    """(G, tier) for one module from its C-bar at G = 16, 32, 64; G = 0 means the MXFP8
+    fallback. Host logic of the library (include/osc.h)."""
+    arr = (ctypes.c_double * 3)(c_bar16, c_bar32, c_bar64)
+    tier = ctypes.c_int(0)
+    g = lib().osc_select_group_size(arr, ctypes.byref(tier))
+    if g < 0:
+        _check("osc_select_group_size", g)
+    return int(g), int(tier.value)
+
+
 def osc_quantize(X, G: int, L, K_L: int, QX, SX, B, stream=None):
     M, K = X.shape
     _check("osc_quantize", lib().osc_quantize(_ptr(X), M, K, G, _ptr(L), K_L, _ptr(QX), _ptr(SX),
@@ -217,8 +229,8 @@ def osc_grouped_plan(counts):
 
 
 def osc_quantize_grouped(X, E: int, off, poff, mblock_expert, Mp: int, G: int, L, K_L: int, QX, SX, B, stream=None):
-    K = X.shape[1]
-    _check("osc_quantize_grouped", lib().osc_quantize_grouped(_ptr(X), E, _ptr(off), _ptr(poff), _ptr(mblock_expert),
+    T, K = X.shape
+    _check("osc_quantize_grouped", lib().osc_quantize_grouped(_ptr(X), T, E, _ptr(off), _ptr(poff), _ptr(mblock_expert),
                                                               Mp, K, G, _ptr(L), K_L, _ptr(QX), _ptr(SX),
                                                               _ptr(B) if K_L else None, _stream(stream)))
 
