@@ -47,8 +47,9 @@ def lib():
         L.orc_build_table.argtypes = [P, i32, i32, i32, f32, i32, P]
         L.orc_density.argtypes = [P, i32, i32, i32, f32, P, P, P]
         L.orc_table_count.argtypes = [P, i32]
-        L.orc_extract.argtypes = [P, i32, i32, i32, P, i32, P, P]
-        L.orc_gather_wl.argtypes = [P, i32, i32, i32, P, i32, P]
+        L.orc_extract.argtypes = [P, i32, i32, i32, P, i32, i32, P, P]
+        L.orc_gather_wl.argtypes = [P, i32, i32, i32, P, i32, i32, P]
+        L.orc_build_table_multi.argtypes = [P, i32, i32, i32, f32, i32, i32, P]
         L.orc_mx_quantize.argtypes = [P, i32, i32, i32, i32, P, P]
         L.orc_mx_dequantize.argtypes = [P, P, i32, i32, i32, i32, P]
         L.orc_linear.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, P, i32, P]
@@ -92,6 +93,26 @@ def build_table(X: np.ndarray, G: int, alpha: float = 5.0, min_hits: int = 5) ->
     return L
 
 
+def build_table_multi(X: np.ndarray, G: int, R: int, alpha: float = 5.0, min_hits: int = 5) -> np.ndarray:
+    """Up to R protected channels per group: K/G x R int8 (slot r from round r of Algorithm 1
+    on the calibration rows with the earlier rounds' channels zeroed)."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    S, K = X.shape
+    L = np.empty((K // G, R), dtype=np.int8)
+    _chk(lib().orc_build_table_multi(_p(X), S, K, G, float(alpha), int(min_hits), int(R), _p(L)),
+         "build_table_multi")
+    return L
+
+
+def _table_shape(L: np.ndarray, K: int, G: int):
+    """A table as K/G entries (one per group) or K/G x R entries: (flat int8 array, R)."""
+    L = np.ascontiguousarray(L, dtype=np.int8)
+    R = 1 if L.ndim == 1 else L.shape[1]
+    if L.size != (K // G) * R:
+        raise ValueError("table size does not match K / G")
+    return L.reshape(-1), R
+
+
 def density(X: np.ndarray, G: int, L: np.ndarray, alpha: float = 5.0):
     """Per-group (N_hit, N_total) of the clustering density C_k = N_hit / N_total."""
     X = np.ascontiguousarray(X, dtype=np.uint16)
@@ -104,28 +125,30 @@ def density(X: np.ndarray, G: int, L: np.ndarray, alpha: float = 5.0):
 
 
 def table_count(L: np.ndarray) -> int:
-    L = np.ascontiguousarray(L, dtype=np.int8)
+    """Number of table entries >= 0 (any table shape)."""
+    L = np.ascontiguousarray(L, dtype=np.int8).reshape(-1)
     return int(lib().orc_table_count(_p(L), L.size))
 
 
 def extract(X: np.ndarray, G: int, L: np.ndarray, K_L: int):
-    """Outlier extraction: returns (X with table slots zeroed, B as M x K_L bf16 bits)."""
+    """Outlier extraction: returns (X with table slots zeroed, B as M x K_L bf16 bits). L is
+    one entry per group (K/G) or K/G x R entries (columns of B in group, slot order)."""
     X = np.ascontiguousarray(X, dtype=np.uint16)
-    L = np.ascontiguousarray(L, dtype=np.int8)
     M, K = X.shape
+    Lf, R = _table_shape(L, K, G)
     Xz = np.empty_like(X)
     B = np.empty((M, K_L), dtype=np.uint16)
-    _chk(lib().orc_extract(_p(X), M, K, G, _p(L), K_L, _p(Xz), _p(B)), "extract")
+    _chk(lib().orc_extract(_p(X), M, K, G, _p(Lf), R, K_L, _p(Xz), _p(B)), "extract")
     return Xz, B
 
 
 def gather_wl(W: np.ndarray, G: int, L: np.ndarray, K_L: int) -> np.ndarray:
     """W_L: N x K_L bf16 bits, the weight columns of the table's channels."""
     W = np.ascontiguousarray(W, dtype=np.uint16)
-    L = np.ascontiguousarray(L, dtype=np.int8)
     N, K = W.shape
+    Lf, R = _table_shape(L, K, G)
     WL = np.empty((N, K_L), dtype=np.uint16)
-    _chk(lib().orc_gather_wl(_p(W), N, K, G, _p(L), K_L, _p(WL)), "gather_wl")
+    _chk(lib().orc_gather_wl(_p(W), N, K, G, _p(Lf), R, K_L, _p(WL)), "gather_wl")
     return WL
 
 

@@ -158,6 +158,36 @@ int orc_density(const uint16_t* X, int S, int K, int G, float alpha,
     return 0;
 }
 
+/* Protection of up to R channels per group (§6, "multi-outlier protection" for extreme
+ * cases; the page gives no procedure). READING: R rounds of Algorithm 1; round r runs on the
+ * calibration activations with the channels of rounds 0 .. r-1 set to zero, i.e. on what
+ * extraction would leave, so a further channel is protected only when it is still a consistent
+ * outlier once the stronger ones are out. L holds K/G x R entries, slot r of group k at
+ * L[k*R + r]; a group whose round r finds nothing keeps -1 from there on (later rounds see the
+ * same data). R = 1 is orc_build_table. */
+int orc_build_table_multi(const uint16_t* X, int S, int K, int G, float alpha,
+                          int min_hits, int R, int8_t* L)
+{
+    if (!X || !L || S < 0 || K <= 0 || G <= 0 || K % G != 0 || R < 1) return -1;
+    int Kg = K / G;
+    uint16_t* work = (uint16_t*)malloc((size_t)S * (size_t)K * sizeof(uint16_t) + 1);
+    int8_t* Lr = (int8_t*)malloc((size_t)Kg + 1);
+    if (!work || !Lr) { free(work); free(Lr); return -1; }
+    memcpy(work, X, (size_t)S * (size_t)K * sizeof(uint16_t));
+    int rc = 0;
+    for (int r = 0; r < R && rc == 0; ++r) {
+        rc = orc_build_table(work, S, K, G, alpha, min_hits, Lr);
+        for (int k = 0; k < Kg && rc == 0; ++k) {
+            L[k * R + r] = Lr[k];
+            if (Lr[k] >= 0)
+                for (int t = 0; t < S; ++t) work[(int64_t)t * K + k * G + Lr[k]] = 0x0000u;
+        }
+    }
+    free(work);
+    free(Lr);
+    return rc;
+}
+
 /* ---- Outlier extraction (§3.2, Figure 2 caption) ----------------------------
  *
  * For every group k whose table entry is j = L[k] >= 0, the value
@@ -174,27 +204,31 @@ int orc_table_count(const int8_t* L, int Kg)
     return c;
 }
 
-int orc_extract(const uint16_t* X, int M, int K, int G, const int8_t* L,
+int orc_extract(const uint16_t* X, int M, int K, int G, const int8_t* L, int R,
                 int K_L, uint16_t* Xz, uint16_t* B)
 {
-    if (!X || !L || !Xz || M < 0 || K <= 0 || G <= 0 || K % G) return -1;
+    if (!X || !L || !Xz || M < 0 || K <= 0 || G <= 0 || K % G || R < 1) return -1;
     int Kg = K / G;
-    int cnt = orc_table_count(L, Kg);
+    int cnt = orc_table_count(L, Kg * R);
     if (K_L < cnt || (K_L > 0 && !B)) return -1;
-    for (int k = 0; k < Kg; ++k)
-        if (L[k] >= G) return -1;
+    for (int i = 0; i < Kg * R; ++i)
+        if (L[i] >= G) return -1;
     memcpy(Xz, X, (size_t)M * (size_t)K * sizeof(uint16_t));
     for (int64_t i = 0; i < (int64_t)M * K_L; ++i) B[i] = 0;
+    /* entries in (group, slot) order; each copies what the earlier ones left in the slot, so
+     * a channel named twice gives its value once and 0 the second time */
     int pos = 0;
-    for (int k = 0; k < Kg; ++k) {
-        if (L[k] < 0) continue;
-        int c = k * G + L[k];
-        for (int t = 0; t < M; ++t) {
-            B[(int64_t)t * K_L + pos] = X[(int64_t)t * K + c];
-            Xz[(int64_t)t * K + c] = 0x0000u;
+    for (int k = 0; k < Kg; ++k)
+        for (int m = 0; m < R; ++m) {
+            int j = L[k * R + m];
+            if (j < 0) continue;
+            int c = k * G + j;
+            for (int t = 0; t < M; ++t) {
+                B[(int64_t)t * K_L + pos] = Xz[(int64_t)t * K + c];
+                Xz[(int64_t)t * K + c] = 0x0000u;
+            }
+            ++pos;
         }
-        ++pos;
-    }
     return 0;
 }
 
@@ -203,21 +237,23 @@ int orc_extract(const uint16_t* X, int M, int K, int G, const int8_t* L,
  * channels), the i-th table channel c_i = k_i*G + L[k_i] gives
  * W_L[n][i] = W[n][c_i]; pad columns are zero. Then B * W_L^T supplies the
  * outlier channels' contribution to Y. */
-int orc_gather_wl(const uint16_t* W, int N, int K, int G, const int8_t* L,
+int orc_gather_wl(const uint16_t* W, int N, int K, int G, const int8_t* L, int R,
                   int K_L, uint16_t* WL)
 {
-    if (!W || !L || N < 0 || K <= 0 || G <= 0 || K % G) return -1;
+    if (!W || !L || N < 0 || K <= 0 || G <= 0 || K % G || R < 1) return -1;
     int Kg = K / G;
-    int cnt = orc_table_count(L, Kg);
+    int cnt = orc_table_count(L, Kg * R);
     if (K_L < cnt || (K_L > 0 && !WL)) return -1;
     for (int64_t i = 0; i < (int64_t)N * K_L; ++i) WL[i] = 0;
     int pos = 0;
-    for (int k = 0; k < Kg; ++k) {
-        if (L[k] < 0) continue;
-        int c = k * G + L[k];
-        for (int n = 0; n < N; ++n) WL[(int64_t)n * K_L + pos] = W[(int64_t)n * K + c];
-        ++pos;
-    }
+    for (int k = 0; k < Kg; ++k)
+        for (int m = 0; m < R; ++m) {
+            int jw = L[(int64_t)k * R + m];
+            if (jw < 0) continue;
+            int c = k * G + jw;
+            for (int n = 0; n < N; ++n) WL[(int64_t)n * K_L + pos] = W[(int64_t)n * K + c];
+            ++pos;
+        }
     return 0;
 }
 

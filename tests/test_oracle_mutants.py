@@ -136,6 +136,19 @@ MUTANTS = [
     ("weights_decoded_as_e2m1", "c",
      "qw[k] = (fmt == ORC_FMT_E2M1) ? orc_decode_e2m1(c) : orc_decode_e4m3(c);",
      "qw[k] = orc_decode_e2m1(c);"),
+    # several protected channels per group
+    ("multi_round_sees_earlier_channels", "c",
+     "for (int t = 0; t < S; ++t) work[(int64_t)t * K + k * G + Lr[k]] = 0x0000u;",
+     "(void)0;"),
+    ("multi_extract_copies_original", "c",
+     "B[(int64_t)t * K_L + pos] = Xz[(int64_t)t * K + c];",
+     "B[(int64_t)t * K_L + pos] = X[(int64_t)t * K + c];"),
+    ("multi_wl_first_slot_only", "c",
+     "int jw = L[(int64_t)k * R + m];",
+     "int jw = L[(int64_t)k * R];"),
+    ("multi_extract_slot_ignored", "c",
+     "int j = L[k * R + m];",
+     "int j = L[k * R];"),
     # the RMSNorm step before the quantize (its order of operations is a stated reading)
     ("rms_sum_left_to_right_over_blocks", "c",
      "for (int h = P / 2; h >= 1; h /= 2)\n        for (int b = 0; b < h; ++b) s[b] = s[b] + s[b + h];",

@@ -567,3 +567,72 @@ def test_rmsnorm_then_osc_is_osc_of_the_normalized_rows(oracle):
     for key in ("cx", "ex", "B"):
         assert np.array_equal(fused[key], plain[key]), key
     assert np.array_equal(fused["Y"], plain["Y"])
+
+
+# ---- several protected channels per group (multi-outlier protection) ----------------------
+
+def test_multi_table_finds_planted_second_channels(oracle):
+    """Two persistent outliers in group 0 (channels 3 and 20), one in group 1 (channel 7), none
+    in group 2, and in group 3 a second outlier on only 3 tokens (below min_hits): round 1
+    finds the larger of each pair, round 2 the smaller one once the first is zeroed, and slots
+    stay -1 once a round finds nothing. R = 1 is the single-entry table."""
+    rng = np.random.default_rng(21)
+    S, G = 60, 32
+    X = rng.standard_normal((S, 4 * G)) * 0.5
+    X[:, 0 * G + 3] = 100.0 * rng.choice([-1, 1], S)
+    X[:, 0 * G + 20] = 60.0 * rng.choice([-1, 1], S)
+    X[:, 1 * G + 7] = -90.0
+    X[:, 3 * G + 11] = 80.0
+    X[:3, 3 * G + 30] = 70.0
+    Xb = I.bf16_bits(X)
+    L3 = oracle.build_table_multi(Xb, G, 3)
+    assert L3.tolist() == [[3, 20, -1], [7, -1, -1], [-1, -1, -1], [11, -1, -1]]
+    assert np.array_equal(oracle.build_table_multi(Xb, G, 1)[:, 0], oracle.build_table(Xb, G))
+    q = I.qkv_case(1)                                         # one planted channel per group
+    L2 = oracle.build_table_multi(q.calib, 32, 2)
+    assert np.array_equal(L2[:, 0], q.planted) and np.all(L2[:, 1] == -1)
+
+
+def test_multi_extract_order_and_repeated_channel(oracle):
+    """Entries are taken in (group, slot) order, each moved to its own B column and zeroed;
+    a channel named twice in one group gives its value once and 0 the second time; W_L takes
+    the same columns in the same order."""
+    rng = np.random.default_rng(22)
+    M, K, G = 5, 128, 32
+    X = I.bf16_bits(rng.standard_normal((M, K)))
+    L = np.array([[4, 9], [-1, -1], [30, 30], [0, -1]], np.int8)
+    Xz, B = oracle.extract(X, G, L, 16)
+    cols = [0 * G + 4, 0 * G + 9, 2 * G + 30, 3 * G + 0]
+    assert np.array_equal(B[:, [0, 1, 2, 4]], X[:, cols])
+    assert np.all(B[:, 3] == 0) and np.all(B[:, 5:] == 0)      # the repeated channel, the pad
+    assert np.all(Xz[:, cols] == 0)
+    keep = np.ones(K, bool); keep[cols] = False
+    assert np.array_equal(Xz[:, keep], X[:, keep])
+    W = I.bf16_bits(rng.standard_normal((7, K)))
+    WL = oracle.gather_wl(W, G, L, 16)
+    assert np.array_equal(WL[:, :5], W[:, [cols[0], cols[1], cols[2], cols[2], cols[3]]])
+    assert oracle.table_count(L) == 5 and np.all(WL[:, 5:] == 0)
+
+
+def test_multi_osc_is_exact_on_representable_inputs(oracle):
+    """With two large outliers in some groups, a two-slot table makes the dual-path output
+    equal X W^T exactly (both channels ride the 16-bit path); keeping only the first slot
+    leaves the second outlier to set its block's scale and the product visibly off."""
+    rng = np.random.default_rng(23)
+    M, K, N, G = 16, 256, 24, 32
+    x = _representable(rng, M, K)
+    w = _representable(rng, N, K)
+    L = np.array([[5, 17], [-1, -1], [0, 31], [12, -1], [-1, -1], [2, 3], [7, -1], [-1, -1]], np.int8)
+    for k in range(8):
+        for j in L[k]:
+            if j >= 0:
+                x[:, k * G + int(j)] = rng.choice([-1, 1], size=M) * rng.uniform(200, 900, size=M)
+    X, W = I.bf16_bits(x), I.bf16_bits(w)
+    xf, wf = I.bf16_to_f32(X).astype(np.float64), I.bf16_to_f32(W).astype(np.float64)
+    cw, ew, WL = oracle.osc_prepare_weight(W, G, L, 16)
+    r = oracle.osc_forward(X, G, L, 16, cw, ew, WL)
+    assert np.allclose(r["Y"], xf @ wf.T, rtol=1e-13, atol=1e-9)
+    L1 = L[:, 0].copy()
+    cw1, ew1, WL1 = oracle.osc_prepare_weight(W, G, L1, 16)
+    r1 = oracle.osc_forward(X, G, L1, 16, cw1, ew1, WL1)
+    assert np.abs(r1["Y"] - xf @ wf.T).max() > 1.0
