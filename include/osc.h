@@ -79,7 +79,8 @@ enum {
   OSC_ERR_CUDA = -4,     /* a CUDA runtime/driver call failed; see osc_last_cuda_error() */
   OSC_ERR_TIMEOUT = -5,  /* (from osc_status) a kernel's bounded wait ran out */
   OSC_ERR_TABLE = -6,    /* (from osc_status) a table entry >= G or more entries than K_L */
-  OSC_ERR_DEVICE = -7    /* the current device is not an sm_100 GPU */
+  OSC_ERR_DEVICE = -7,   /* the current device is not an sm_100 GPU */
+  OSC_ERR_SCRATCH = -8   /* (osc_linear_splitk_noalloc) the call needs more than its fixed scratch */
 };
 
 /* Library version string. */
@@ -188,6 +189,30 @@ OSC_API int osc_linear_splitk(const uint8_t* QX, const uint8_t* SX, const uint16
                               const uint8_t* QW, const uint8_t* SW, const uint16_t* WL,
                               int M, int N, int K, int G, int K_L, uint16_t* Y, float* Yf32,
                               float* workspace, size_t workspace_bytes, osc_stream_t stream);
+
+/* Allocation-free form of osc_linear_splitk (the OSC page has no counterpart: this is a
+ * deployment convenience of this library). Some callers cannot allocate device memory at all:
+ * plugins of an inference engine that owns every device buffer and hands a plugin only its
+ * inputs and outputs, or serving loops that forbid allocation after start-up (an allocation
+ * there could fail under fragmentation or stall other streams). They cannot provide the
+ * workspace osc_linear_splitk needs, so this entry point keeps the fp32 partials in one fixed
+ * buffer inside the library instead: OSC_NOALLOC_SCRATCH_BYTES (16 MiB) of device memory that
+ * every GPU which loads the library holds until the process exits. Arguments and results as
+ * osc_linear_splitk without the workspace; the library still allocates nothing, and the caller
+ * passes inputs and outputs as usual.
+ *   - The first call on a device looks up the buffer's device address (once per device, with
+ *     that device current); make that first call before any stream capture.
+ *   - A call whose split needs more partial bytes than the buffer holds (S x M x N x 4, see
+ *     osc_linear_workspace_bytes) returns OSC_ERR_SCRATCH and launches nothing; calls that
+ *     need no split (M > 128, or one part per weight tile) use no scratch.
+ *   - Every call shares the one buffer and it keeps the last call's contents; nothing in it
+ *     needs to start at zero (each call writes every partial it reads). Calls that overlap on
+ *     the GPU (different streams, or different host threads without ordering) race on it. */
+#define OSC_NOALLOC_SCRATCH_BYTES (16u << 20)
+OSC_API int osc_linear_splitk_noalloc(const uint8_t* QX, const uint8_t* SX, const uint16_t* B,
+                                      const uint8_t* QW, const uint8_t* SW, const uint16_t* WL,
+                                      int M, int N, int K, int G, int K_L, uint16_t* Y, float* Yf32,
+                                      osc_stream_t stream);
 
 /* §4 FP8 fallback, quantize side: X (M x K bf16) -> QX8 (M x K E4M3 codes),
  * SX (osc_scale_bytes(M, K, 0)); per-32 E8M0 scales, no separation. Also used for the

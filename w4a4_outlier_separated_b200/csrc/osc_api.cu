@@ -295,6 +295,7 @@ const char* osc_error_string(int code) {
     case OSC_ERR_TIMEOUT: return "a kernel wait ran out of time";
     case OSC_ERR_TABLE: return "table entry out of range or more entries than K_L";
     case OSC_ERR_DEVICE: return "current device is not an sm_100 GPU";
+    case OSC_ERR_SCRATCH: return "the split needs more partials than the fixed 16 MiB scratch holds";
     default: return "unknown error";
   }
 }
@@ -621,3 +622,60 @@ int osc_status(int* raw, osc_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---- the allocation-free split product ------------------------------------------------------
+// Some callers cannot allocate device memory (an engine plugin that is handed only its inputs
+// and outputs, a serving loop that forbids allocation after start-up), so they cannot give
+// osc_linear_splitk a workspace. For them the partials live in this fixed, file-scope device
+// buffer. In host code the name g_noalloc_scratch is only a host-side stand-in; the kernels get
+// the device address that cudaGetSymbolAddress returns, looked up once per device.
+namespace {
+
+static __device__ __align__(256) float g_noalloc_scratch[OSC_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+struct ScratchAddr {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+  float* ptr = nullptr;
+};
+
+// Device address of the buffer on the current device (looked up on the first call for it).
+int noalloc_scratch(float** out) {
+  static ScratchAddr addr[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (dev < 0 || dev >= kMaxDevices) return OSC_ERR_DEVICE;
+  ScratchAddr& a = addr[dev];
+  std::call_once(a.once, [&] {
+    void* p = nullptr;
+    a.err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    a.ptr = static_cast<float*>(p);
+  });
+  if (a.err != cudaSuccess) return fail_cuda(a.err);
+  *out = a.ptr;
+  return OSC_OK;
+}
+
+}  // namespace
+
+extern "C" int osc_linear_splitk_noalloc(const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const uint8_t* QW,
+                                         const uint8_t* SW, const uint16_t* WL, int M, int N, int K, int G, int K_L,
+                                         uint16_t* Y, float* Yf32, osc_stream_t stream) {
+  if (!valid_g(G)) return OSC_ERR_G;
+  if (M == 0 && N > 0 && K > 0 && K_L >= 0) return OSC_OK;  // nothing to read or write
+  int rc = check_linear_common(QX, SX, QW, SW, M, N, K, Y, Yf32);
+  if (rc != OSC_OK) return rc;
+  if (K_L < 0 || K_L % 16 != 0) return K_L < 0 ? OSC_ERR_ARG : OSC_ERR_ALIGN;
+  if (K_L > 0 && (!B || !WL)) return OSC_ERR_ARG;
+  if (K_L > 0 && (!a16(B) || !a16(WL))) return OSC_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(&ds)) != OSC_OK) return rc;
+  const int kind = G == 16 ? osc::KIND_MXF4_B16 : osc::KIND_MXF4_B32;
+  if (M <= 128 && small_plan(kind, M, N, K, K_L, ds->sms, true).partial_bytes > (size_t)OSC_NOALLOC_SCRATCH_BYTES)
+    return OSC_ERR_SCRATCH;
+  float* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch)) != OSC_OK) return rc;
+  return run_gemm(kind, QX, SX, B, QW, SW, WL, M, N, K, K_L, 1, nullptr, nullptr, Y, Yf32, (cudaStream_t)stream,
+                  scratch, (size_t)OSC_NOALLOC_SCRATCH_BYTES);
+}

@@ -17,7 +17,8 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libosc.so"
 
 OSC_OK = 0
 ERRORS = {-1: "OSC_ERR_ARG", -2: "OSC_ERR_ALIGN", -3: "OSC_ERR_G", -4: "OSC_ERR_CUDA",
-          -5: "OSC_ERR_TIMEOUT", -6: "OSC_ERR_TABLE", -7: "OSC_ERR_DEVICE"}
+          -5: "OSC_ERR_TIMEOUT", -6: "OSC_ERR_TABLE", -7: "OSC_ERR_DEVICE",
+          -8: "OSC_ERR_SCRATCH"}
 
 
 class OSCError(RuntimeError):
@@ -54,6 +55,7 @@ def lib() -> ctypes.CDLL:
             "osc_linear": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P], i32),
             "osc_linear_workspace_bytes": ([i32, i32, i32, i32], ctypes.c_size_t),
             "osc_linear_splitk": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P, ctypes.c_size_t, P], i32),
+            "osc_linear_splitk_noalloc": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P], i32),
             "osc_quantize_fp8": ([P, i32, i32, P, P, P], i32),
             "osc_linear_fp8_fallback": ([P, P, P, P, i32, i32, i32, P, P, P], i32),
             "osc_grouped_plan": ([P, i32, P, P, P, i32], i32),
@@ -198,6 +200,15 @@ def osc_linear_splitk(QX, SX, B, QW, SW, WL, M: int, N: int, K: int, G: int, K_L
                                                         _ptr(SW), _ptr(WL) if K_L else None, M, N, K, G, K_L,
                                                         _ptr(Y), _ptr(Yf32), _ptr(workspace), nbytes,
                                                         _stream(stream)))
+
+
+def osc_linear_splitk_noalloc(QX, SX, B, QW, SW, WL, M: int, N: int, K: int, G: int, K_L: int, Y, Yf32=None,
+                              stream=None):
+    """osc_linear_splitk with the partials in the library's fixed device buffer (no workspace):
+    for callers that cannot allocate device memory."""
+    _check("osc_linear_splitk_noalloc", lib().osc_linear_splitk_noalloc(
+        _ptr(QX), _ptr(SX), _ptr(B) if K_L else None, _ptr(QW), _ptr(SW), _ptr(WL) if K_L else None,
+        M, N, K, G, K_L, _ptr(Y), _ptr(Yf32), _stream(stream)))
 
 
 def osc_quantize_fp8(X, QX8, SX, stream=None):
