@@ -46,9 +46,11 @@
  *            rows hold 0. Size: osc_scale_bytes().
  *            Shared exponent e = floor(log2(amax)) - 2 (E2M1) or - 8 (E4M3), clamped to
  *            [-127, 127]; an all-zero block gets e = -127.
- *   L        int8, K/G entries: local channel 0..G-1 of the group's outlier, or -1.
- *   B        M x K_L bf16: column i holds the i-th table channel (groups with L >= 0 in
- *            ascending order); columns past the entry count are 0.
+ *   L        int8, K/G x R entries (R = 1..3 protected channels per group): slot r of group k
+ *            at L[k*R + r], the local channel 0..G-1 of an outlier, or -1.
+ *   B        M x K_L bf16: column i holds the i-th table entry >= 0 in (group, slot) order;
+ *            columns past the entry count are 0. Entries are moved out in that order, so a
+ *            channel named twice in a group gives its value once and 0 the second time.
  *   W_L      N x K_L bf16: W_L[n][i] = W[n][channel of table entry i]; pad columns 0.
  *   K_L      the compensation width: the number of table entries rounded up to a multiple
  *            of 16 (osc_table_kl), or any larger multiple of 16.
@@ -94,8 +96,9 @@ OSC_API int osc_last_cuda_error(void);
  * or for the MXFP8 path when G == 0. Returns 0 on invalid arguments. */
 OSC_API size_t osc_scale_bytes(int rows, int K, int G);
 
-/* K_L for a table held in HOST memory: count of entries >= 0, rounded up to 16. */
-OSC_API int osc_table_kl(const int8_t* L_host, int Kg);
+/* K_L for a table held in HOST memory: count of its n entries (K/G x R) that are >= 0, rounded
+ * up to 16. */
+OSC_API int osc_table_kl(const int8_t* L_host, int n);
 
 /* §3.1 Algorithm 1 (offline), one (position, layer): S x K calibration activations Xcal
  * -> L (K/G entries, device). alpha is the page's threshold (default 5); min_hits is the
@@ -105,6 +108,15 @@ OSC_API int osc_table_kl(const int8_t* L_host, int Kg);
  * events (lowest on ties) if it has >= min_hits, else -1. */
 OSC_API int osc_build_table(const uint16_t* Xcal, int S, int K, int G, float alpha, int min_hits,
                     int8_t* L, osc_stream_t stream);
+
+/* §6 multi-outlier protection (up to R = 1..3 channels per group, "for extreme cases"; the
+ * page gives no procedure): R rounds of the osc_build_table rule, round r counting events with
+ * the channels of rounds 0 .. r-1 read as zero (what extraction leaves of the group), so a
+ * further channel is protected only while it stays a consistent outlier once the stronger ones
+ * are out. L receives K/G x R entries (device), slot r of group k at L[k*R + r]; once a round
+ * finds no channel for a group its later slots are -1. R = 1 is osc_build_table. */
+OSC_API int osc_build_table_multi(const uint16_t* Xcal, int S, int K, int G, float alpha, int min_hits,
+                                  int R, int8_t* L, osc_stream_t stream);
 
 /* §2.2 clustering density of a table on S x K activations X (device), with the event of
  * osc_build_table: n_total[k] counts group k's outlier events over the S tokens and n_hit[k]
@@ -141,9 +153,10 @@ OSC_API int osc_select_group_size(const double* c_bar, int* tier);
 
 /* §3.2, Figure 2 (online): extraction + zeroing through the table, then MXFP4 quantization
  * of the zeroed tensor. X (M x K bf16) -> QX (M x K/2), SX (osc_scale_bytes(M, K, G)),
- * B (M x K_L bf16). L may be NULL (no table: plain MXFP4; then K_L must be 0 and B may be
- * NULL). X is not modified. With a table, K/G may be at most 1024. */
-OSC_API int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int K_L,
+ * B (M x K_L bf16). L: K/G x R entries (R = 1..3 protected channels per group, see L below),
+ * or NULL (no table: plain MXFP4; then K_L must be 0, B may be NULL and R is not used, pass 1).
+ * X is not modified. With a table, K/G x R may be at most 4096. */
+OSC_API int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int R, int K_L,
                  uint8_t* QX, uint8_t* SX, uint16_t* B, osc_stream_t stream);
 
 /* Figure 2 (§3.2) with the step that produces the projection's input: RMSNorm of each row,
@@ -155,13 +168,13 @@ OSC_API int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L
  * bf16((x * inv) * gamma). Outputs and table arguments as osc_quantize (the table comes from
  * calibration rows that were normalized the same way). K must be at most 6144. */
 OSC_API int osc_rmsnorm_quantize(const uint16_t* X, const uint16_t* gamma, float eps, int M, int K, int G,
-                                 const int8_t* L, int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B,
+                                 const int8_t* L, int R, int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B,
                                  osc_stream_t stream);
 
 /* §3.3 weight side (offline): W (N x K bf16) -> QW (N x K/2), SW (osc_scale_bytes(N, K, G))
  * quantized with no table (its outlier columns meet zeroed activations), and
- * W_L (N x K_L bf16) gathered through L (device; may be NULL when K_L == 0). */
-OSC_API int osc_prepare_weight(const uint16_t* W, int N, int K, int G, const int8_t* L, int K_L,
+ * W_L (N x K_L bf16) gathered through L (K/G x R entries, device; may be NULL when K_L == 0). */
+OSC_API int osc_prepare_weight(const uint16_t* W, int N, int K, int G, const int8_t* L, int R, int K_L,
                        uint8_t* QW, uint8_t* SW, uint16_t* WL, osc_stream_t stream);
 
 /* §3.2 equation for Y: Y (M x N bf16, round to nearest even from the fp32 accumulator)
@@ -239,12 +252,13 @@ OSC_API int osc_grouped_plan(const int* counts, int E, int* off, int* poff, int*
 
 /* Per-expert extraction + MXFP4 quantization. X: T x K bf16 (device), T = off[E] the routed
  * rows (the value of off[E] on the host, passed so that the call needs no copy back). off, poff,
- * mblock_expert: device copies of the plan. L: E x K/G (device), expert e's table at e*K/G.
+ * mblock_expert: device copies of the plan. L: E x K/G x R (device), expert e's table at
+ * e*K/G*R.
  * Outputs over the padded rows: QX (Mp x K/2), SX (osc_scale_bytes(Mp, K, G)),
  * B (Mp x K_L bf16, K_L a common width >= every expert's entry count); pad rows are 0.
- * E x K/G may be at most about 68000 table entries (they are staged in shared memory). */
+ * E x K/G x R may be at most about 68000 table entries (they are staged in shared memory). */
 OSC_API int osc_quantize_grouped(const uint16_t* X, int T, int E, const int* off, const int* poff,
-                         const int* mblock_expert, int Mp, int K, int G, const int8_t* L,
+                         const int* mblock_expert, int Mp, int K, int G, const int8_t* L, int R,
                          int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B, osc_stream_t stream);
 
 /* Per-expert dual-path product over the padded rows. QW: E x N x K/2, SW: E blocks of

@@ -78,12 +78,15 @@ def test_argument_checks_return_before_any_cuda_call(lib):
     buf = (ctypes.c_uint8 * 4096)()
     p = ctypes.cast(buf, V)
     p16 = V((ctypes.addressof(buf) + 15) // 16 * 16)
-    lib.osc_quantize.argtypes = [V, ctypes.c_int, ctypes.c_int, ctypes.c_int, V, ctypes.c_int, V, V, V, V]
-    assert lib.osc_quantize(p16, 4, 256, 24, None, 0, p16, p16, None, None) == -3          # G
-    assert lib.osc_quantize(None, 4, 256, 32, None, 0, p16, p16, None, None) == -1         # null
-    assert lib.osc_quantize(p16, 4, 200, 32, None, 0, p16, p16, None, None) == -2          # K % 256
-    assert lib.osc_quantize(V(p16.value + 2), 4, 256, 32, None, 0, p16, p16, None, None) == -2  # alignment
-    assert lib.osc_quantize(p16, 4, 256, 32, None, 16, p16, p16, p16, None) == -1          # K_L without table
+    lib.osc_quantize.argtypes = [V, ctypes.c_int, ctypes.c_int, ctypes.c_int, V, ctypes.c_int, ctypes.c_int,
+                                 V, V, V, V]
+    assert lib.osc_quantize(p16, 4, 256, 24, None, 1, 0, p16, p16, None, None) == -3          # G
+    assert lib.osc_quantize(None, 4, 256, 32, None, 1, 0, p16, p16, None, None) == -1         # null
+    assert lib.osc_quantize(p16, 4, 200, 32, None, 1, 0, p16, p16, None, None) == -2          # K % 256
+    assert lib.osc_quantize(V(p16.value + 2), 4, 256, 32, None, 1, 0, p16, p16, None, None) == -2  # alignment
+    assert lib.osc_quantize(p16, 4, 256, 32, None, 1, 16, p16, p16, p16, None) == -1          # K_L without table
+    assert lib.osc_quantize(p16, 4, 256, 32, p16, 0, 0, p16, p16, None, None) == -1           # R < 1
+    assert lib.osc_quantize(p16, 4, 256, 32, p16, 4, 0, p16, p16, None, None) == -1           # R > 3
     lib.osc_linear.argtypes = [V] * 6 + [ctypes.c_int] * 5 + [V, V, V]
     assert lib.osc_linear(p16, p16, None, p16, p16, None, 4, 100, 256, 32, 0, p16, None, None) == -2  # N % 16
     assert lib.osc_linear(p16, p16, None, p16, p16, None, 4, 128, 256, 32, 8, p16, None, None) == -2  # K_L % 16
@@ -104,12 +107,13 @@ def test_argument_limits_of_every_entry_point(lib):
     buf = (ctypes.c_uint8 * 4096)()
     p16 = V((ctypes.addressof(buf) + 15) // 16 * 16)
     q = lib.osc_quantize
-    q.argtypes = [V, I, I, I, V, I, V, V, V, V]
-    assert q(p16, 4, 33024, 32, p16, 0, p16, p16, None, None) == -1        # K / G = 1032 > 1024 with a table
-    assert q(p16, 4, 4096, 32, p16, 32784, p16, p16, p16, None) == -1      # K_L > 32767
-    assert q(p16, 1 << 30, 256, 32, None, 0, p16, p16, None, None) == -1   # (M + 127) * K / 32 >= 2^31
-    assert q(p16, 4, 256, 32, p16, 16, p16, p16, None, None) == -1         # K_L > 0 needs B
-    assert q(p16, 0, 256, 32, None, 0, None, None, None, None) == 0        # M = 0: no-op, NULLs allowed
+    q.argtypes = [V, I, I, I, V, I, I, V, V, V, V]
+    assert q(p16, 4, 131328, 32, p16, 1, 0, p16, p16, None, None) == -1    # K / G = 4104 > 4096 entries
+    assert q(p16, 4, 45056, 32, p16, 3, 0, p16, p16, None, None) == -1     # 1408 groups x 3 slots > 4096
+    assert q(p16, 4, 4096, 32, p16, 1, 32784, p16, p16, p16, None) == -1   # K_L > 32767
+    assert q(p16, 1 << 30, 256, 32, None, 1, 0, p16, p16, None, None) == -1   # (M + 127) * K / 32 >= 2^31
+    assert q(p16, 4, 256, 32, p16, 1, 16, p16, p16, None, None) == -1      # K_L > 0 needs B
+    assert q(p16, 0, 256, 32, None, 1, 0, None, None, None, None) == 0     # M = 0: no-op, NULLs allowed
     li = lib.osc_linear
     li.argtypes = [V] * 6 + [I] * 5 + [V, V, V]
     assert li(None, None, None, None, None, None, 0, 128, 256, 32, 0, None, None, None) == 0   # M = 0: no-op
@@ -121,10 +125,11 @@ def test_argument_limits_of_every_entry_point(lib):
     l8.argtypes = [V, V, V, V, I, I, I, V, V, V]
     assert l8(None, None, None, None, 0, 64, 256, None, None, None) == 0  # M = 0: no-op
     w = lib.osc_prepare_weight
-    w.argtypes = [V, I, I, I, V, I, V, V, V, V]
-    assert w(p16, 4, 256, 48, None, 0, p16, p16, None, None) == -3         # G
-    assert w(p16, 4, 256, 32, None, 16, p16, p16, p16, None) == -1         # K_L > 0 needs L
-    assert w(p16, 4, 512, 32, p16, 8, p16, p16, p16, None) == -2           # K_L % 16
+    w.argtypes = [V, I, I, I, V, I, I, V, V, V, V]
+    assert w(p16, 4, 256, 48, None, 1, 0, p16, p16, None, None) == -3      # G
+    assert w(p16, 4, 256, 32, None, 1, 16, p16, p16, p16, None) == -1      # K_L > 0 needs L
+    assert w(p16, 4, 512, 32, p16, 1, 8, p16, p16, p16, None) == -2        # K_L % 16
+    assert w(p16, 4, 512, 32, p16, 5, 16, p16, p16, p16, None) == -1       # R > 3
     f8 = lib.osc_quantize_fp8
     f8.argtypes = [V, I, I, V, V, V]
     assert f8(p16, 4, 384, p16, p16, None) == -2                           # K % 256
@@ -138,12 +143,18 @@ def test_argument_limits_of_every_entry_point(lib):
     assert bt(p16, 8, 250, 32, 5.0, 5, p16, None) == -1                    # K % G
     assert bt(p16, 8, 256, 8, 5.0, 5, p16, None) == -3                     # G
     qg = lib.osc_quantize_grouped
-    qg.argtypes = [V, I, I, V, V, V, I, I, I, V, I, V, V, V, V]
-    assert qg(p16, 100, 2, p16, p16, p16, 200, 256, 32, p16, 0, p16, p16, None, None) == -2   # Mp % 128
-    assert qg(p16, 100, 2, p16, p16, p16, 256, 256, 32, None, 0, p16, p16, None, None) == -1  # tables required
-    assert qg(p16, 100, 2, p16, p16, p16, 1 << 30, 256, 32, p16, 0, p16, p16, None, None) == -1  # scale index overflow
-    assert qg(p16, 300, 2, p16, p16, p16, 256, 256, 32, p16, 0, p16, p16, None, None) == -1   # T > Mp
-    assert qg(p16, -1, 2, p16, p16, p16, 256, 256, 32, p16, 0, p16, p16, None, None) == -1    # T < 0
+    qg.argtypes = [V, I, I, V, V, V, I, I, I, V, I, I, V, V, V, V]
+    assert qg(p16, 100, 2, p16, p16, p16, 200, 256, 32, p16, 1, 0, p16, p16, None, None) == -2   # Mp % 128
+    assert qg(p16, 100, 2, p16, p16, p16, 256, 256, 32, None, 1, 0, p16, p16, None, None) == -1  # tables required
+    assert qg(p16, 100, 2, p16, p16, p16, 1 << 30, 256, 32, p16, 1, 0, p16, p16, None, None) == -1  # scale index
+    assert qg(p16, 300, 2, p16, p16, p16, 256, 256, 32, p16, 1, 0, p16, p16, None, None) == -1   # T > Mp
+    assert qg(p16, -1, 2, p16, p16, p16, 256, 256, 32, p16, 1, 0, p16, p16, None, None) == -1    # T < 0
+    assert qg(p16, 100, 2, p16, p16, p16, 256, 256, 32, p16, 0, 0, p16, p16, None, None) == -1   # R < 1
+    bm = lib.osc_build_table_multi
+    bm.argtypes = [V, I, I, I, ctypes.c_float, I, I, V, V]
+    assert bm(p16, 8, 256, 32, 5.0, 5, 4, p16, None) == -1                 # R > 3
+    assert bm(p16, 8, 256, 32, 5.0, 5, 0, p16, None) == -1                 # R < 1
+    assert bm(p16, 8, 256, 24, 5.0, 5, 2, p16, None) == -3                 # G
     lg = lib.osc_linear_grouped
     lg.argtypes = [V, V, V, V, V, V, V, V, I, I, I, I, I, I, V, V, V]
     assert lg(p16, p16, None, p16, p16, None, p16, None, 2, 200, 256, 256, 32, 0, p16, None, None) == -2  # Mp % 128
@@ -161,14 +172,15 @@ def test_argument_limits_of_every_entry_point(lib):
     stt.argtypes = [I, V]
     assert stt(0, None) == -1 and stt(2_000_000, None) == -1                # limit out of range
     rq = lib.osc_rmsnorm_quantize
-    rq.argtypes = [V, V, ctypes.c_float, I, I, I, V, I, V, V, V, V]
-    assert rq(p16, p16, -1.0, 4, 256, 32, None, 0, p16, p16, None, None) == -1       # eps < 0
-    assert rq(p16, p16, float("nan"), 4, 256, 32, None, 0, p16, p16, None, None) == -1
-    assert rq(p16, p16, 1e-6, 4, 8192, 32, None, 0, p16, p16, None, None) == -1       # K above 6144
-    assert rq(p16, None, 1e-6, 4, 256, 32, None, 0, p16, p16, None, None) == -1       # gamma required
-    assert rq(p16, V(p16.value + 2), 1e-6, 4, 256, 32, None, 0, p16, p16, None, None) == -2  # gamma alignment
-    assert rq(p16, p16, 1e-6, 4, 256, 24, None, 0, p16, p16, None, None) == -3        # G
-    assert rq(None, None, 1e-6, 0, 256, 32, None, 0, None, None, None, None) == 0     # M = 0: no-op
+    rq.argtypes = [V, V, ctypes.c_float, I, I, I, V, I, I, V, V, V, V]
+    assert rq(p16, p16, -1.0, 4, 256, 32, None, 1, 0, p16, p16, None, None) == -1       # eps < 0
+    assert rq(p16, p16, float("nan"), 4, 256, 32, None, 1, 0, p16, p16, None, None) == -1
+    assert rq(p16, p16, 1e-6, 4, 8192, 32, None, 1, 0, p16, p16, None, None) == -1       # K above 6144
+    assert rq(p16, None, 1e-6, 4, 256, 32, None, 1, 0, p16, p16, None, None) == -1       # gamma required
+    assert rq(p16, V(p16.value + 2), 1e-6, 4, 256, 32, None, 1, 0, p16, p16, None, None) == -2  # gamma alignment
+    assert rq(p16, p16, 1e-6, 4, 256, 24, None, 1, 0, p16, p16, None, None) == -3        # G
+    assert rq(None, None, 1e-6, 0, 256, 32, None, 1, 0, None, None, None, None) == 0     # M = 0: no-op
+    assert rq(p16, p16, 1e-6, 4, 256, 32, p16, 4, 0, p16, p16, None, None) == -1         # R > 3
     sk = lib.osc_linear_splitk
     sk.argtypes = [V] * 6 + [I] * 5 + [V, V, V, ctypes.c_size_t, V]
     assert sk(p16, p16, None, p16, p16, None, 4, 128, 256, 32, 0, p16, None, None, 64, None) == -1   # bytes, no buffer

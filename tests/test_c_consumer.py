@@ -30,7 +30,7 @@ int main(void) {
   int hit[2] = {3, 1}, tot[2] = {5, 4};
   double c = 0.0;
   CHECK(osc_select_tier(hit, tot, 2, &c) == OSC_TIER_MID && fabs(c - 0.425) < 1e-12);
-  CHECK(osc_quantize(NULL, 4, 256, 24, NULL, 0, NULL, NULL, NULL, NULL) == OSC_ERR_G);
+  CHECK(osc_quantize(NULL, 4, 256, 24, NULL, 1, 0, NULL, NULL, NULL, NULL) == OSC_ERR_G);
   CHECK(osc_set_tile_n(96) == OSC_ERR_ARG);
   CHECK(strcmp(osc_error_string(OSC_ERR_TABLE), "table entry out of range or more entries than K_L") == 0);
   printf("%s\n", fails ? "C consumer: FAILED" : "C consumer: ok");

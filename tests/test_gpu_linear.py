@@ -175,12 +175,19 @@ def test_all_minus_one_table_is_mxfp4_direct(oracle, osc):
     _run_osc(oracle, osc, c.X, c.W[:512], 32, None)
 
 
-def _moe(oracle, osc, counts, which="gateup", block_sample=False):
+def _moe(oracle, osc, counts, which="gateup", block_sample=False, R=1):
     case = I.moe_case(which, E=len(counts), counts_override=counts) if counts is not None else I.moe_case(which)
     K, N, G = case.K, case.N, 32
     counts, E = case.counts, case.E
     tables = np.stack([oracle.build_table(case.calib[e], G) if case.calib[e].shape[0] else
                        np.full(K // G, -1, np.int8) for e in range(E)])
+    if R > 1:                                  # slot 1: a second channel in a third of the used groups
+        rng = np.random.default_rng(77)
+        second = np.full(tables.shape, -1, np.int8)
+        for e in range(E):
+            for k in np.nonzero(tables[e] >= 0)[0][::3]:
+                second[e, k] = (int(tables[e, k]) + 1 + int(rng.integers(0, G - 1))) % G
+        tables = np.stack([tables, second] + [np.full(tables.shape, -1, np.int8)] * (R - 2), axis=-1)
     kls = np.array([I.pad16(oracle.table_count(tables[e])) for e in range(E)], np.int32)
     K_L = max(16, int(kls.max()))
     off, poff, mbe = osc.osc_grouped_plan(counts)
@@ -335,3 +342,28 @@ def test_few_rows_fp8_fallback(oracle, osc):
     torch.cuda.synchronize()
     assert osc.osc_status() == (0, 0)
     _compare(to_np(Y), to_np(Yf), oracle.fp8_forward(c.X, c.W)["Y"])
+
+
+# ---- several protected channels per group ---------------------------------------------------
+
+@pytest.mark.parametrize("M", [256, 2048])
+def test_multi_table_product(oracle, osc, M):
+    """The dual-path product with a two-slot table (second outliers of the two-outlier
+    workload on the 16-bit path): every row at M = 256, every 128-row block at M = 2048 in the
+    CTA-pair configuration."""
+    c = I.two_outlier_case(M)
+    L = oracle.build_table_multi(c.calib, 32, 2)
+    rows = None if M <= 256 else I.block_rows(M, seed=M)
+    _run_osc(oracle, osc, c.X, c.W, 32, L, rows=rows)
+
+
+def test_multi_table_few_rows(oracle, osc):
+    c = I.two_outlier_case(16)
+    L = oracle.build_table_multi(c.calib, 32, 2)
+    _split_and_plain(oracle, osc, c.X, c.W, 32, L, I.pad16(oracle.table_count(L)))
+
+
+def test_moe_grouped_multi_table(oracle, osc):
+    """Grouped form with two-slot expert tables: the Algorithm 1 entry in slot 0 and, in a
+    third of the groups that have one, a second channel in slot 1."""
+    _moe(oracle, osc, [130, 0, 1, 257, 64, 3, 128, 40], R=2)

@@ -329,3 +329,48 @@ def test_rmsnorm_quantize_edge_rows(oracle, osc):
     L = np.full(K // 32, -1, np.int8)
     L[[0, 7, 15]] = [0, 31, 9]
     _check_rmsnorm_quant(oracle, osc, X, gamma, 1e-6, 32, L, 16)
+
+
+# ---- several protected channels per group ---------------------------------------------------
+
+@pytest.mark.parametrize("G,R", [(32, 2), (32, 3), (16, 2), (64, 3)])
+def test_multi_table_build_and_quantize(oracle, osc, G, R):
+    """Up to R channels per group: the GPU build (R rounds, earlier channels read as zero)
+    equals the oracle's table, and the quantize moves every entry out in (group, slot) order:
+    codes, scales and B bit for bit on every row."""
+    c = I.two_outlier_case(512)
+    Lref = oracle.build_table_multi(c.calib, G, R)
+    Ld = torch.empty((4096 // G, R), dtype=torch.int8, device="cuda")
+    osc.osc_build_table_multi(to_dev(c.calib), G, 5.0, 5, R, Ld)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(Ld), Lref)
+    assert (Lref[:, 1] >= 0).sum() > 10                        # second slots are in use
+    _check_quant(oracle, osc, c.X, G, Lref, I.pad16(oracle.table_count(Lref)))
+
+
+def test_multi_table_hand_made_entries(oracle, osc):
+    """A hand-made 3-slot table with a repeated channel, channels 0 and G-1 and a group whose
+    later slot is set while an earlier one is not: the GPU follows the table order exactly
+    (the repeated channel's second B column is 0). Also W_L of the same table."""
+    rng = np.random.default_rng(41)
+    M, K, G, R = 130, 512, 32, 3
+    X = I.bf16_bits(rng.standard_normal((M, K)) * 4)
+    L = np.full((K // G, R), -1, np.int8)
+    L[0] = [4, 9, 4]
+    L[3] = [0, 31, -1]
+    L[7] = [-1, 12, -1]
+    L[15] = [30, 2, 17]
+    K_L = 16
+    _check_quant(oracle, osc, X, G, L, K_L)
+    W = I.gen_weights(96, K, seed=41)
+    _, _, WL = osc.prepare_weight(to_dev(W), G, to_dev(L), K_L)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(WL), oracle.gather_wl(W, G, L, K_L))
+
+
+@pytest.mark.parametrize("G", [32, 64])
+def test_multi_table_rmsnorm_quantize(oracle, osc, G):
+    c = I.two_outlier_case(256)
+    gamma = _gamma(4096, 7)
+    L = oracle.build_table_multi(oracle.rmsnorm(c.calib[:512], gamma, 1e-6)[0], G, 2)
+    _check_rmsnorm_quant(oracle, osc, c.X, gamma, 1e-6, G, L, I.pad16(oracle.table_count(L)))

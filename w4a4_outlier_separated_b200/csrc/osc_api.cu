@@ -329,16 +329,21 @@ int osc_set_cta_pair(int mode) {
   return g_pair.exchange(mode);
 }
 
-int osc_build_table(const uint16_t* Xcal, int S, int K, int G, float alpha, int min_hits, int8_t* L,
-                    osc_stream_t stream) {
+int osc_build_table_multi(const uint16_t* Xcal, int S, int K, int G, float alpha, int min_hits, int R, int8_t* L,
+                          osc_stream_t stream) {
   if (!valid_g(G)) return OSC_ERR_G;
-  if (!Xcal || !L || S < 0 || K <= 0 || K % G != 0) return OSC_ERR_ARG;
+  if (!Xcal || !L || S < 0 || K <= 0 || K % G != 0 || R < 1 || R > osc::MAX_R) return OSC_ERR_ARG;
   if (!a16(Xcal)) return OSC_ERR_ALIGN;
   DeviceState* ds = nullptr;
   int rc = device_state(&ds);
   if (rc != OSC_OK) return rc;
-  osc::TableParams p{Xcal, S, K, G, alpha, min_hits, L};
+  osc::TableParams p{Xcal, S, K, G, alpha, min_hits, R, L};
   return launch_result(osc::launch_build_table(p, ds->sms, (cudaStream_t)stream));
+}
+
+int osc_build_table(const uint16_t* Xcal, int S, int K, int G, float alpha, int min_hits, int8_t* L,
+                    osc_stream_t stream) {
+  return osc_build_table_multi(Xcal, S, K, G, alpha, min_hits, 1, L, stream);
 }
 
 int osc_density(const uint16_t* X, int S, int K, int G, float alpha, const int8_t* L, int* n_hit, int* n_total,
@@ -396,30 +401,32 @@ int osc_select_tier(const int* n_hit, const int* n_total, int Kg, double* c_bar)
   return tier_of(c);
 }
 
-int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int K_L, uint8_t* QX, uint8_t* SX,
+int osc_quantize(const uint16_t* X, int M, int K, int G, const int8_t* L, int R, int K_L, uint8_t* QX, uint8_t* SX,
                  uint16_t* B, osc_stream_t stream) {
   if (!valid_g(G)) return OSC_ERR_G;
+  if (R < 1 || R > osc::MAX_R) return OSC_ERR_ARG;
   if (M == 0 && K > 0 && K_L >= 0) return OSC_OK;          // nothing to read or write
   if (!X || !QX || !SX || M < 0 || K <= 0 || K_L < 0) return OSC_ERR_ARG;
   if ((long long)(M + 127) * (K / 32) >= (1LL << 31)) return OSC_ERR_ARG;
   if (L == nullptr && K_L != 0) return OSC_ERR_ARG;
   if (L != nullptr && K_L > 0 && !B) return OSC_ERR_ARG;
-  if (K_L > 32767 || (L != nullptr && K / G > 1024)) return OSC_ERR_ARG;
+  if (K_L > 32767 || (L != nullptr && (long long)(K / G) * R > osc::MAX_TAB)) return OSC_ERR_ARG;
   if (!a16(X) || !a16(QX) || !a16(SX) || (B && !a16(B))) return OSC_ERR_ALIGN;
   if (K % 256 != 0 || K_L % 16 != 0) return OSC_ERR_ALIGN;
   DeviceState* ds = nullptr;
   int rc = device_state(&ds);
   if (rc != OSC_OK) return rc;
   if (M == 0) return OSC_OK;
-  osc::QuantParams p{X, M, K, G, K / G, L, K_L, QX, SX, B, ds->status};
+  osc::QuantParams p{X, M, K, G, K / G, L, R, K_L, QX, SX, B, ds->status};
   CUtensorMap tm;
   if ((rc = make_block_map(&tm, X, M, K))) return rc;
   return launch_result(osc::launch_quantize(tm, p, false, ds->sms, (cudaStream_t)stream));
 }
 
 int osc_rmsnorm_quantize(const uint16_t* X, const uint16_t* gamma, float eps, int M, int K, int G, const int8_t* L,
-                         int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B, osc_stream_t stream) {
+                         int R, int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B, osc_stream_t stream) {
   if (!valid_g(G)) return OSC_ERR_G;
+  if (R < 1 || R > osc::MAX_R) return OSC_ERR_ARG;
   if (!(eps >= 0.0f) || !std::isfinite(eps)) return OSC_ERR_ARG;
   if (M == 0 && K > 0 && K_L >= 0) return OSC_OK;          // nothing to read or write
   if (!X || !gamma || !QX || !SX || M < 0 || K <= 0 || K_L < 0) return OSC_ERR_ARG;
@@ -433,15 +440,16 @@ int osc_rmsnorm_quantize(const uint16_t* X, const uint16_t* gamma, float eps, in
   DeviceState* ds = nullptr;
   int rc = device_state(&ds);
   if (rc != OSC_OK) return rc;
-  osc::NormQuantParams p{X, gamma, eps, M, K, G, K / G, L, K_L, QX, SX, B, ds->status};
+  osc::NormQuantParams p{X, gamma, eps, M, K, G, K / G, L, R, K_L, QX, SX, B, ds->status};
   CUtensorMap tm;
   if ((rc = make_row_map(&tm, X, M, K))) return rc;
   return launch_result(osc::launch_rmsnorm_quantize(tm, p, ds->sms, (cudaStream_t)stream));
 }
 
-int osc_prepare_weight(const uint16_t* W, int N, int K, int G, const int8_t* L, int K_L, uint8_t* QW, uint8_t* SW,
-                       uint16_t* WL, osc_stream_t stream) {
+int osc_prepare_weight(const uint16_t* W, int N, int K, int G, const int8_t* L, int R, int K_L, uint8_t* QW,
+                       uint8_t* SW, uint16_t* WL, osc_stream_t stream) {
   if (!valid_g(G)) return OSC_ERR_G;
+  if (R < 1 || R > osc::MAX_R) return OSC_ERR_ARG;
   if (!W || !QW || !SW || N < 0 || K <= 0 || K_L < 0) return OSC_ERR_ARG;
   if ((long long)(N + 127) * (K / 32) >= (1LL << 31)) return OSC_ERR_ARG;
   if (K_L > 0 && (!L || !WL)) return OSC_ERR_ARG;
@@ -451,12 +459,12 @@ int osc_prepare_weight(const uint16_t* W, int N, int K, int G, const int8_t* L, 
   int rc = device_state(&ds);
   if (rc != OSC_OK) return rc;
   if (N == 0) return OSC_OK;
-  osc::QuantParams p{W, N, K, G, K / G, nullptr, 0, QW, SW, nullptr, ds->status};
+  osc::QuantParams p{W, N, K, G, K / G, nullptr, 1, 0, QW, SW, nullptr, ds->status};
   CUtensorMap tm;
   if ((rc = make_block_map(&tm, W, N, K))) return rc;
   cudaError_t e = osc::launch_quantize(tm, p, false, ds->sms, (cudaStream_t)stream);
   if (e != cudaSuccess) return fail_cuda(e);
-  return launch_result(osc::launch_gather_wl(W, N, K, G, L, K_L, WL, ds->status, ds->sms, (cudaStream_t)stream));
+  return launch_result(osc::launch_gather_wl(W, N, K, G, L, R, K_L, WL, ds->status, ds->sms, (cudaStream_t)stream));
 }
 
 int osc_linear(const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const uint8_t* QW, const uint8_t* SW,
@@ -511,7 +519,7 @@ int osc_quantize_fp8(const uint16_t* X, int M, int K, uint8_t* QX8, uint8_t* SX,
   int rc = device_state(&ds);
   if (rc != OSC_OK) return rc;
   if (M == 0) return OSC_OK;
-  osc::QuantParams p{X, M, K, 32, K / 32, nullptr, 0, QX8, SX, nullptr, ds->status};
+  osc::QuantParams p{X, M, K, 32, K / 32, nullptr, 1, 0, QX8, SX, nullptr, ds->status};
   CUtensorMap tm;
   if ((rc = make_block_map(&tm, X, M, K))) return rc;
   return launch_result(osc::launch_quantize(tm, p, true, ds->sms, (cudaStream_t)stream));
@@ -551,9 +559,10 @@ int osc_grouped_plan(const int* counts, int E, int* off, int* poff, int* mblock_
 }
 
 int osc_quantize_grouped(const uint16_t* X, int T, int E, const int* off, const int* poff, const int* mblock_expert,
-                         int Mp, int K, int G, const int8_t* L, int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B,
+                         int Mp, int K, int G, const int8_t* L, int R, int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B,
                          osc_stream_t stream) {
   if (!valid_g(G)) return OSC_ERR_G;
+  if (R < 1 || R > osc::MAX_R) return OSC_ERR_ARG;
   if (!X || !off || !poff || !mblock_expert || !L || !QX || !SX || E <= 0 || Mp < 0 || K <= 0 || K_L < 0)
     return OSC_ERR_ARG;
   if (T < 0 || T > Mp) return OSC_ERR_ARG;
@@ -562,13 +571,13 @@ int osc_quantize_grouped(const uint16_t* X, int T, int E, const int* off, const 
   if ((long long)(Mp + 127) * (K / 32) >= (1LL << 31)) return OSC_ERR_ARG;
   if (!a16(X) || !a16(QX) || !a16(SX) || (B && !a16(B))) return OSC_ERR_ALIGN;
   if (K % 256 != 0 || K_L % 16 != 0 || Mp % 128 != 0) return OSC_ERR_ALIGN;
-  if (osc::grouped_quant_smem(E, K / G) > (size_t)osc::GROUPED_QUANT_SMEM_MAX) return OSC_ERR_ARG;   // E x K/G table entries
+  if (osc::grouped_quant_smem(E, K / G, R) > (size_t)osc::GROUPED_QUANT_SMEM_MAX) return OSC_ERR_ARG;   // E x K/G x R entries
   DeviceState* ds = nullptr;
   int rc = device_state(&ds);
   if (rc != OSC_OK) return rc;
   if (Mp == 0) return OSC_OK;
-  osc::GroupedQuantParams p{X, off, poff, mblock_expert, E, Mp, K, G, K / G, L, K_L, QX, SX, B, ds->status};
-  if (T > 0 && osc::grouped_tma_smem(E, K / G) <= (size_t)osc::GROUPED_TMA_SMEM_MAX) {
+  osc::GroupedQuantParams p{X, off, poff, mblock_expert, E, Mp, K, G, K / G, L, R, K_L, QX, SX, B, ds->status};
+  if (T > 0 && osc::grouped_tma_smem(E, K / G, R) <= (size_t)osc::GROUPED_TMA_SMEM_MAX) {
     CUtensorMap tm;
     if ((rc = make_block_map(&tm, X, T, K))) return rc;
     return launch_result(osc::launch_quantize_grouped_tma(tm, p, T, ds->sms, (cudaStream_t)stream));

@@ -26,10 +26,17 @@ struct PerDeviceOnce {
   }
 };
 
+// Protected channels per group: a table holds K/G x R entries (R <= MAX_R), slot r of group k
+// at L[k * R + r], -1 = none.
+constexpr int MAX_R = 3;
+// Largest table (K/G x R entries) the dense quantize stages in shared memory.
+constexpr int MAX_TAB = 4096;
+
 struct QuantParams {
   const uint16_t* X;   // M x K bf16
   int M, K, G, Kg;
-  const int8_t* L;     // Kg entries (device) or nullptr for no table
+  const int8_t* L;     // Kg x R entries (device) or nullptr for no table
+  int R;
   int K_L;
   uint8_t* Q;          // packed codes
   uint8_t* S;          // scales in the MMA layout
@@ -50,7 +57,8 @@ struct NormQuantParams {
   const uint16_t* gamma;   // K bf16
   float eps;
   int M, K, G, Kg;
-  const int8_t* L;         // Kg entries (device) or nullptr
+  const int8_t* L;         // Kg x R entries (device) or nullptr
+  int R;
   int K_L;
   uint8_t* Q;
   uint8_t* S;
@@ -68,7 +76,8 @@ struct GroupedQuantParams {
   const int* poff;            // E+1 (device)
   const int* mblock_expert;   // Mp/128 (device)
   int E, Mp, K, G, Kg;
-  const int8_t* L;            // E x Kg (device)
+  const int8_t* L;            // E x Kg x R (device)
+  int R;
   int K_L;
   uint8_t* Q;
   uint8_t* S;
@@ -79,12 +88,12 @@ cudaError_t launch_quantize_grouped(const GroupedQuantParams& p, int num_sms, cu
 // TMA form over the T = off[E] routed rows (tmX: the dense kernel's block view of those rows)
 cudaError_t launch_quantize_grouped_tma(const CUtensorMap& tmX, const GroupedQuantParams& p, int T, int num_sms,
                                         cudaStream_t s);
-size_t grouped_tma_smem(int E, int Kg);
+size_t grouped_tma_smem(int E, int Kg, int R);
 constexpr int GROUPED_TMA_SMEM_MAX = 200 * 1024;
 // shared memory the grouped quantize needs to stage every expert's table, and its limit
-size_t grouped_quant_smem(int E, int Kg);
+size_t grouped_quant_smem(int E, int Kg, int R);
 constexpr int GROUPED_QUANT_SMEM_MAX = 200 * 1024;
-cudaError_t launch_gather_wl(const uint16_t* W, int N, int K, int G, const int8_t* L, int K_L, uint16_t* WL,
+cudaError_t launch_gather_wl(const uint16_t* W, int N, int K, int G, const int8_t* L, int R, int K_L, uint16_t* WL,
                              int* status, int num_sms, cudaStream_t s);
 
 // GEMM operand kinds
@@ -135,7 +144,8 @@ struct TableParams {
   int S, K, G;
   float alpha;
   int min_hits;
-  int8_t* L;
+  int R;               // rounds: protected channels per group
+  int8_t* L;           // K/G x R
 };
 cudaError_t launch_build_table(const TableParams& p, int num_sms, cudaStream_t s);
 

@@ -129,58 +129,90 @@ __device__ __forceinline__ uint2 codes16(const uint32_t (&w)[16], uint32_t f2) {
   return r;
 }
 
-// Table facts of one 32-channel block for a thread: up to two table channels (two only for
-// G = 16, where the block holds two groups), each with its slot in the block and its B column.
+// Table facts of one 32-channel block for a thread: the table entries whose channels fall in
+// the block, in table order (group, slot): for G = 32 the R slots of the block's group, for
+// G = 16 the R slots of each of its two groups, for G = 64 the slots of its group that lie in
+// this half of it. Entry e: the channel within the block (lw, -1 = none) and its B column.
+constexpr int BT_SLOTS = 2 * MAX_R;
 struct BlockTable {
-  int lw0, pos0;   // lw < 0: none
-  int lw1, pos1;
+  int lw[BT_SLOTS];
+  int pos[BT_SLOTS];
 };
 
-template <int G>
-__device__ __forceinline__ BlockTable block_table(int blk, const int8_t* Ls, const int16_t* Ps) {
-  BlockTable t{-1, 0, -1, 0};
-  if constexpr (G == 32) {
-    const int l = Ls[blk];
-    if (l >= 0) { t.lw0 = l; t.pos0 = Ps[blk]; }
-  } else if constexpr (G == 64) {
-    const int g = blk >> 1, l = Ls[g];
-    if (l >= 0 && (l >> 5) == (blk & 1)) { t.lw0 = l & 31; t.pos0 = Ps[g]; }
-  } else {
-    const int l0 = Ls[2 * blk], l1 = Ls[2 * blk + 1];
-    if (l0 >= 0) { t.lw0 = l0; t.pos0 = Ps[2 * blk]; }
-    if (l1 >= 0) { t.lw1 = 16 + l1; t.pos1 = Ps[2 * blk + 1]; }
-  }
+__device__ __forceinline__ BlockTable no_table() {
+  BlockTable t;
+#pragma unroll
+  for (int e = 0; e < BT_SLOTS; ++e) { t.lw[e] = -1; t.pos[e] = 0; }
   return t;
 }
 
-// Table entry and B column of one group packed in one word: (column << 8) | (entry & 0xFF),
-// entry -1 (0xFF) meaning none.
+// The group holding slot h (h = 0, 1; two only for G = 16) of block blk.
 template <int G>
-__device__ __forceinline__ BlockTable block_table_packed(int blk, const int* tab) {
-  BlockTable t{-1, 0, -1, 0};
-  if constexpr (G == 32) {
-    const int v = tab[blk], l = (int)(int8_t)(v & 0xFF);
-    if (l >= 0) { t.lw0 = l; t.pos0 = v >> 8; }
-  } else if constexpr (G == 64) {
-    const int v = tab[blk >> 1], l = (int)(int8_t)(v & 0xFF);
-    if (l >= 0 && (l >> 5) == (blk & 1)) { t.lw0 = l & 31; t.pos0 = v >> 8; }
-  } else {
-    const int2 v = *reinterpret_cast<const int2*>(tab + 2 * blk);
-    const int l0 = (int)(int8_t)(v.x & 0xFF), l1 = (int)(int8_t)(v.y & 0xFF);
-    if (l0 >= 0) { t.lw0 = l0; t.pos0 = v.x >> 8; }
-    if (l1 >= 0) { t.lw1 = 16 + l1; t.pos1 = v.y >> 8; }
-  }
+__device__ __forceinline__ int block_group(int blk, int h) {
+  return G == 16 ? 2 * blk + h : (G == 64 ? blk >> 1 : blk);
+}
+
+// From separate arrays: entry channel (int8) and B column (int16), R slots per group.
+template <int G>
+__device__ __forceinline__ BlockTable block_table(int blk, const int8_t* Ls, const int16_t* Ps, int R) {
+  BlockTable t = no_table();
+#pragma unroll
+  for (int h = 0; h < (G == 16 ? 2 : 1); ++h)
+#pragma unroll
+    for (int m = 0; m < MAX_R; ++m) {
+      if (m >= R) continue;
+      const int i = block_group<G>(blk, h) * R + m;
+      const int l = Ls[i];
+      if (l < 0 || (G == 64 && (l >> 5) != (blk & 1))) continue;
+      t.lw[h * MAX_R + m] = G == 16 ? 16 * h + l : (l & 31);
+      t.pos[h * MAX_R + m] = Ps[i];
+    }
   return t;
 }
 
-// Stage one table (Kg entries) in shared memory, packed with each entry's B column; returns
-// the number of entries (at most K_L). Entries >= G or beyond K_L columns are reported and
-// dropped.
+// From packed words (column << 8) | (entry & 0xFF), entry -1 (0xFF) meaning none.
+template <int G>
+__device__ __forceinline__ BlockTable block_table_packed(int blk, const int* tab, int R) {
+  BlockTable t = no_table();
+#pragma unroll
+  for (int h = 0; h < (G == 16 ? 2 : 1); ++h)
+#pragma unroll
+    for (int m = 0; m < MAX_R; ++m) {
+      if (m >= R) continue;
+      const int v = tab[block_group<G>(blk, h) * R + m], l = (int)(int8_t)(v & 0xFF);
+      if (l < 0 || (G == 64 && (l >> 5) != (blk & 1))) continue;
+      t.lw[h * MAX_R + m] = G == 16 ? 16 * h + l : (l & 31);
+      t.pos[h * MAX_R + m] = v >> 8;
+    }
+  return t;
+}
+
+// Move the block's table channels out of its 64-byte item in shared memory (64-byte swizzle:
+// the 2 bytes of channel lw sit in 16-byte chunk (lw / 8) ^ swz at byte (lw % 8) * 2), in table
+// order: each value to its B column of the row (Brow, when live), +0 left in its slot. A
+// channel named twice yields its value once and then the 0 the first move left.
+template <int G>
+__device__ __forceinline__ void extract_from_item(uint8_t* item, int swz, const BlockTable& t, bool loaded, bool live,
+                                                  uint16_t* __restrict__ Brow) {
+#pragma unroll
+  for (int e = 0; e < (G == 16 ? 2 : 1) * MAX_R; ++e) {
+    const int lw = t.lw[e];
+    if (lw < 0) continue;
+    uint16_t* pv = reinterpret_cast<uint16_t*>(item + (((lw >> 3) ^ swz) * 16) + (lw & 7) * 2);
+    const uint16_t v = loaded ? *pv : (uint16_t)0;
+    if (loaded) *pv = 0;
+    if (live) Brow[t.pos[e]] = v;
+  }
+}
+
+// Stage one table (n = K/G x R entries, in (group, slot) order) in shared memory, packed with
+// each entry's B column; returns the number of entries (at most K_L). Entries >= G or beyond
+// K_L columns are reported and dropped.
 template <int G, int NTHREADS = 256>
-__device__ int stage_table(const int8_t* __restrict__ L, int Kg, int K_L, int* tab, int* s_warp, int* status) {
+__device__ int stage_table(const int8_t* __restrict__ L, int n, int K_L, int* tab, int* s_warp, int* status) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int per = (Kg + NTHREADS - 1) / NTHREADS;
-  const int i0 = threadIdx.x * per, i1 = min(Kg, i0 + per);
+  const int per = (n + NTHREADS - 1) / NTHREADS;
+  const int i0 = threadIdx.x * per, i1 = min(n, i0 + per);
   int local = 0;
   for (int i = i0; i < i1; ++i) {
     int v = L[i];
@@ -221,13 +253,11 @@ __device__ __forceinline__ void quant_block(uint32_t (&w)[16], int row, int blk,
   const int lane = threadIdx.x & 31;
   live = live && valid;
   if constexpr (TABLE) {
-    if (t.lw0 >= 0) {
-      const uint16_t v = take_channel(w, t.lw0);
-      if (live) B[(size_t)row * K_L + t.pos0] = v;
-    }
-    if (G == 16 && t.lw1 >= 0) {
-      const uint16_t v = take_channel(w, t.lw1);
-      if (live) B[(size_t)row * K_L + t.pos1] = v;
+#pragma unroll
+    for (int e = 0; e < (G == 16 ? 2 : 1) * MAX_R; ++e) {
+      if (t.lw[e] < 0) continue;
+      const uint16_t v = take_channel(w, t.lw[e]);
+      if (live) B[(size_t)row * K_L + t.pos[e]] = v;
     }
     if (live && blk == 0)
       for (int i = count; i < K_L; ++i) B[(size_t)row * K_L + i] = 0;
@@ -285,7 +315,6 @@ __device__ __forceinline__ void load_block(const uint16_t* __restrict__ X, size_
   }
 }
 
-constexpr int MAX_KG = 1024;
 
 // Dense form, TMA-fed. X is viewed as a 2-D tensor of 32-channel blocks (items): rows of 64
 // bytes, one per (row, block) in row-major order, so a warp step's 64 items are one
@@ -307,11 +336,11 @@ __device__ __forceinline__ void load_block_smem(const uint8_t* slot, int r, uint
 
 template <int G, bool FP8, bool TABLE>
 __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant__ CUtensorMap tmX, QuantParams p) {
-  extern __shared__ uint8_t q_dyn[];                          // QWARPS x 2 boxes of 4 KB, 1 KB aligned
+  extern __shared__ uint8_t q_dyn[];      // QWARPS x 2 boxes of 4 KB (1 KB aligned), then the table
   uint8_t* boxes = q_dyn + ((1024u - (smem_u32(q_dyn) & 1023u)) & 1023u);
   auto box_at = [&](int wp, int sl) { return boxes + (wp * 2 + sl) * (QSTEP * 64); };
+  int* s_tab = reinterpret_cast<int*>(boxes + QWARPS * 2 * QSTEP * 64);   // K/G x R packed entries
   __shared__ __align__(8) uint64_t s_bar[QWARPS][2];
-  __shared__ __align__(8) int s_tab[TABLE ? MAX_KG : 2];
   __shared__ int s_warp[8];
   __shared__ int s_abort;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -332,6 +361,14 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
   if (lane == 0) { mbar_init(smem_u32(&s_bar[warp][0]), 1); mbar_init(smem_u32(&s_bar[warp][1]), 1); }
   fence_barrier_init();
   __syncwarp();
+  // Every box this warp will load goes to L2 before the wait for the previous kernel: a
+  // prefetch changes no value a later load returns (L2 is where the previous kernel's writes
+  // land), so it is safe even when X is that kernel's output, and when X is already resident it
+  // costs nothing. If this CTA starts while the previous kernel's last wave still runs, X
+  // streams in meanwhile.
+  if (lane == 0)
+    for (uint32_t st = step; st < cta_end; st += wstride)
+      if (st * QSTEP < real_items) tma_prefetch_l2_2d(&tmX, 0, (int)(st * QSTEP));
   // X, L and the outputs are free of the previous kernel. No early trigger for the next one:
   // quantize CTAs are small enough to share SMs, so an early-launched next grid would hold SM
   // slots while it waits; the next kernel is released when this grid completes.
@@ -348,7 +385,7 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
   if (step < cta_end) issue(step, 0);
   if (step + wstride < cta_end) issue(step + wstride, 1);
   int count = 0;
-  if constexpr (TABLE) count = stage_table<G>(p.L, p.Kg, p.K_L, s_tab, s_warp, p.status);
+  if constexpr (TABLE) count = stage_table<G>(p.L, p.Kg * p.R, p.K_L, s_tab, s_warp, p.status);
   else __syncthreads();
   uint32_t phbits = 0;                                        // bit s: parity of slot s's next phase
   int slot = 0;
@@ -385,23 +422,10 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
       const bool live = row < p.M;
       uint8_t* item = box + r * 64;
       const int swz = (r >> 1) & 3;
-      BlockTable t{-1, 0, -1, 0};
       if constexpr (TABLE) {
-        t = block_table_packed<G>(blk, s_tab);
-        // move the table channel(s) out of the box: its 2 bytes sit in 16-byte chunk
-        // (lw / 8) ^ swz at byte (lw % 8) * 2
-        if (t.lw0 >= 0) {
-          uint16_t* pv = reinterpret_cast<uint16_t*>(item + (((t.lw0 >> 3) ^ swz) * 16) + (t.lw0 & 7) * 2);
-          const uint16_t v = loaded ? *pv : (uint16_t)0;
-          if (loaded) *pv = 0;
-          if (live) p.B[(size_t)row * p.K_L + t.pos0] = v;
-        }
-        if (G == 16 && t.lw1 >= 0) {
-          uint16_t* pv = reinterpret_cast<uint16_t*>(item + (((t.lw1 >> 3) ^ swz) * 16) + (t.lw1 & 7) * 2);
-          const uint16_t v = loaded ? *pv : (uint16_t)0;
-          if (loaded) *pv = 0;
-          if (live) p.B[(size_t)row * p.K_L + t.pos1] = v;
-        }
+        // move the table channels out of the box (in table order), then clear B's pad columns
+        const BlockTable t = block_table_packed<G>(blk, s_tab, p.R);
+        extract_from_item<G>(item, swz, t, loaded, live, p.B + (size_t)row * p.K_L);
         if (live && blk == 0)
           for (int i = count; i < p.K_L; ++i) p.B[(size_t)row * p.K_L + i] = 0;
       }
@@ -411,8 +435,7 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
 #pragma unroll
         for (int j = 0; j < 16; ++j) w[j] = 0u;
       }
-      const BlockTable none{-1, 0, -1, 0};
-      quant_block<G, FP8, false>(w, row, blk, live, none, count, p.K, p.K_L, p.B, p.Q, p.S);
+      quant_block<G, FP8, false>(w, row, blk, live, no_table(), count, p.K, p.K_L, p.B, p.Q, p.S);
     }
     __syncwarp();                                             // every lane is done with this slot
     if (step + 2 * wstride < cta_end) { fence_proxy_async_smem(); issue(step + 2 * wstride, slot); }
@@ -451,7 +474,7 @@ __global__ void __launch_bounds__(NQ_THREADS, 1) rmsnorm_quantize_kernel(const _
   uint8_t* gam = base;
   auto row_buf = [&](int wp, int sl) { return base + slot_bytes * (1u + (uint32_t)(wp * nslots + sl)); };
   __shared__ __align__(8) uint64_t s_bar[NQ_WARPS][2];
-  __shared__ __align__(8) int s_tab[TABLE ? MAX_KG : 2];
+  __shared__ __align__(8) int s_tab[TABLE ? NQ_MAX_K / 16 * MAX_R : 2];
   __shared__ int s_warp[NQ_WARPS];
   __shared__ int s_abort;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -481,7 +504,7 @@ __global__ void __launch_bounds__(NQ_THREADS, 1) rmsnorm_quantize_kernel(const _
     *reinterpret_cast<uint4*>(gam + b * 64 + ((c ^ ((b >> 1) & 3)) * 16)) = v;
   }
   int count = 0;
-  if constexpr (TABLE) count = stage_table<G, NQ_THREADS>(p.L, p.Kg, p.K_L, s_tab, s_warp, p.status);
+  if constexpr (TABLE) count = stage_table<G, NQ_THREADS>(p.L, p.Kg * p.R, p.K_L, s_tab, s_warp, p.status);
   else __syncthreads();
   const int iters = (nb + 31) / 32;                          // blocks per lane (<= NQ_PARTS)
   uint32_t phbits = 0;
@@ -558,8 +581,8 @@ __global__ void __launch_bounds__(NQ_THREADS, 1) rmsnorm_quantize_kernel(const _
 #pragma unroll
         for (int j = 0; j < 16; ++j) w[j] = 0u;
       }
-      BlockTable t{-1, 0, -1, 0};
-      if constexpr (TABLE) t = block_table_packed<G>(valid ? blk : 0, s_tab);
+      BlockTable t = no_table();
+      if constexpr (TABLE) t = block_table_packed<G>(valid ? blk : 0, s_tab, p.R);
       quant_block<G, false, TABLE>(w, (int)row, blk, loaded, t, count, p.K, p.K_L, p.B, p.Q, p.S, valid);
     }
     __syncwarp();                                             // every lane is done with this buffer
@@ -597,7 +620,7 @@ static cudaError_t launch_nq(const CUtensorMap& tmX, const NormQuantParams& p, i
 cudaError_t launch_rmsnorm_quantize(const CUtensorMap& tmX, const NormQuantParams& p, int num_sms, cudaStream_t s) {
   if (p.K % 256 != 0 || p.K > NQ_MAX_K) return cudaErrorInvalidValue;
   const bool table = p.L != nullptr;
-  if (table && p.Kg > MAX_KG) return cudaErrorInvalidValue;
+  if (table && p.Kg * p.R > NQ_MAX_K / 16 * MAX_R) return cudaErrorInvalidValue;
   const size_t smem = rmsnorm_quant_smem(p.K);
   const long long rows = (long long)(p.M + 127) / 128 * 128;
   // one CTA of 16 warps per SM (its registers, up to 128 a thread, fill the SM's file)
@@ -627,8 +650,8 @@ __device__ __forceinline__ int last_le(const int* a, int n, int v) {   // larges
   return lo;
 }
 
-size_t grouped_tma_smem(int E, int Kg) {
-  return (size_t)QWARPS * 2 * QSTEP * 64 + 1024 + 4 * ((size_t)E * Kg + 2 * ((size_t)E + 1) + (size_t)E);
+size_t grouped_tma_smem(int E, int Kg, int R) {
+  return (size_t)QWARPS * 2 * QSTEP * 64 + 1024 + 4 * ((size_t)E * Kg * R + 2 * ((size_t)E + 1) + (size_t)E);
 }
 
 template <int G>
@@ -637,8 +660,9 @@ __global__ void __launch_bounds__(256) quantize_grouped_tma_kernel(const __grid_
   extern __shared__ uint8_t q_dyn[];
   uint8_t* boxes = q_dyn + ((1024u - (smem_u32(q_dyn) & 1023u)) & 1023u);
   auto box_at = [&](int wp, int sl) { return boxes + (wp * 2 + sl) * (QSTEP * 64); };
+  const int nt = p.Kg * p.R;                                 // table entries per expert
   int* s_tab = reinterpret_cast<int*>(boxes + QWARPS * 2 * QSTEP * 64);
-  int* s_off = s_tab + p.E * p.Kg;
+  int* s_off = s_tab + p.E * nt;
   int* s_poff = s_off + (p.E + 1);
   int* s_cnt = s_poff + (p.E + 1);
   __shared__ __align__(8) uint64_t s_bar[QWARPS][2];
@@ -669,10 +693,10 @@ __global__ void __launch_bounds__(256) quantize_grouped_tma_kernel(const __grid_
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) { s_off[i] = p.off[i]; s_poff[i] = p.poff[i]; }
   for (int e = threadIdx.x; e < p.E; e += blockDim.x) {     // one thread per expert table
     int run = 0;
-    for (int g = 0; g < p.Kg; ++g) {
-      int v = p.L[(size_t)e * p.Kg + g];
+    for (int g = 0; g < nt; ++g) {
+      int v = p.L[(size_t)e * nt + g];
       if (v >= G || (v >= 0 && run >= p.K_L)) { record_status(p.status, DEV_BAD_TABLE); v = -1; }
-      s_tab[e * p.Kg + g] = v < 0 ? 0xFF : ((run++ << 8) | v);
+      s_tab[e * nt + g] = v < 0 ? 0xFF : ((run++ << 8) | v);
     }
     s_cnt[e] = run;
   }
@@ -712,23 +736,13 @@ __global__ void __launch_bounds__(256) quantize_grouped_tma_kernel(const __grid_
       const int row = live ? dest0 + t : 0;
       uint8_t* item = box + r * 64;
       const int swz = (r >> 1) & 3;
-      const BlockTable tb = live ? block_table_packed<G>(blk, s_tab + e * p.Kg) : BlockTable{-1, 0, -1, 0};
-      if (tb.lw0 >= 0) {
-        uint16_t* pv = reinterpret_cast<uint16_t*>(item + (((tb.lw0 >> 3) ^ swz) * 16) + (tb.lw0 & 7) * 2);
-        p.B[(size_t)row * p.K_L + tb.pos0] = *pv;
-        *pv = 0;
-      }
-      if (G == 16 && tb.lw1 >= 0) {
-        uint16_t* pv = reinterpret_cast<uint16_t*>(item + (((tb.lw1 >> 3) ^ swz) * 16) + (tb.lw1 & 7) * 2);
-        p.B[(size_t)row * p.K_L + tb.pos1] = *pv;
-        *pv = 0;
-      }
+      const BlockTable tb = live ? block_table_packed<G>(blk, s_tab + e * nt, p.R) : no_table();
+      extract_from_item<G>(item, swz, tb, true, live, p.B + (size_t)row * p.K_L);
       if (live && blk == 0)
         for (int i = s_cnt[e]; i < p.K_L; ++i) p.B[(size_t)row * p.K_L + i] = 0;
       uint32_t w[16];
       load_block_smem(box, r, w);
-      const BlockTable none{-1, 0, -1, 0};
-      quant_block<G, false, false>(w, row, blk, live, none, 0, p.K, p.K_L, p.B, p.Q, p.S, live);
+      quant_block<G, false, false>(w, row, blk, live, no_table(), 0, p.K, p.K_L, p.B, p.Q, p.S, live);
     }
     __syncwarp();
     if (step + 2 * wstride < cta_end) { fence_proxy_async_smem(); issue(step + 2 * wstride, slot); }
@@ -777,7 +791,7 @@ static cudaError_t launch_grouped_tma_g(const CUtensorMap& tmX, const GroupedQua
 cudaError_t launch_quantize_grouped_tma(const CUtensorMap& tmX, const GroupedQuantParams& p, int T, int num_sms,
                                         cudaStream_t s) {
   if (p.Mp == 0) return cudaSuccess;
-  const size_t smem = grouped_tma_smem(p.E, p.Kg);
+  const size_t smem = grouped_tma_smem(p.E, p.Kg, p.R);
   if (smem > (size_t)GROUPED_TMA_SMEM_MAX) return cudaErrorInvalidValue;
   const int per_sm = std::max(1, std::min(QMAXK, (int)(227 * 1024 / (smem + 1024))));
   const long long steps = std::max<long long>(1, ((long long)T * (p.K / 32) + QSTEP - 1) / QSTEP);
@@ -799,21 +813,22 @@ cudaError_t launch_quantize_grouped_tma(const CUtensorMap& tmX, const GroupedQua
 // Grouped (MoE) form, one lane per block with plain loads: the fallback for tables too large
 // to stage beside the TMA boxes. Over the padded row space: a row's expert comes from its 128-row block;
 // rows past the expert's token count are padding and come out as zeros. The CTA stages every
-// expert's table (E x Kg entries) with per-expert B columns.
+// expert's table (E x K/G x R entries) with per-expert B columns.
 template <int G>
 __global__ void __launch_bounds__(256) quantize_grouped_kernel(GroupedQuantParams p) {
   extern __shared__ __align__(16) unsigned char gsm[];
-  const int n = p.E * p.Kg;
+  const int nt = p.Kg * p.R;                                 // table entries per expert
+  const int n = p.E * nt;
   int8_t* s_l = reinterpret_cast<int8_t*>(gsm);
   int16_t* s_pos = reinterpret_cast<int16_t*>(gsm + ((n + 15) & ~15));
   int* s_cnt = reinterpret_cast<int*>(gsm + ((n + 15) & ~15) + ((2 * n + 15) & ~15));
   for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
     int run = 0;
-    for (int g = 0; g < p.Kg; ++g) {
-      int v = p.L[(size_t)e * p.Kg + g];
+    for (int g = 0; g < nt; ++g) {
+      int v = p.L[(size_t)e * nt + g];
       if (v >= G || (v >= 0 && run >= p.K_L)) { record_status(p.status, DEV_BAD_TABLE); v = -1; }
-      s_l[e * p.Kg + g] = (int8_t)v;
-      if (v >= 0) s_pos[e * p.Kg + g] = (int16_t)run++;
+      s_l[e * nt + g] = (int8_t)v;
+      if (v >= 0) s_pos[e * nt + g] = (int16_t)run++;
     }
     s_cnt[e] = run;
   }
@@ -829,24 +844,28 @@ __global__ void __launch_bounds__(256) quantize_grouped_kernel(GroupedQuantParam
     const bool valid = local < __ldg(p.off + e + 1) - src0;
     uint32_t w[16];
     load_block(p.X, (size_t)(src0 + local) * p.K + (size_t)blk * 32, valid, w);
-    const BlockTable t = block_table<G>(blk, s_l + e * p.Kg, s_pos + e * p.Kg);
+    const BlockTable t = block_table<G>(blk, s_l + e * nt, s_pos + e * nt, p.R);
     quant_block<G, false, true>(w, row, blk, true, t, s_cnt[e], p.K, p.K_L, p.B, p.Q, p.S);
   }
 }
 
 constexpr int QSMEM = QWARPS * 2 * QSTEP * 64 + 1024;
 
+// Dynamic shared memory of the dense kernel: the boxes, then the table (n entries).
+size_t quant_smem(int n_table) { return (size_t)QSMEM + (((size_t)n_table * 4 + 15) & ~(size_t)15); }
+
 template <int G, bool FP8, bool TABLE>
-static cudaError_t launch_quant(const CUtensorMap& tmX, const QuantParams& p, int grid, cudaStream_t s) {
+static cudaError_t launch_quant(const CUtensorMap& tmX, const QuantParams& p, int grid, size_t smem, cudaStream_t s) {
   static PerDeviceOnce smem_attr;
   const cudaError_t ae = smem_attr.run([] {
-    return cudaFuncSetAttribute(quantize_tma_kernel<G, FP8, TABLE>, cudaFuncAttributeMaxDynamicSharedMemorySize, QSMEM);
+    return cudaFuncSetAttribute(quantize_tma_kernel<G, FP8, TABLE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)quant_smem(MAX_TAB));
   });
   if (ae != cudaSuccess) return ae;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(256, 1, 1);
-  cfg.dynamicSmemBytes = QSMEM;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -860,33 +879,38 @@ cudaError_t launch_quantize(const CUtensorMap& tmX, const QuantParams& p, bool f
   // 1..3 CTAs per SM: the fewest steps for the busiest warp (the critical path; a CTA's run of
   // ceil(steps / CTAs) steps is shared by its QWARPS warps), and on a tie the most resident warps
   // (more warps per scheduler hide more of each warp's latency)
+  const bool table = p.L != nullptr;
+  const int n_table = table ? p.Kg * p.R : 0;
+  if (n_table > MAX_TAB) return cudaErrorInvalidValue;
+  const size_t smem = quant_smem(n_table);
+  // resident CTAs per SM: at most QMAXK, fewer when a large table grows the shared memory
+  // (each CTA also holds ~1 KB of static and system shared memory)
+  const int fit = (int)std::max<size_t>(1, (size_t)232448 / (smem + 2048));
   const long long steps = (long long)((p.M + 127) / 128 * 128) * (p.K / 32) / QSTEP;
   int grid = 1;
   long long best = -1;
-  for (int k = 1; k <= QMAXK; ++k) {
+  for (int k = 1; k <= std::min(QMAXK, fit); ++k) {
     const long long ctas = std::max<long long>(1, std::min<long long>((steps + QWARPS - 1) / QWARPS, (long long)num_sms * k));
     const long long busiest = ((steps + ctas - 1) / ctas + QWARPS - 1) / QWARPS;
     if (best < 0 || busiest <= best) { best = busiest; grid = (int)ctas; }
   }
-  const bool table = p.L != nullptr;
-  if (table && p.Kg > MAX_KG) return cudaErrorInvalidValue;
-  if (fp8) return launch_quant<32, true, false>(tmX, p, grid, s);
+  if (fp8) return launch_quant<32, true, false>(tmX, p, grid, smem, s);
   switch (p.G) {
-    case 16: return table ? launch_quant<16, false, true>(tmX, p, grid, s) : launch_quant<16, false, false>(tmX, p, grid, s);
-    case 32: return table ? launch_quant<32, false, true>(tmX, p, grid, s) : launch_quant<32, false, false>(tmX, p, grid, s);
-    case 64: return table ? launch_quant<64, false, true>(tmX, p, grid, s) : launch_quant<64, false, false>(tmX, p, grid, s);
+    case 16: return table ? launch_quant<16, false, true>(tmX, p, grid, smem, s) : launch_quant<16, false, false>(tmX, p, grid, smem, s);
+    case 32: return table ? launch_quant<32, false, true>(tmX, p, grid, smem, s) : launch_quant<32, false, false>(tmX, p, grid, smem, s);
+    case 64: return table ? launch_quant<64, false, true>(tmX, p, grid, smem, s) : launch_quant<64, false, false>(tmX, p, grid, smem, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-size_t grouped_quant_smem(int E, int Kg) {
-  const size_t n = (size_t)E * Kg;
+size_t grouped_quant_smem(int E, int Kg, int R) {
+  const size_t n = (size_t)E * Kg * R;
   return ((n + 15) & ~(size_t)15) + ((2 * n + 15) & ~(size_t)15) + (size_t)E * sizeof(int);
 }
 
 cudaError_t launch_quantize_grouped(const GroupedQuantParams& p, int num_sms, cudaStream_t s) {
   if (p.Mp == 0) return cudaSuccess;
-  const size_t smem = grouped_quant_smem(p.E, p.Kg);
+  const size_t smem = grouped_quant_smem(p.E, p.Kg, p.R);
   if (smem > GROUPED_QUANT_SMEM_MAX) return cudaErrorInvalidValue;
   const long long items = (long long)p.Mp * (p.K / 32);
   const int grid = (int)std::max<long long>(1, std::min<long long>((items + 255) / 256, (long long)num_sms * 4));
@@ -913,19 +937,19 @@ cudaError_t launch_quantize_grouped(const GroupedQuantParams& p, int num_sms, cu
 }
 
 // W_L (§3.2/§3.3): the bf16 weight columns of the table's channels, one contiguous
-// N x K_L block; pad columns are zero.
+// N x K_L block in table order (group, slot); pad columns are zero.
 __global__ void __launch_bounds__(256) gather_wl_kernel(const uint16_t* __restrict__ W, int N, int K, int G,
-                                                        const int8_t* __restrict__ L, int Kg, int K_L,
+                                                        const int8_t* __restrict__ L, int n_table, int R, int K_L,
                                                         uint16_t* __restrict__ WL, int* status) {
   extern __shared__ int chan[];          // K_L entries: source channel, or -1 for pad
   if (threadIdx.x == 0) {
     int c = 0;
-    for (int k = 0; k < Kg; ++k) {
-      int v = L[k];
+    for (int i = 0; i < n_table; ++i) {
+      const int v = L[i];
       if (v >= G) { record_status(status, DEV_BAD_TABLE); continue; }
       if (v < 0) continue;
       if (c >= K_L) { record_status(status, DEV_BAD_TABLE); break; }
-      chan[c++] = k * G + v;
+      chan[c++] = (i / R) * G + v;
     }
     for (; c < K_L; ++c) chan[c] = -1;
   }
@@ -938,12 +962,12 @@ __global__ void __launch_bounds__(256) gather_wl_kernel(const uint16_t* __restri
   }
 }
 
-cudaError_t launch_gather_wl(const uint16_t* W, int N, int K, int G, const int8_t* L, int K_L, uint16_t* WL,
+cudaError_t launch_gather_wl(const uint16_t* W, int N, int K, int G, const int8_t* L, int R, int K_L, uint16_t* WL,
                              int* status, int num_sms, cudaStream_t s) {
   if (K_L == 0 || N == 0) return cudaSuccess;
   long long total = (long long)N * K_L;
   int grid = (int)std::min<long long>((total + 255) / 256, (long long)num_sms * 4);
-  gather_wl_kernel<<<grid, 256, (size_t)K_L * sizeof(int), s>>>(W, N, K, G, L, K / G, K_L, WL, status);
+  gather_wl_kernel<<<grid, 256, (size_t)K_L * sizeof(int), s>>>(W, N, K, G, L, (K / G) * R, R, K_L, WL, status);
   return cudaGetLastError();
 }
 

@@ -22,8 +22,10 @@ namespace osc {
 
 // One token's group of G bf16 values at xg (16-byte aligned): the channel of largest |x|
 // (lowest on ties, compared on the magnitude bits) and whether it is an outlier event.
+// Channels whose bit is set in `masked` count as zero (they were protected in an earlier
+// round of a multi-entry table build).
 template <int G>
-__device__ __forceinline__ bool group_event(const uint16_t* xg, float alpha, int* j_out) {
+__device__ __forceinline__ bool group_event(const uint16_t* xg, float alpha, int* j_out, uint64_t masked = 0) {
   const uint4* src = reinterpret_cast<const uint4*>(xg);
   float s = 0.0f;
   uint32_t best = 0;
@@ -34,7 +36,8 @@ __device__ __forceinline__ bool group_event(const uint16_t* xg, float alpha, int
     const uint32_t w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
-      const uint32_t mag = (h & 1) ? (w[h >> 1] >> 16) & 0x7FFFu : w[h >> 1] & 0x7FFFu;
+      uint32_t mag = (h & 1) ? (w[h >> 1] >> 16) & 0x7FFFu : w[h >> 1] & 0x7FFFu;
+      if ((masked >> (v * 8 + h)) & 1u) mag = 0u;
       s += __uint_as_float(mag << 16);
       if (mag > best) { best = mag; jb = v * 8 + h; }
     }
@@ -44,22 +47,34 @@ __device__ __forceinline__ bool group_event(const uint16_t* xg, float alpha, int
   return best != 0u && (double)G * amax >= (double)alpha * (double)s;
 }
 
+// R rounds (R protected channels at most): round r repeats the count with the channels of the
+// earlier rounds read as zero, which is what extraction leaves of the group; once a round finds
+// no channel the later ones find none either.
 template <int G>
 __global__ void __launch_bounds__(256) build_table_kernel(TableParams p) {
   __shared__ int hist[G];
+  __shared__ int s_pick;
   const int k = blockIdx.x;
-  for (int j = threadIdx.x; j < G; j += blockDim.x) hist[j] = 0;
-  __syncthreads();
-  for (int t = threadIdx.x; t < p.S; t += blockDim.x) {
-    int jb;
-    if (group_event<G>(p.X + (size_t)t * p.K + (size_t)k * G, p.alpha, &jb)) atomicAdd(&hist[jb], 1);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int js = 0;
-    for (int j = 1; j < G; ++j)
-      if (hist[j] > hist[js]) js = j;
-    p.L[k] = (hist[js] > 0 && hist[js] >= p.min_hits) ? (int8_t)js : (int8_t)-1;
+  uint64_t masked = 0;
+  for (int r = 0; r < p.R; ++r) {
+    for (int j = threadIdx.x; j < G; j += blockDim.x) hist[j] = 0;
+    __syncthreads();
+    for (int t = threadIdx.x; t < p.S; t += blockDim.x) {
+      int jb;
+      if (group_event<G>(p.X + (size_t)t * p.K + (size_t)k * G, p.alpha, &jb, masked)) atomicAdd(&hist[jb], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int js = 0;
+      for (int j = 1; j < G; ++j)
+        if (hist[j] > hist[js]) js = j;
+      s_pick = (hist[js] > 0 && hist[js] >= p.min_hits) ? js : -1;
+      p.L[(size_t)k * p.R + r] = (int8_t)s_pick;
+    }
+    __syncthreads();
+    const int pick = s_pick;
+    if (pick >= 0) masked |= 1ull << pick;
+    __syncthreads();                         // s_pick is read by all before the next round
   }
 }
 

@@ -160,6 +160,42 @@ def qkv_case(M: int, calib_tokens: int = 1536) -> LinearCase:
     return LinearCase(f"qkv_m{M}", M, 4096, 6144, 32, X, W, calib, planted_table(st, 32))
 
 
+def second_channel(st: Structure, frac: float, seed: int) -> Structure:
+    """A second fixed outlier channel in a fraction of the blocks that already hold one (the
+    extreme case of the OSC page's §6 multi-outlier protection): a structure whose fixed
+    channels are those second channels, drawn distinct from the first."""
+    rng = np.random.default_rng(seed)
+    fixed = np.full_like(st.fixed_ch, -1)
+    blocks = np.nonzero(st.fixed_ch >= 0)[0]
+    pick = rng.permutation(blocks)[: int(round(frac * blocks.size))]
+    for b in pick:
+        first = int(st.fixed_ch[b]) - b * BLOCK
+        j = int(rng.integers(0, BLOCK - 1))
+        fixed[b] = b * BLOCK + (j if j < first else j + 1)
+    return Structure(K=st.K, fixed_ch=fixed, sign=np.where(rng.random(st.fixed_ch.size) < 0.5, -1.0, 1.0))
+
+
+def two_outlier_case(M: int, calib_tokens: int = 1536) -> LinearCase:
+    """The QKV shape (K=4096, N=6144, G=32) where 40% of the blocks with a fixed channel
+    (+-U(20,80)) hold a second fixed channel at +-U(8,16) on every token: smaller than the
+    first, yet still an outlier once the first is taken out."""
+    st = make_structure(4096, 0.70, seed=1002)
+    st2 = second_channel(st, 0.40, seed=1202)
+
+    def draw(n, seed):
+        X = bf16_to_f32(gen_tokens(st, n, seed=seed, spike_frac=0.05)).copy()
+        rng = np.random.default_rng(seed + 1)
+        b = np.nonzero(st2.fixed_ch >= 0)[0]
+        vals = rng.uniform(8.0, 16.0, size=(n, b.size)) * st2.sign[b][None, :]
+        X[:, st2.fixed_ch[b]] = vals
+        return bf16_bits(X)
+
+    X = draw(M, 1302 + M)
+    calib = draw(calib_tokens, 1402)
+    W = gen_weights(6144, 4096, seed=2002)
+    return LinearCase(f"qkv2_m{M}", M, 4096, 6144, 32, X, W, calib, planted_table(st, 32))
+
+
 def ffn_case(G: int, M: int = 4096, calib_tokens: int = 1536) -> LinearCase:
     """Qwen3-8B FFN up/gate: K=4096, N=24576, fixed channels in 65% of 32-blocks."""
     st = make_structure(4096, 0.65, seed=1003)

@@ -46,12 +46,13 @@ def lib() -> ctypes.CDLL:
             "osc_scale_bytes": ([i32, i32, i32], ctypes.c_size_t),
             "osc_table_kl": ([P, i32], i32),
             "osc_build_table": ([P, i32, i32, i32, f32, i32, P, P], i32),
+            "osc_build_table_multi": ([P, i32, i32, i32, f32, i32, i32, P, P], i32),
             "osc_density": ([P, i32, i32, i32, f32, P, P, P, P], i32),
             "osc_select_tier": ([P, P, i32, P], i32),
             "osc_select_group_size": ([P, P], i32),
-            "osc_quantize": ([P, i32, i32, i32, P, i32, P, P, P, P], i32),
-            "osc_rmsnorm_quantize": ([P, P, f32, i32, i32, i32, P, i32, P, P, P, P], i32),
-            "osc_prepare_weight": ([P, i32, i32, i32, P, i32, P, P, P, P], i32),
+            "osc_quantize": ([P, i32, i32, i32, P, i32, i32, P, P, P, P], i32),
+            "osc_rmsnorm_quantize": ([P, P, f32, i32, i32, i32, P, i32, i32, P, P, P, P], i32),
+            "osc_prepare_weight": ([P, i32, i32, i32, P, i32, i32, P, P, P, P], i32),
             "osc_linear": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P], i32),
             "osc_linear_workspace_bytes": ([i32, i32, i32, i32], ctypes.c_size_t),
             "osc_linear_splitk": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P, ctypes.c_size_t, P], i32),
@@ -59,7 +60,7 @@ def lib() -> ctypes.CDLL:
             "osc_quantize_fp8": ([P, i32, i32, P, P, P], i32),
             "osc_linear_fp8_fallback": ([P, P, P, P, i32, i32, i32, P, P, P], i32),
             "osc_grouped_plan": ([P, i32, P, P, P, i32], i32),
-            "osc_quantize_grouped": ([P, i32, i32, P, P, P, i32, i32, i32, P, i32, P, P, P, P], i32),
+            "osc_quantize_grouped": ([P, i32, i32, P, P, P, i32, i32, i32, P, i32, i32, P, P, P, P], i32),
             "osc_linear_grouped": ([P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P], i32),
             "osc_status": ([P, P], i32),
             "osc_selftest_timeout": ([i32, P], i32),
@@ -125,6 +126,22 @@ def osc_build_table(Xcal, G: int, alpha: float, min_hits: int, L, stream=None):
     _check("osc_build_table", lib().osc_build_table(_ptr(Xcal), S, K, G, alpha, min_hits, _ptr(L), _stream(stream)))
 
 
+def osc_build_table_multi(Xcal, G: int, alpha: float, min_hits: int, R: int, L, stream=None):
+    """Up to R protected channels per group into L (int8 CUDA tensor of K/G x R entries)."""
+    S, K = Xcal.shape
+    _check("osc_build_table_multi", lib().osc_build_table_multi(_ptr(Xcal), S, K, G, alpha, min_hits, R, _ptr(L),
+                                                                _stream(stream)))
+
+
+def _slots(L, groups: int) -> int:
+    """Protected channels per group of a table tensor holding `groups` groups (1 without one)."""
+    if L is None:
+        return 1
+    if L.numel() % groups:
+        raise ValueError("table size is not a multiple of the group count")
+    return L.numel() // groups
+
+
 def osc_density(X, G: int, alpha: float, L, n_hit, n_total, stream=None):
     """Per-group outlier-event and table-hit counts (int32 CUDA tensors of K/G entries)."""
     S, K = X.shape
@@ -163,20 +180,22 @@ def osc_select_group_size(c_bar16: float, c_bar32: float, c_bar64: float):
 
 def osc_quantize(X, G: int, L, K_L: int, QX, SX, B, stream=None):
     M, K = X.shape
-    _check("osc_quantize", lib().osc_quantize(_ptr(X), M, K, G, _ptr(L), K_L, _ptr(QX), _ptr(SX),
+    _check("osc_quantize", lib().osc_quantize(_ptr(X), M, K, G, _ptr(L), _slots(L, K // G), K_L, _ptr(QX), _ptr(SX),
                                               _ptr(B) if K_L else None, _stream(stream)))
 
 
 def osc_rmsnorm_quantize(X, gamma, eps: float, G: int, L, K_L: int, QX, SX, B, stream=None):
     M, K = X.shape
-    _check("osc_rmsnorm_quantize", lib().osc_rmsnorm_quantize(_ptr(X), _ptr(gamma), eps, M, K, G, _ptr(L), K_L,
+    _check("osc_rmsnorm_quantize", lib().osc_rmsnorm_quantize(_ptr(X), _ptr(gamma), eps, M, K, G, _ptr(L),
+                                                              _slots(L, K // G), K_L,
                                                               _ptr(QX), _ptr(SX), _ptr(B) if K_L else None,
                                                               _stream(stream)))
 
 
 def osc_prepare_weight(W, G: int, L, K_L: int, QW, SW, WL, stream=None):
     N, K = W.shape
-    _check("osc_prepare_weight", lib().osc_prepare_weight(_ptr(W), N, K, G, _ptr(L), K_L, _ptr(QW), _ptr(SW),
+    _check("osc_prepare_weight", lib().osc_prepare_weight(_ptr(W), N, K, G, _ptr(L), _slots(L, K // G), K_L,
+                                                          _ptr(QW), _ptr(SW),
                                                           _ptr(WL) if K_L else None, _stream(stream)))
 
 
@@ -242,7 +261,8 @@ def osc_grouped_plan(counts):
 def osc_quantize_grouped(X, E: int, off, poff, mblock_expert, Mp: int, G: int, L, K_L: int, QX, SX, B, stream=None):
     T, K = X.shape
     _check("osc_quantize_grouped", lib().osc_quantize_grouped(_ptr(X), T, E, _ptr(off), _ptr(poff), _ptr(mblock_expert),
-                                                              Mp, K, G, _ptr(L), K_L, _ptr(QX), _ptr(SX),
+                                                              Mp, K, G, _ptr(L), _slots(L, E * (K // G)), K_L,
+                                                              _ptr(QX), _ptr(SX),
                                                               _ptr(B) if K_L else None, _stream(stream)))
 
 

@@ -7,6 +7,7 @@ bench.py, which sweeps every row.
 CASE:
   qkv           osc_quantize + osc_linear, QKV projection (K=4096, N=6144), M=--m (2048), G=--g (32)
   weight_bound  osc_linear alone at few token rows (QKV weights, M=--m, default 16)
+  weight_bound_split  osc_linear_splitk at few token rows (K split over SMs, chained reduction)
   ffn           osc_quantize + osc_linear, FFN up (K=4096, N=24576, M=4096), G=--g
   w2_osc        osc_quantize + osc_linear, down projection (K=12288, N=4096, M=4096), G=32
   w2_fp8        osc_quantize_fp8 + osc_linear_fp8_fallback on the down projection
@@ -39,7 +40,7 @@ def _table(calib, K, G):
     return Ld, osc.osc_table_kl(Ld.cpu().numpy())
 
 
-def _dense(case, G, launches, linear_only=False, M=None):
+def _dense(case, G, launches, linear_only=False, M=None, split=False):
     X = case.X if M is None else case.X[:M]
     M, K = X.shape
     N = case.W.shape[0]
@@ -48,10 +49,14 @@ def _dense(case, G, launches, linear_only=False, M=None):
     Xd = _dev(X)
     QX, SX, B = osc.quantize(Xd, G, Ld, K_L)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(max(16, osc.osc_linear_workspace_bytes(M, N, K, K_L)), dtype=torch.uint8, device="cuda")
     for _ in range(launches):
         if not linear_only:
             osc.osc_quantize(Xd, G, Ld, K_L, QX, SX, B)
-        osc.osc_linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y)
+        if split:
+            osc.osc_linear_splitk(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y, ws)
+        else:
+            osc.osc_linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y)
 
 
 def _fp8(case, launches):
@@ -97,7 +102,8 @@ def _moe(which, launches):
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("case", choices=["qkv", "weight_bound", "ffn", "w2_osc", "w2_fp8", "moe_gateup", "moe_down"])
+    ap.add_argument("case", choices=["qkv", "weight_bound", "weight_bound_split", "ffn", "w2_osc", "w2_fp8",
+                                     "moe_gateup", "moe_down"])
     ap.add_argument("--launches", type=int, default=4, help="rounds of the workload's kernels")
     ap.add_argument("--m", type=int, default=None, help="token rows (qkv: 2048, weight_bound: 16)")
     ap.add_argument("--g", type=int, default=32, help="group size (qkv, ffn)")
@@ -105,8 +111,8 @@ def main(argv=None):
     osc.lib()
     if a.case == "qkv":
         _dense(I.qkv_case(a.m or 2048), a.g, a.launches)
-    elif a.case == "weight_bound":
-        _dense(I.qkv_case(a.m or 16), 32, a.launches, linear_only=True)
+    elif a.case in ("weight_bound", "weight_bound_split"):
+        _dense(I.qkv_case(a.m or 16), 32, a.launches, linear_only=True, split=a.case.endswith("split"))
     elif a.case == "ffn":
         _dense(I.ffn_case(a.g), a.g, a.launches)
     elif a.case == "w2_osc":
