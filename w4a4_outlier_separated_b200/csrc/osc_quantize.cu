@@ -361,14 +361,6 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
   if (lane == 0) { mbar_init(smem_u32(&s_bar[warp][0]), 1); mbar_init(smem_u32(&s_bar[warp][1]), 1); }
   fence_barrier_init();
   __syncwarp();
-  // Every box this warp will load goes to L2 before the wait for the previous kernel: a
-  // prefetch changes no value a later load returns (L2 is where the previous kernel's writes
-  // land), so it is safe even when X is that kernel's output, and when X is already resident it
-  // costs nothing. If this CTA starts while the previous kernel's last wave still runs, X
-  // streams in meanwhile.
-  if (lane == 0)
-    for (uint32_t st = step; st < cta_end; st += wstride)
-      if (st * QSTEP < real_items) tma_prefetch_l2_2d(&tmX, 0, (int)(st * QSTEP));
   // X, L and the outputs are free of the previous kernel. No early trigger for the next one:
   // quantize CTAs are small enough to share SMs, so an early-launched next grid would hold SM
   // slots while it waits; the next kernel is released when this grid completes.

@@ -8,6 +8,7 @@ CASE:
   qkv           osc_quantize + osc_linear, QKV projection (K=4096, N=6144), M=--m (2048), G=--g (32)
   weight_bound  osc_linear alone at few token rows (QKV weights, M=--m, default 16)
   weight_bound_split  osc_linear_splitk at few token rows (K split over SMs, chained reduction)
+  qkv_rmsnorm   osc_rmsnorm_quantize + osc_linear at the QKV shape (M=--m, default 2048), G=--g
   ffn           osc_quantize + osc_linear, FFN up (K=4096, N=24576, M=4096), G=--g
   w2_osc        osc_quantize + osc_linear, down projection (K=12288, N=4096, M=4096), G=32
   w2_fp8        osc_quantize_fp8 + osc_linear_fp8_fallback on the down projection
@@ -59,6 +60,21 @@ def _dense(case, G, launches, linear_only=False, M=None, split=False):
             osc.osc_linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y)
 
 
+def _rmsnorm(case, G, launches):
+    M, K = case.X.shape
+    N = case.W.shape[0]
+    gamma = torch.from_numpy((1.0 + 0.1 * np.random.default_rng(1).standard_normal(K)).astype(np.float32))
+    gbits = gamma.to(torch.bfloat16).view(torch.int16).cuda()
+    Ld, K_L = _table(case.calib, K, G)
+    QW, SW, WL = osc.prepare_weight(_dev(case.W), G, Ld, K_L)
+    Xd = _dev(case.X)
+    QX, SX, B = osc.alloc_quantize_outputs(M, K, G, K_L, "cuda")
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    for _ in range(launches):
+        osc.osc_rmsnorm_quantize(Xd, gbits, 1e-6, G, Ld, K_L, QX, SX, B)
+        osc.osc_linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y)
+
+
 def _fp8(case, launches):
     M, K = case.X.shape
     N = case.W.shape[0]
@@ -102,8 +118,8 @@ def _moe(which, launches):
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("case", choices=["qkv", "weight_bound", "weight_bound_split", "ffn", "w2_osc", "w2_fp8",
-                                     "moe_gateup", "moe_down"])
+    ap.add_argument("case", choices=["qkv", "qkv_rmsnorm", "weight_bound", "weight_bound_split", "ffn", "w2_osc",
+                                     "w2_fp8", "moe_gateup", "moe_down"])
     ap.add_argument("--launches", type=int, default=4, help="rounds of the workload's kernels")
     ap.add_argument("--m", type=int, default=None, help="token rows (qkv: 2048, weight_bound: 16)")
     ap.add_argument("--g", type=int, default=32, help="group size (qkv, ffn)")
@@ -111,6 +127,8 @@ def main(argv=None):
     osc.lib()
     if a.case == "qkv":
         _dense(I.qkv_case(a.m or 2048), a.g, a.launches)
+    elif a.case == "qkv_rmsnorm":
+        _rmsnorm(I.qkv_case(a.m or 2048), a.g, a.launches)
     elif a.case in ("weight_bound", "weight_bound_split"):
         _dense(I.qkv_case(a.m or 16), 32, a.launches, linear_only=True, split=a.case.endswith("split"))
     elif a.case == "ffn":
