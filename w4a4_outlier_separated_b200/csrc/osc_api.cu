@@ -161,8 +161,10 @@ int run_gemm_small(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_
     if ((rc = make_map(&maps.x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, QX, dx, st, boxx, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
   }
   {
+    // boxes of a whole scale chunk: SMALL_CHUNK_ATOMS atoms of one 128-row block
     uint64_t d[3] = {128, (uint64_t)nslot4, (uint64_t)((N + 127) / 128)}, st[2] = {512, (uint64_t)nslot4 * 512};
-    uint32_t box[3] = {128, aps, 1};
+    uint32_t box[3] = {128, (uint32_t)osc::SMALL_CHUNK_ATOMS, 1};
+    (void)aps;
     if ((rc = make_map(&maps.sw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, SW, d, st, box, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
     uint64_t dx[3] = {128, (uint64_t)nslot4, 1};
     if ((rc = make_map(&maps.sx, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, SX, dx, st, box, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
@@ -179,6 +181,9 @@ int run_gemm_small(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_
   std::memset(&p, 0, sizeof(p));
   p.M = M; p.N = N; p.K = K; p.K_L = K_L;
   p.S = pl.S; p.n_tiles = pl.n_tiles; p.num_sms = ds->sms;
+  // a grid that leaves at least half the SMs free lets the next launch's CTAs start early:
+  // they prefetch their weights into L2 while this one runs
+  p.prefetch = pl.n_tiles * pl.S <= ds->sms / 2 ? 1 : 0;
   p.Y = Y; p.Yf32 = Yf32; p.partial = pl.S > 1 ? workspace : nullptr;
   p.status = ds->status;
   const int units = pl.n_tiles * pl.S;

@@ -128,6 +128,7 @@ cudaError_t launch_gemm(int kind, int bn, int cg, const GemmMaps& maps, const Ge
 struct SmallParams {
   int M, N, K, K_L;
   int S, n_tiles, num_sms;
+  int prefetch;          // 1: prefetch each unit's weights into L2 before the dependency wait
   uint16_t* Y;
   float* Yf32;
   float* partial;
@@ -137,6 +138,9 @@ struct SmallMaps {
   CUtensorMap w, x, sw, sx, wl, b;
 };
 int small_token_tile(int M);   // MMA N for M token rows: 16, 32, 64 or 128
+// Scale atoms (512 bytes: 128 rows x 4 slots) one scale chunk of the few-row product holds
+// per operand: the host encodes the scale maps with boxes of this many atoms.
+constexpr int SMALL_CHUNK_ATOMS = 16;
 cudaError_t launch_gemm_small(int kind, const SmallMaps& maps, const SmallParams& p, int grid, cudaStream_t s);
 
 struct TableParams {

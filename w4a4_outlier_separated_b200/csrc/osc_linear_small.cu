@@ -18,8 +18,8 @@
 // S = 1 the unit writes Y itself. Either way the result does not depend on timing.
 //
 // Roles (256 threads): warp 0 lane 0 TMA producer; warp 1 lane 0 MMA issuer; warp 2 TMEM
-// allocator, then (lane 0) scale copier of odd stages; warp 3 lane 0 scale copier of even
-// stages; warps 4..7 epilogue, warp w reading TMEM lanes 32 (w % 4) .. + 31 (weight rows).
+// allocator; warp 3 lane 0 scale copier; warps 4..7 epilogue, warp w reading TMEM lanes
+// 32 (w % 4) .. + 31 (weight rows).
 #include "osc_device.cuh"
 #include "osc_internal.h"
 
@@ -31,24 +31,26 @@ struct SmallCfg {
   static constexpr int V = KIND == KIND_MXF4_B16 ? 16 : 32;
   static constexpr int ELEMS = FP8 ? 128 : 256;                 // K elements per stage (128 bytes a row)
   static constexpr int APS = ELEMS / (4 * V);                   // scale atoms per stage and operand
+  static constexpr int SC = SMALL_CHUNK_ATOMS / APS;            // FP4/FP8 stages per scale chunk
   static constexpr int A_BYTES = 128 * 128;                     // weight tile: 128 rows x 128 bytes
   static constexpr int B_BYTES = NT * 128;                      // token tile: NT rows x 128 bytes
-  static constexpr int SF_BYTES = APS * 512;
-  static constexpr int STAGE_RAW = A_BYTES + B_BYTES + 2 * SF_BYTES;
-  static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;         // a multiple of 1 KB
+  static constexpr int CHUNK_OP_BYTES = SMALL_CHUNK_ATOMS * 512;
+  static constexpr int CHUNK_BYTES = 2 * CHUNK_OP_BYTES;        // weight atoms, then token atoms
+  static constexpr int CHUNKS = 2;                              // scale chunk buffers
   static constexpr int BAR_BYTES = 1024;
   static constexpr int SMEM_LIMIT = 232448;
-  static constexpr int STAGES_FIT = (SMEM_LIMIT - BAR_BYTES - 1024) / STAGE_BYTES;
+  static constexpr int STAGES_FIT = (SMEM_LIMIT - BAR_BYTES - 1024 - CHUNKS * CHUNK_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
-  static constexpr int SMEM_TOTAL = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static constexpr int SMEM_TOTAL = STAGES * STAGE_BYTES + CHUNKS * CHUNK_BYTES + BAR_BYTES + 1024;
   static constexpr int ACC_COLS = NT < 32 ? 32 : NT;            // one accumulator (TMEM columns)
-  static constexpr int SF_SET = 2 * APS * 4;                    // weight atoms, then token atoms
-  static constexpr int SFW_COL = 2 * ACC_COLS;                  // two accumulators, then the scale sets
+  static constexpr int CHUNK_COLS = 2 * SMALL_CHUNK_ATOMS * 4;  // TMEM columns of one chunk's scales
+  static constexpr int SF_COL = 2 * ACC_COLS;                   // two accumulators, then the chunks
   static constexpr int TMEM_COLS = 512;
-  static constexpr uint32_t MAIN_TX = A_BYTES + B_BYTES + 2 * SF_BYTES;
-  static constexpr uint32_t COMP_TX = A_BYTES + B_BYTES;
-  static_assert(SFW_COL + STAGES * SF_SET <= TMEM_COLS, "TMEM budget");
+  static constexpr uint32_t DATA_TX = A_BYTES + B_BYTES;        // every stage (FP4 and compensation)
+  static_assert(SF_COL + CHUNKS * CHUNK_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(STAGES >= 3, "smem budget");
+  static_assert(SC >= 1 && SC * APS == SMALL_CHUNK_ATOMS, "chunk of whole stages");
   static_assert(NT == 16 || NT == 32 || NT == 64 || NT == 128, "token tile");
 };
 
@@ -60,6 +62,11 @@ __device__ __forceinline__ void unit_range(int s, int S, int T, int& i0, int& i1
 
 constexpr int SMALL_THREADS = 256;
 
+// The scales of a unit's block-scaled stages come in chunks of SC stages (SMALL_CHUNK_ATOMS
+// atoms per operand, one TMA box each), double-buffered in shared memory and TMEM: one thread
+// copies a whole chunk into TMEM back to back and publishes it once, so the MMA issuer waits
+// for scales once per chunk instead of once per stage, and the per-stage ring carries only the
+// operand tiles.
 template <int NT, int KIND>
 __global__ void __launch_bounds__(SMALL_THREADS, 1)
 gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -72,16 +79,19 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
   const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw_addr + pad;
-  uint8_t* bar_area = smem + C::STAGES * C::STAGE_BYTES;
+  const uint32_t schunk0 = sbase + C::STAGES * C::STAGE_BYTES;            // chunk buffers
+  uint8_t* bar_area = smem + C::STAGES * C::STAGE_BYTES + C::CHUNKS * C::CHUNK_BYTES;
   const uint32_t bar0 = smem_u32(bar_area);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
-  auto sfready_bar = [&](int s) { return bar0 + 8u * (2 * C::STAGES + s); };
-  auto accf_bar = [&](int a) { return bar0 + 8u * (3 * C::STAGES + a); };
-  auto acce_bar = [&](int a) { return bar0 + 8u * (3 * C::STAGES + 2 + a); };
-  auto tear_bar = [&](int i) { return bar0 + 8u * (3 * C::STAGES + 4 + i); };   // 3 of them
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 8 * (3 * C::STAGES + 8));
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (3 * C::STAGES + 8) + 8);
+  auto cfull_bar = [&](int c) { return bar0 + 8u * (2 * C::STAGES + c); };       // chunk landed
+  auto cready_bar = [&](int c) { return bar0 + 8u * (2 * C::STAGES + 2 + c); };  // chunk in TMEM
+  auto cempty_bar = [&](int c) { return bar0 + 8u * (2 * C::STAGES + 4 + c); };  // chunk's MMAs done
+  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 6 + a); };
+  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 8 + a); };
+  auto tear_bar = [&](int i) { return bar0 + 8u * (2 * C::STAGES + 10 + i); };  // 2 of them
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 8 * (2 * C::STAGES + 12));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (2 * C::STAGES + 12) + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_k = p.K / C::ELEMS;
@@ -89,30 +99,14 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
   const int T = n_k + n_c;
   const int units = p.n_tiles * p.S;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); mbar_init(sfready_bar(s), 1);
-    }
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
+    for (int c = 0; c < C::CHUNKS; ++c) { mbar_init(cfull_bar(c), 1); mbar_init(cready_bar(c), 1); mbar_init(cempty_bar(c), 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(accf_bar(a), 1); mbar_init(acce_bar(a), 4); }
-    for (int i = 0; i < 3; ++i) mbar_init(tear_bar(i), 1);
+    for (int i = 0; i < 2; ++i) mbar_init(tear_bar(i), 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmW); tma_prefetch_desc(&tmX); tma_prefetch_desc(&tmSW); tma_prefetch_desc(&tmSX);
     if (p.K_L > 0) { tma_prefetch_desc(&tmWL); tma_prefetch_desc(&tmB); }
-    // the weights of this CTA's first two units go to L2 now, before waiting for the previous
-    // kernel: they are not its output, and a prefetch changes no value a later load returns
-    for (int u = blockIdx.x, r = 0; u < units && r < 2; u += gridDim.x, ++r) {
-      const int tile = u / p.S, s = u % p.S, n0 = tile * 128;
-      int i0, i1;
-      unit_range(s, p.S, T, i0, i1);
-      for (int i = i0; i < i1; ++i) {
-        if (i < n_k) {
-          tma_prefetch_l2_2d(&tmW, i * 128, n0);
-          tma_prefetch_l2_3d(&tmSW, 0, i * C::APS, n0 / 128);
-        } else {
-          tma_prefetch_l2_2d(&tmWL, (i - n_k) * 64, n0);
-        }
-      }
-    }
   }
   if (warp == 2) { tc_alloc<1>(smem_u32(tmem_slot), C::TMEM_COLS); tc_relinquish<1>(); }
   tc_fence_before();
@@ -120,30 +114,52 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) grid_dep_launch();   // the split's reduction may be scheduled now
+  if (warp == 0 && lane == 0 && p.prefetch) {
+    // When the grid leaves SMs free, this CTA may start while the previous kernel still runs:
+    // the weights of its first two units go to L2 now. They are not that kernel's output, and
+    // a prefetch changes no value a later load returns.
+    for (int u = blockIdx.x, r = 0; u < units && r < 2; u += gridDim.x, ++r) {
+      const int tile = u / p.S, s = u % p.S, n0 = tile * 128;
+      int i0, i1;
+      unit_range(s, p.S, T, i0, i1);
+      for (int i = i0; i < i1; ++i) {
+        if (i < n_k) tma_prefetch_l2_2d(&tmW, i * 128, n0);
+        else tma_prefetch_l2_2d(&tmWL, (i - n_k) * 64, n0);
+      }
+    }
+  }
   grid_dep_wait();                           // Q_X, S_X and B of the previous kernel are visible
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------------ TMA producer
     int stage = 0; uint32_t phase = 0;
-    long long fills = 0;
+    int cb = 0; uint32_t cphase = 0;
+    long long fills = 0, cfills = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       const int tile = u / p.S, s = u % p.S, n0 = tile * 128;
       int i0, i1;
       unit_range(s, p.S, T, i0, i1);
       for (int i = i0; i < i1; ++i) {
+        if (i < n_k && (i - i0) % C::SC == 0) {
+          // the scale chunk of stages i .. i + SC - 1 (atoms past the unit's range are unused)
+          if (!(ok = mbar_wait(cempty_bar(cb), cphase ^ 1, abort_flag, p.status))) break;
+          const uint32_t dst = schunk0 + cb * C::CHUNK_BYTES;
+          mbar_arrive_expect_tx(cfull_bar(cb), C::CHUNK_BYTES);
+          tma_load_3d(dst, &tmSW, 0, i * C::APS, n0 / 128, cfull_bar(cb));
+          tma_load_3d(dst + C::CHUNK_OP_BYTES, &tmSX, 0, i * C::APS, 0, cfull_bar(cb));
+          ++cfills;
+          if (++cb == C::CHUNKS) { cb = 0; cphase ^= 1; }
+        }
         if (!(ok = mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, p.status))) break;
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
         const uint32_t fb = full_bar(stage);
+        mbar_arrive_expect_tx(fb, C::DATA_TX);
         if (i < n_k) {
-          mbar_arrive_expect_tx(fb, C::MAIN_TX);
           tma_load_2d(st, &tmW, i * 128, n0, fb);
           tma_load_2d(st + C::A_BYTES, &tmX, i * 128, 0, fb);
-          tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSW, 0, i * C::APS, n0 / 128, fb);
-          tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SF_BYTES, &tmSX, 0, i * C::APS, 0, fb);
         } else {
           const int c = i - n_k;
-          mbar_arrive_expect_tx(fb, C::COMP_TX);
           tma_load_2d(st, &tmWL, c * 64, n0, fb);
           tma_load_2d(st + C::A_BYTES, &tmB, c * 64, 0, fb);
         }
@@ -153,32 +169,40 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
     }
     if (*abort_flag) {
       // let the copies armed on this CTA's barriers land before the CTA exits
+      volatile int never = 0;
       const long long last = fills < C::STAGES ? fills : C::STAGES;
-      for (long long f = fills - last; f < fills; ++f) {
-        volatile int never = 0;
+      for (long long f = fills - last; f < fills; ++f)
         mbar_wait(full_bar((int)(f % C::STAGES)), (uint32_t)((f / C::STAGES) & 1), &never, nullptr, 100000000ull);
-      }
+      const long long clast = cfills < C::CHUNKS ? cfills : C::CHUNKS;
+      for (long long f = cfills - clast; f < cfills; ++f)
+        mbar_wait(cfull_bar((int)(f % C::CHUNKS)), (uint32_t)((f / C::CHUNKS) & 1), &never, nullptr, 100000000ull);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------------ MMA issuer
     int stage = 0; uint32_t phase = 0;
+    int cb = 0; uint32_t cphase = 0;
     int acc = 0; uint32_t aphase = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       const int s = u % p.S;
       int i0, i1;
       unit_range(s, p.S, T, i0, i1);
+      const int fp_end = min(i1, n_k);                        // the unit's block-scaled stages end here
       if (!(ok = mbar_wait(acce_bar(acc), aphase ^ 1, abort_flag, p.status))) break;
       tc_fence_after();
       const uint32_t d = tmem + acc * C::ACC_COLS;
       bool first = true;
       for (int i = i0; i < i1; ++i) {
+        const int in_chunk = (i - i0) % C::SC;
+        if (i < n_k && in_chunk == 0) {
+          if (!(ok = mbar_wait(cready_bar(cb), cphase, abort_flag, p.status))) break;   // scales in TMEM
+        }
         if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, p.status))) break;
-        if (!(ok = mbar_wait(sfready_bar(stage), phase, abort_flag, p.status))) break;
         tc_fence_after();
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
-        const uint32_t sfo = tmem + C::SFW_COL + stage * C::SF_SET;   // weight atoms, then token atoms
         if (i < n_k) {
+          const uint32_t sfw = tmem + C::SF_COL + cb * C::CHUNK_COLS + in_chunk * C::APS * 4;
+          const uint32_t sfx = sfw + SMALL_CHUNK_ATOMS * 4;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint64_t ad = desc_kmajor_sw128(st + 32 * j);
@@ -188,13 +212,17 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
             if constexpr (KIND == KIND_MXF4_B32) {
               const uint32_t sf = 2 * (j & 1), atom = j >> 1;
               tc_mma_mxf4_b32_g<1>(d, ad, bd, idesc_bs_m(FMT_MXF4_E2M1, 128, NT, sf, sf),
-                                   sfo + 4 * atom, sfo + C::APS * 4 + 4 * atom, accum);
+                                   sfw + 4 * atom, sfx + 4 * atom, accum);
             } else if constexpr (KIND == KIND_MXF4_B16) {
-              tc_mma_mxf4_b16_g<1>(d, ad, bd, idesc_bs_m(FMT_MXF4_E2M1, 128, NT, 0, 0),
-                                   sfo + 4 * j, sfo + C::APS * 4 + 4 * j, accum);
+              tc_mma_mxf4_b16_g<1>(d, ad, bd, idesc_bs_m(FMT_MXF4_E2M1, 128, NT, 0, 0), sfw + 4 * j, sfx + 4 * j, accum);
             } else {
-              tc_mma_mxf8_g<1>(d, ad, bd, idesc_bs_m(FMT_F8_E4M3, 128, NT, j, j), sfo, sfo + C::APS * 4, accum);
+              tc_mma_mxf8_g<1>(d, ad, bd, idesc_bs_m(FMT_F8_E4M3, 128, NT, j, j), sfw, sfx, accum);
             }
+          }
+          tc_commit_to<1>(empty_bar(stage));
+          if (in_chunk == C::SC - 1 || i == fp_end - 1) {     // the chunk's MMAs are all issued
+            tc_commit_to<1>(cempty_bar(cb));
+            if (++cb == C::CHUNKS) { cb = 0; cphase ^= 1; }
           }
         } else {
           const int c = i - n_k;
@@ -204,8 +232,8 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
                              idesc_bf16_m(128, NT), first ? 0u : 1u);
             first = false;
           }
+          tc_commit_to<1>(empty_bar(stage));
         }
-        tc_commit_to<1>(empty_bar(stage));
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
       if (!ok) break;
@@ -218,41 +246,35 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
       volatile int never = 0;
       mbar_wait(tear_bar(0), 0, &never, nullptr, 100000000ull);
     }
-  } else if ((warp == 2 || warp == 3) && lane == 0) {
-    // ------------------------------------------------------------------ scale copiers
-    // alternate stages of the sequence the MMA issuer walks; a stage's scale set is free again
-    // once its data has landed anew (the producer refills a stage only after the MMAs that read
-    // it, and its scale set, have completed)
-    const uint32_t mine = warp == 3 ? 0u : 1u;
-    int stage = 0; uint32_t phase = 0;
-    uint32_t seq = 0;
+  } else if (warp == 3 && lane == 0) {
+    // ------------------------------------------------------------------ scale copier
+    // a chunk's TMEM set is free again once its smem buffer is refilled: the producer reloads
+    // a buffer only after the MMAs that read the previous chunk there have completed
+    int cb = 0; uint32_t cphase = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       const int s = u % p.S;
       int i0, i1;
       unit_range(s, p.S, T, i0, i1);
-      for (int i = i0; i < i1; ++i, ++seq) {
-        if ((seq & 1u) == mine) {
-          if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, p.status))) break;
-          if (i < n_k) {
-            tc_fence_after();
-            const uint32_t s_sf = sbase + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
-            const uint32_t sfo = tmem + C::SFW_COL + stage * C::SF_SET;
-#pragma unroll
-            for (int a = 0; a < 2 * C::APS; ++a) tc_cp_atom<1>(sfo + 4 * a, desc_scale_atom(s_sf + 512 * a));
-            tc_commit_local<1>(sfready_bar(stage));
-          } else {
-            mbar_arrive(sfready_bar(stage));                 // compensation stages carry no scales
-          }
+      const int n_fp = max(0, min(i1, n_k) - i0);
+      for (int c = 0; c < (n_fp + C::SC - 1) / C::SC; ++c) {
+        if (!(ok = mbar_wait(cfull_bar(cb), cphase, abort_flag, p.status))) break;
+        tc_fence_after();
+        const uint32_t src = schunk0 + cb * C::CHUNK_BYTES;
+        const uint32_t dst = tmem + C::SF_COL + cb * C::CHUNK_COLS;
+        const int atoms = min(C::SC, n_fp - c * C::SC) * C::APS;   // the atoms the chunk's MMAs read
+        for (int a = 0; a < atoms; ++a) {
+          tc_cp_atom<1>(dst + 4 * a, desc_scale_atom(src + 512 * a));
+          tc_cp_atom<1>(dst + SMALL_CHUNK_ATOMS * 4 + 4 * a, desc_scale_atom(src + C::CHUNK_OP_BYTES + 512 * a));
         }
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        tc_commit_local<1>(cready_bar(cb));
+        if (++cb == C::CHUNKS) { cb = 0; cphase ^= 1; }
       }
     }
     if (*abort_flag) {
-      const uint32_t tb = tear_bar(warp == 3 ? 1 : 2);
-      tc_commit_local<1>(tb);
+      tc_commit_local<1>(tear_bar(1));
       volatile int never = 0;
-      mbar_wait(tb, 0, &never, nullptr, 100000000ull);
+      mbar_wait(tear_bar(1), 0, &never, nullptr, 100000000ull);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ epilogue
