@@ -351,7 +351,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const int half = (warp - 4) >> 2;                  // which half of the accumulator columns
     const int ew = warp - 4;
     const uint32_t stg = s_staging + ew * (32 * 32);
-    uint8_t* stg_ptr = smem + C::STAGES * C::STAGE_BYTES + ew * (32 * 32);
+    uint8_t* stg_ptr = smem + C::STAGES * C::STAGE_BYTES + C::CHUNKS * C::CHUNK_BYTES + ew * (32 * 32);
     constexpr int NCH = C::EPI_COLS / 32;              // 32-column chunks per warp (4 or 2)
     int acc = 0; uint32_t aphase = 0;
     for (int t = unit; t < num_tiles; t += nunits) {
