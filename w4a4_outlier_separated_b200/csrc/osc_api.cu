@@ -238,7 +238,7 @@ int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
     // scale buffers as (128 words of an atom) x (atoms along K) x (128-row blocks)
     const uint64_t mblk = (uint64_t)((M + 127) / 128);
     uint64_t d[3] = {128, (uint64_t)nslot4, mblk}, st[2] = {512, (uint64_t)nslot4 * 512};
-    uint32_t box[3] = {128, (uint32_t)osc::GEMM_CHUNK_ATOMS, 1};            // one scale chunk
+    uint32_t box[3] = {128, (uint32_t)(fp8 ? 1 : (V == 16 ? 4 : 2)), 1};
     if ((rc = make_map(&maps.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, SX, d, st, box, CU_TENSOR_MAP_SWIZZLE_NONE))) return rc;
     const uint64_t nblk = (uint64_t)((N + 127) / 128) * (uint64_t)E;
     uint64_t d2[3] = {128, (uint64_t)nslot4, nblk};

@@ -96,10 +96,6 @@ constexpr int GROUPED_QUANT_SMEM_MAX = 200 * 1024;
 cudaError_t launch_gather_wl(const uint16_t* W, int N, int K, int G, const int8_t* L, int R, int K_L, uint16_t* WL,
                              int* status, int num_sms, cudaStream_t s);
 
-// Scale atoms (128 rows x 4 slots) per 128-row block in one scale chunk of the general product:
-// the host encodes its scale maps with boxes of this many atoms.
-constexpr int GEMM_CHUNK_ATOMS = 8;
-
 // GEMM operand kinds
 enum GemmKind : int { KIND_MXF4_B32 = 0, KIND_MXF4_B16 = 1, KIND_MXF8_B32 = 2 };
 

@@ -12,15 +12,12 @@
 // per-expert grouped form for MoE layers.
 //
 // Structure: persistent CTAs (one per SM), 12 warps.
-//   warp 0 (one lane)   TMA producer: operand tiles (128B swizzle) into the stage ring, and
-//                       the scale atoms in chunks of GEMM_CHUNK_ATOMS per 128-row block
-//                       (4 k-stages at G = 32) into two chunk buffers of their own
-//   warp 1 (one lane)   MMA issuer: tcgen05.mma, tcgen05.commit; waits for scales once per
-//                       chunk, for operands once per stage
-//   warp 2              TMEM allocator, then (one lane) scale copier of odd chunks
-//   warp 3 (one lane)   scale copier of even chunks: tcgen05.cp of a chunk's atoms into that
-//                       chunk's TMEM scale set, back to back; copies issued by threads other
-//                       than the MMA issuer overlap the MMAs instead of queueing in front of them
+//   warp 0 (one lane)   TMA producer: operand tiles (128B swizzle) and scale atoms
+//   warp 1 (one lane)   MMA issuer: tcgen05.mma, tcgen05.commit
+//   warp 2              TMEM allocator, then (one lane) scale copier of odd stages
+//   warp 3 (one lane)   scale copier of even stages: tcgen05.cp of a stage's scale atoms into
+//                       that stage's own TMEM scale set; copies issued by threads other than
+//                       the MMA issuer overlap the MMAs instead of queueing in front of them
 //   warps 4..11         epilogue, two warps per TMEM lane quadrant (warp % 4), each owning half
 //                       of the accumulator columns: tcgen05.ld all of them in one round trip,
 //                       release the accumulator, then bf16 -> smem -> TMA store
@@ -46,34 +43,29 @@ struct GemmCfg {
   static constexpr int BROWS = BN / CG;                              // B rows this CTA loads
   static constexpr int A_BYTES = 128 * 128;
   static constexpr int B_BYTES = BROWS * 128;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;              // a multiple of 1 KB
-  // scales travel in chunks of CA atoms per 128-row block (SCH k-stages), apart from the ring
-  static constexpr int CA = GEMM_CHUNK_ATOMS;
-  static constexpr int SCH = CA / APS;
-  static constexpr int CSFA_BYTES = CA * 512;
-  static constexpr int CSFB_BYTES = (BN / 128) * CA * 512;           // every CTA holds all BN rows
-  static constexpr int CHUNK_BYTES = CSFA_BYTES + CSFB_BYTES;
-  static constexpr int CHUNKS = 2;
+  static constexpr int SFA_BYTES = APS * 512;
+  static constexpr int SFB_BYTES = (BN / 128) * APS * 512;           // every CTA holds all BN rows
+  static constexpr int STAGE_RAW = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
   static constexpr int EPI_WARPS = 8;                                // two per TMEM lane quadrant
   static constexpr int EPI_COLS = BN / 2;                            // accumulator columns per epilogue warp
   static constexpr int STAGING_BYTES = EPI_WARPS * 32 * 32;          // one 32x16 bf16 tile per epilogue warp
   static constexpr int BAR_BYTES = 1024;
   static constexpr int SMEM_LIMIT = 232448;
-  static constexpr int STAGES_FIT =
-      (SMEM_LIMIT - STAGING_BYTES - BAR_BYTES - 1024 - CHUNKS * CHUNK_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES_FIT = (SMEM_LIMIT - STAGING_BYTES - BAR_BYTES - 1024) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-  static constexpr int SMEM_TOTAL = STAGES * STAGE_BYTES + CHUNKS * CHUNK_BYTES + STAGING_BYTES + BAR_BYTES + 1024;
-  static constexpr int CSFA_COLS = CA * 4;
-  static constexpr int CSFB_COLS = CA * (BN / 32);
-  static constexpr int CHUNK_COLS = CSFA_COLS + CSFB_COLS;           // TMEM columns of one chunk's scales
-  static constexpr int ACC_STAGES = (2 * BN + CHUNKS * CHUNK_COLS <= 512) ? 2 : 1;
-  static constexpr int SF_COL = ACC_STAGES * BN;                     // chunk c's scales at SF_COL + c * CHUNK_COLS
+  static constexpr int SMEM_TOTAL = STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES + 1024;
+  static constexpr int SFA_COLS = APS * 4;
+  static constexpr int SFB_COLS = APS * (BN / 32);
+  static constexpr int SF_SET = SFA_COLS + SFB_COLS;                 // TMEM columns of one stage's scales
+  static constexpr int ACC_STAGES = (2 * BN + STAGES * SF_SET <= 512) ? 2 : 1;
+  static constexpr int SFA_COL = ACC_STAGES * BN;                    // scale set s starts at SFA_COL + s * SF_SET
+  static constexpr int SFB_COL = SFA_COL + SFA_COLS;
   static constexpr int TMEM_COLS = 512;
-  static constexpr uint32_t MAIN_TX = A_BYTES + B_BYTES;             // per CTA and stage
+  static constexpr uint32_t MAIN_TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // per CTA and stage
   static constexpr uint32_t COMP_TX = A_BYTES + B_BYTES;
-  static_assert(SF_COL + CHUNKS * CHUNK_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(SFA_COL + STAGES * SF_SET <= TMEM_COLS, "TMEM budget");
   static_assert(STAGES >= 2, "smem budget");
-  static_assert(SCH >= 1 && SCH * APS == CA, "chunk of whole stages");
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "tile width");
   static_assert(CG == 1 || (CG == 2 && BN == 256), "the CTA pair uses 256-wide tiles");
 };
@@ -120,9 +112,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw_addr + pad;
-  const uint32_t schunk0 = sbase + C::STAGES * C::STAGE_BYTES;      // the scale chunk buffers
-  const uint32_t s_staging = schunk0 + C::CHUNKS * C::CHUNK_BYTES;
-  uint8_t* bar_area = smem + C::STAGES * C::STAGE_BYTES + C::CHUNKS * C::CHUNK_BYTES + C::STAGING_BYTES;
+  const uint32_t s_staging = sbase + C::STAGES * C::STAGE_BYTES;
+  uint8_t* bar_area = smem + C::STAGES * C::STAGE_BYTES + C::STAGING_BYTES;
   const uint32_t bar0 = smem_u32(bar_area);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
@@ -130,14 +121,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   auto acce_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 2 + a); };
   const uint32_t tear_bar = bar0 + 8u * (2 * C::STAGES + 4);
   const uint32_t tear2_bar = bar0 + 8u * (2 * C::STAGES + 5);
-  const uint32_t tear3_bar = bar0 + 8u * (2 * C::STAGES + 6);
-  auto cfull_bar = [&](int c) { return bar0 + 8u * (2 * C::STAGES + 7 + c); };    // chunk landed
-  auto cready_bar = [&](int c) { return bar0 + 8u * (2 * C::STAGES + 9 + c); };   // chunk in TMEM
-  auto cempty_bar = [&](int c) { return bar0 + 8u * (2 * C::STAGES + 11 + c); };  // chunk's MMAs done
-  constexpr int NBARS = 2 * C::STAGES + 13;
-  static_assert(8 * NBARS + 16 <= C::BAR_BYTES, "barrier area");
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 8 * NBARS);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * NBARS + 8);
+  auto sfready_bar = [&](int s) { return bar0 + 8u * (2 * C::STAGES + 6 + s); };
+  const uint32_t tear3_bar = bar0 + 8u * (3 * C::STAGES + 6);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 8 * (3 * C::STAGES + 7));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 8 * (3 * C::STAGES + 7) + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = CG == 2 ? (int)cluster_ctarank() : 0;
@@ -148,7 +135,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     mbar_init(tear_bar, 1);
     mbar_init(tear2_bar, 1);
     mbar_init(tear3_bar, 1);
-    for (int c = 0; c < C::CHUNKS; ++c) { mbar_init(cfull_bar(c), 1); mbar_init(cready_bar(c), 1); mbar_init(cempty_bar(c), 1); }
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(sfready_bar(s), 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB); tma_prefetch_desc(&tmY);
@@ -172,31 +159,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------------ TMA producer
     int stage = 0; uint32_t phase = 0;
-    int cb = 0; uint32_t cphase = 0;
-    long long fills = 0, cfills = 0;
+    long long fills = 0;
     for (int t = unit; t < num_tiles; t += nunits) {
       const TileInfo ti = tile_info<CG>(t, p, BN, rank);
       const int brow = ti.n0 + rank * C::BROWS;
       bool ok = true;
       for (int ks = 0; ks < n_k && ok; ++ks) {
-        if (ks % C::SCH == 0) {
-          // the scale chunk of stages ks .. ks + SCH - 1 (atoms past K come zero-filled, unused)
-          if (!(ok = mbar_wait(cempty_bar(cb), cphase ^ 1, abort_flag, p.status))) break;
-          const uint32_t sc = schunk0 + cb * C::CHUNK_BYTES;
-          const int sfb_blk = ti.e * n_rb + ti.n0 / 128;
-          if constexpr (CG == 1) {
-            mbar_arrive_expect_tx(cfull_bar(cb), C::CHUNK_BYTES);
-            tma_load_3d(sc, &tmSFA, 0, ks * C::APS, ti.m0 / 128, cfull_bar(cb));
-            tma_load_3d(sc + C::CSFA_BYTES, &tmSFB, 0, ks * C::APS, sfb_blk, cfull_bar(cb));
-          } else {
-            const uint32_t fb = mapa_shared(cfull_bar(cb), 0);        // the leader counts both CTAs' bytes
-            if (leader) mbar_arrive_expect_tx(cfull_bar(cb), 2 * C::CHUNK_BYTES);
-            tma_load_3d_pair(sc, &tmSFA, 0, ks * C::APS, ti.m0 / 128, fb);
-            tma_load_3d_pair(sc + C::CSFA_BYTES, &tmSFB, 0, ks * C::APS, sfb_blk, fb);
-          }
-          ++cfills;
-          if (++cb == C::CHUNKS) { cb = 0; cphase ^= 1; }
-        }
         if (!(ok = mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, p.status))) break;
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
         if constexpr (CG == 1) {
@@ -204,11 +172,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           mbar_arrive_expect_tx(fb, C::MAIN_TX);
           tma_load_2d(st, &tmA, ks * 128, ti.m0, fb);
           tma_load_3d(st + C::A_BYTES, &tmB, ks * 128, brow, ti.e, fb);
+          tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFA, 0, ks * C::APS, ti.m0 / 128, fb);
+          tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, 0, ks * C::APS,
+                      ti.e * n_rb + ti.n0 / 128, fb);
         } else {
           const uint32_t fb = mapa_shared(full_bar(stage), 0);     // the leader counts both CTAs' bytes
           if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * C::MAIN_TX);
           tma_load_2d_pair(st, &tmA, ks * 128, ti.m0, fb);
           tma_load_3d_pair(st + C::A_BYTES, &tmB, ks * 128, brow, ti.e, fb);
+          tma_load_3d_pair(st + C::A_BYTES + C::B_BYTES, &tmSFA, 0, ks * C::APS, ti.m0 / 128, fb);
+          tma_load_3d_pair(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, 0, ks * C::APS,
+                           ti.e * n_rb + ti.n0 / 128, fb);
         }
         ++fills;
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
@@ -235,18 +209,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     }
     if (*abort_flag && leader) {
       // let the copies armed on this CTA's barriers land before the CTA exits
-      volatile int never = 0;
       const long long last = fills < C::STAGES ? fills : C::STAGES;
-      for (long long f = fills - last; f < fills; ++f)
+      for (long long f = fills - last; f < fills; ++f) {
+        volatile int never = 0;
         mbar_wait(full_bar((int)(f % C::STAGES)), (uint32_t)((f / C::STAGES) & 1), &never, nullptr, 100000000ull);
-      const long long clast = cfills < C::CHUNKS ? cfills : C::CHUNKS;
-      for (long long f = cfills - clast; f < cfills; ++f)
-        mbar_wait(cfull_bar((int)(f % C::CHUNKS)), (uint32_t)((f / C::CHUNKS) & 1), &never, nullptr, 100000000ull);
+      }
     }
   } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------------------------------------------------ MMA issuer
     int stage = 0; uint32_t phase = 0;
-    int cb = 0; uint32_t cphase = 0;
     int acc = 0; uint32_t aphase = 0;
     bool ok = true;
     for (int t = unit; t < num_tiles && ok; t += nunits) {
@@ -255,41 +226,35 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       tc_fence_after();
       const uint32_t d = tmem + acc * BN;
       for (int ks = 0; ks < n_k; ++ks) {
-        const int kc = ks % C::SCH;                       // stage within the scale chunk
-        if (kc == 0 && !(ok = mbar_wait(cready_bar(cb), cphase, abort_flag, p.status))) break;   // scales in TMEM
         if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, p.status))) break;
+        if (!(ok = mbar_wait(sfready_bar(stage), phase, abort_flag, p.status))) break;   // scales in TMEM
         tc_fence_after();
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
-        const uint32_t sfa0 = tmem + C::SF_COL + cb * C::CHUNK_COLS;     // this chunk's scale columns
-        const uint32_t sfb0 = sfa0 + C::CSFA_COLS;
+        const uint32_t sfo = tmem + stage * C::SF_SET;      // this stage's scale set
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const uint64_t ad = desc_kmajor_sw128(st + 32 * j);
           const uint64_t bd = desc_kmajor_sw128(st + C::A_BYTES + 32 * j);
           const uint32_t accum = (ks > 0 || j > 0) ? 1u : 0u;
           if constexpr (KIND == KIND_MXF4_B32) {
-            const uint32_t sf = 2 * (j & 1), atom = kc * C::APS + (j >> 1);
+            const uint32_t sf = 2 * (j & 1), atom = j >> 1;
             tc_mma_mxf4_b32_g<CG>(d, ad, bd, idesc_bs_m(FMT_MXF4_E2M1, C::MMA_M, BN, sf, sf),
-                                  sfa0 + 4 * atom, sfb0 + atom * (BN / 32), accum);
+                                  sfo + C::SFA_COL + 4 * atom, sfo + C::SFB_COL + atom * (BN / 32), accum);
           } else if constexpr (KIND == KIND_MXF4_B16) {
-            const uint32_t atom = kc * C::APS + j;
             tc_mma_mxf4_b16_g<CG>(d, ad, bd, idesc_bs_m(FMT_MXF4_E2M1, C::MMA_M, BN, 0, 0),
-                                  sfa0 + 4 * atom, sfb0 + atom * (BN / 32), accum);
+                                  sfo + C::SFA_COL + 4 * j, sfo + C::SFB_COL + j * (BN / 32), accum);
           } else {
             tc_mma_mxf8_g<CG>(d, ad, bd, idesc_bs_m(FMT_F8_E4M3, C::MMA_M, BN, j, j),
-                              sfa0 + 4 * kc, sfb0 + kc * (BN / 32), accum);
+                              sfo + C::SFA_COL, sfo + C::SFB_COL, accum);
           }
         }
         tc_commit_to<CG>(empty_bar(stage));
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
-        if (kc == C::SCH - 1 || ks == n_k - 1) {          // the chunk's MMAs are all issued
-          tc_commit_to<CG>(cempty_bar(cb));
-          if (++cb == C::CHUNKS) { cb = 0; cphase ^= 1; }
-        }
       }
       const int n_c = (ti.kl + 63) / 64;
       for (int c = 0; c < n_c && ok; ++c) {
         if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, p.status))) break;
+        if (!(ok = mbar_wait(sfready_bar(stage), phase, abort_flag, p.status))) break;   // keeps phases aligned
         tc_fence_after();
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
         const int nm = min(4, (ti.kl - 64 * c) / 16);
@@ -311,32 +276,38 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   } else if ((warp == 3 || warp == 2) && lane == 0 && leader) {
     // ------------------------------------------------------------------ scale copiers
     // Two copier threads (warps 3 and 2; warp 2 is free once TMEM is allocated) take alternate
-    // scale chunks. A chunk's TMEM set is free again once its buffer has been refilled: the
-    // producer reloads a buffer only after the MMAs that read the previous chunk there (and
-    // its TMEM set) have completed.
+    // stages of the sequence the MMA issuer walks: six atom copies take about one stage of MMA
+    // time when issued beside running MMAs, so a single copier falls behind. A stage's scale
+    // set is free once the stage's data has landed again (the producer refills a stage only
+    // after the MMAs that read it - and its scale set - have completed).
     const uint32_t mine = warp == 3 ? 0u : 1u;
-    int cb = 0; uint32_t cphase = 0;
-    uint32_t seq = 0;                                      // position in the chunk sequence
+    int stage = 0; uint32_t phase = 0;
+    uint32_t seq = 0;                                      // position in the stage sequence
     bool ok = true;
-    const int nch = (n_k + C::SCH - 1) / C::SCH;
     for (int t = unit; t < num_tiles && ok; t += nunits) {
-      for (int c = 0; c < nch; ++c, ++seq) {
+      const TileInfo ti = tile_info<CG>(t, p, BN, rank);
+      const int n_c = (ti.kl + 63) / 64;
+      for (int i = 0; i < n_k + n_c; ++i, ++seq) {
         if ((seq & 1u) == mine) {
-          if (!(ok = mbar_wait(cfull_bar(cb), cphase, abort_flag, p.status))) break;
-          tc_fence_after();
-          const uint32_t sc = schunk0 + cb * C::CHUNK_BYTES;
-          const uint32_t sfa0 = tmem + C::SF_COL + cb * C::CHUNK_COLS;
-          const uint32_t sfb0 = sfa0 + C::CSFA_COLS;
-          const int atoms = min(C::SCH, n_k - c * C::SCH) * C::APS;   // the atoms the chunk's MMAs read
-          for (int a = 0; a < atoms; ++a) {
-            tc_cp_atom<CG>(sfa0 + 4 * a, desc_scale_atom(sc + 512 * a));
+          if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, p.status))) break;
+          if (i < n_k) {
+            tc_fence_after();
+            const uint32_t s_sfa = sbase + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
+            const uint32_t s_sfb = s_sfa + C::SFA_BYTES;
+            const uint32_t sfo = tmem + stage * C::SF_SET;
 #pragma unroll
-            for (int r = 0; r < BN / 128; ++r)
-              tc_cp_atom<CG>(sfb0 + a * (BN / 32) + 4 * r, desc_scale_atom(sc + C::CSFA_BYTES + (r * C::CA + a) * 512));
+            for (int a = 0; a < C::APS; ++a) {
+              tc_cp_atom<CG>(sfo + C::SFA_COL + 4 * a, desc_scale_atom(s_sfa + 512 * a));
+#pragma unroll
+              for (int r = 0; r < BN / 128; ++r)
+                tc_cp_atom<CG>(sfo + C::SFB_COL + a * (BN / 32) + 4 * r, desc_scale_atom(s_sfb + (r * C::APS + a) * 512));
+            }
+            tc_commit_local<CG>(sfready_bar(stage));
+          } else {
+            mbar_arrive(sfready_bar(stage));               // compensation stages carry no scales
           }
-          tc_commit_local<CG>(cready_bar(cb));
         }
-        if (++cb == C::CHUNKS) { cb = 0; cphase ^= 1; }
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
     }
     if (*abort_flag) {
@@ -351,7 +322,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const int half = (warp - 4) >> 2;                  // which half of the accumulator columns
     const int ew = warp - 4;
     const uint32_t stg = s_staging + ew * (32 * 32);
-    uint8_t* stg_ptr = smem + C::STAGES * C::STAGE_BYTES + C::CHUNKS * C::CHUNK_BYTES + ew * (32 * 32);
+    uint8_t* stg_ptr = smem + C::STAGES * C::STAGE_BYTES + ew * (32 * 32);
     constexpr int NCH = C::EPI_COLS / 32;              // 32-column chunks per warp (4 or 2)
     int acc = 0; uint32_t aphase = 0;
     for (int t = unit; t < num_tiles; t += nunits) {
