@@ -187,16 +187,18 @@ OSC_API int osc_linear(const uint8_t* QX, const uint8_t* SX, const uint16_t* B,
                osc_stream_t stream);
 
 /* The product of osc_linear for few token rows, with the weight stream split over more SMs.
- * For M <= 128 the product is weight-bound: every call reads all of QW, SW and W_L. osc_linear
- * already computes it transposed (the weight tile as the 128-row tensor-core operand, the M
- * token rows as its narrow side), one 128-row weight tile per SM. osc_linear_splitk also
- * splits each tile's K range over S SMs: each part writes its fp32 partial product (M x N) into
- * `workspace`, and a second kernel on the same stream adds the S partials in a fixed order
- * (part 0 first) and rounds to bf16, so Y does not depend on timing. Arguments as osc_linear,
- * plus workspace: caller-allocated device memory of workspace_bytes bytes (16-byte aligned).
- * Its contents need no initial value and are left undefined; calls that share a workspace
- * must not overlap on the GPU. When workspace_bytes < osc_linear_workspace_bytes(M, N, K, K_L)
- * (or M > 128) the call runs exactly as osc_linear. */
+ * For M <= 16 (decoding) the product is weight-bound: every call reads all of QW, SW and W_L,
+ * and osc_linear gives each 128-row weight tile one SM. osc_linear_splitk computes the product
+ * transposed (the weight tile as the 128-row tensor-core operand, the token rows as its
+ * 16-wide side) and splits each tile's K range over S SMs: each part writes its fp32 partial
+ * product (M x N) into `workspace`, and a second kernel on the same stream adds the S partials
+ * in a fixed order (part 0 first) and rounds to bf16, so Y does not depend on timing.
+ * Arguments as osc_linear, plus workspace: caller-allocated device memory of workspace_bytes
+ * bytes (16-byte aligned). Its contents need no initial value and are left undefined; calls
+ * that share a workspace must not overlap on the GPU. osc_linear_workspace_bytes(M, N, K, K_L)
+ * gives the bytes the split needs, 0 when no split applies (M > 16, or the weight tiles
+ * alone fill the SMs); when no split applies or workspace_bytes is smaller, the call runs
+ * exactly as osc_linear. */
 OSC_API size_t osc_linear_workspace_bytes(int M, int N, int K, int K_L);
 OSC_API int osc_linear_splitk(const uint8_t* QX, const uint8_t* SX, const uint16_t* B,
                               const uint8_t* QW, const uint8_t* SW, const uint16_t* WL,
@@ -217,7 +219,7 @@ OSC_API int osc_linear_splitk(const uint8_t* QX, const uint8_t* SX, const uint16
  *     that device current); make that first call before any stream capture.
  *   - A call whose split needs more partial bytes than the buffer holds (S x M x N x 4, see
  *     osc_linear_workspace_bytes) returns OSC_ERR_SCRATCH and launches nothing; calls that
- *     need no split (M > 128, or one part per weight tile) use no scratch.
+ *     need no split (M > 16, or one part per weight tile) use no scratch.
  *   - Every call shares the one buffer and it keeps the last call's contents; nothing in it
  *     needs to start at zero (each call writes every partial it reads). Calls that overlap on
  *     the GPU (different streams, or different host threads without ordering) race on it. */

@@ -190,7 +190,7 @@ def test_argument_limits_of_every_entry_point(lib):
     wb = lib.osc_linear_workspace_bytes
     wb.argtypes = [I, I, I, I]
     wb.restype = ctypes.c_size_t
-    assert wb(129, 6144, 4096, 96) == 0 and wb(16, 6144, 4000, 96) == 0                # M > 128, K % 256
+    assert wb(17, 6144, 4096, 96) == 0 and wb(16, 6144, 4000, 96) == 0                 # M > 16, K % 256
     lib.osc_set_cta_pair.argtypes = [I]
     assert lib.osc_set_cta_pair(3) == -1
     prev = lib.osc_set_cta_pair(1)

@@ -256,15 +256,19 @@ def _prep(osc, X, W, G, L, K_L):
 
 
 def _split_and_plain(oracle, osc, X, W, G, L, K_L):
-    """osc_linear_splitk with its workspace (K split over several SMs, partials added by the
-    chained reduction) and osc_linear (one part per weight tile), each launched with and without
-    the fp32 output; both against the oracle on every row and column."""
+    """osc_linear_splitk with its workspace (at M <= 16: K split over several SMs, partials added
+    by the chained reduction; above that no split applies and it runs as osc_linear) and
+    osc_linear (one part per weight tile), each launched with and without the fp32 output; both
+    against the oracle on every row and column."""
     M, K = X.shape
     N = W.shape[0]
     QX, SX, B, QW, SW, WL = _prep(osc, X, W, G, L, K_L)
     nbytes = osc.osc_linear_workspace_bytes(M, N, K, K_L)
-    assert nbytes > 0 and nbytes % (4 * M * N) == 0                # S >= 2 parts of M x N fp32
-    ws = torch.empty(nbytes // 4, dtype=torch.float32, device="cuda")
+    if M <= 16:
+        assert nbytes > 0 and nbytes % (4 * M * N) == 0            # S >= 2 parts of M x N fp32
+    else:
+        assert nbytes == 0                                         # no split above 16 rows
+    ws = torch.empty(max(4, nbytes) // 4, dtype=torch.float32, device="cuda")
     Y = [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _ in range(4)]
     Yf = [torch.empty((M, N), dtype=torch.float32, device="cuda") for _ in range(2)]
     osc.osc_linear_splitk(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y[0], ws, Yf[0])
@@ -285,8 +289,9 @@ def _split_and_plain(oracle, osc, X, W, G, L, K_L):
 
 @pytest.mark.parametrize("M", [1, 5, 16, 33, 64, 100, 128])
 def test_few_rows_qkv(oracle, osc, M):
-    """Few token rows at the QKV shape: token tiles of 16, 32, 64 and 128 (ragged M inside each),
-    K split over several SMs, the compensation stages dealt out with the FP4 ones."""
+    """Few token rows at the QKV shape: the split product at M <= 16 (ragged M inside its 16-row
+    token tile, the compensation stages dealt out with the FP4 ones), the general kernel's
+    128-row tile at 33 .. 128 rows."""
     c = I.qkv_case(M)
     L = oracle.build_table(c.calib, 32)
     _split_and_plain(oracle, osc, c.X, c.W, 32, L, I.pad16(oracle.table_count(L)))
@@ -328,8 +333,7 @@ def test_few_rows_ragged_and_small_workspace(oracle, osc):
 
 
 def test_few_rows_fp8_fallback(oracle, osc):
-    """The MXFP8 product at few token rows takes the same transposed path (K = 12288, the W2
-    shape, 16 rows)."""
+    """The MXFP8 product at few token rows (K = 12288, the W2 shape, 16 rows)."""
     c = I.w2_case(M=16)
     M, K, N = 16, 12288, 4096
     QX, SX, _ = osc.alloc_quantize_outputs(M, K, 32, 0, fp8=True)

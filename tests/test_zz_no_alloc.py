@@ -67,7 +67,7 @@ def _close(ref, got):
 
 
 def test_noalloc_matches_the_workspace_form_on_two_calls_in_a_row(osc):
-    first = _layer(osc, 128)                         # fills the most of the buffer
+    first = _layer(osc, 16)                          # the most rows the split takes
     ref, got = _both(osc, first)
     _close(ref, got)
     second = _layer(osc, 5)                          # smaller: the first call's partials remain around it

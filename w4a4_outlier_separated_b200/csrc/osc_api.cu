@@ -120,32 +120,31 @@ int launch_result(cudaError_t e) { return e == cudaSuccess ? OSC_OK : fail_cuda(
 namespace {
 
 // The split plan of the few-row product: S parts of K per 128-row weight tile, so that
-// tiles x S CTAs (at most one per SM) stream the weights; S = 1 when there is no room for a
-// split or no workspace for its partials.
+// tiles x S CTAs (at most one per SM) stream the weights. S = 1 (no split: the general kernel
+// runs instead) above SPLIT_MAX_M token rows or when the tiles alone fill the SMs.
 struct SmallPlan {
   int S, n_tiles;
   size_t partial_bytes;
 };
-SmallPlan small_plan(int kind, int M, int N, int K, int K_L, int sms, bool with_workspace) {
+SmallPlan small_plan(int kind, int M, int N, int K, int K_L, int sms) {
   SmallPlan pl;
   pl.n_tiles = (N + 127) / 128;
   const int T = K / (kind == osc::KIND_MXF8_B32 ? 128 : 256) + (K_L + 63) / 64;
-  int S = with_workspace ? sms / std::max(1, pl.n_tiles) : 1;
+  int S = M <= osc::SPLIT_MAX_M ? sms / std::max(1, pl.n_tiles) : 1;
   S = std::max(1, std::min(S, std::min(8, T / 2)));
   pl.S = S;
   pl.partial_bytes = S > 1 ? (size_t)S * (size_t)M * (size_t)N * sizeof(float) : 0;
   return pl;
 }
 
-// Few-row product (M <= 128, dense calls): see osc_linear_small.cu.
+// Split few-row product (M <= SPLIT_MAX_M, dense calls with a workspace that holds the plan's
+// partials): see osc_linear_small.cu.
 int run_gemm_small(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const uint8_t* QW,
                    const uint8_t* SW, const uint16_t* WL, int M, int N, int K, int K_L, uint16_t* Y, float* Yf32,
-                   float* workspace, size_t workspace_bytes, const DeviceState* ds, cudaStream_t stream) {
+                   float* workspace, const SmallPlan& pl, const DeviceState* ds, cudaStream_t stream) {
   const bool fp8 = kind == osc::KIND_MXF8_B32;
   const int V = kind == osc::KIND_MXF4_B16 ? 16 : 32;
-  SmallPlan pl = small_plan(kind, M, N, K, K_L, ds->sms, workspace != nullptr);
-  if (pl.S > 1 && workspace_bytes < pl.partial_bytes) pl = small_plan(kind, M, N, K, K_L, ds->sms, false);
-  const int nt = osc::small_token_tile(M);
+  const int nt = osc::SPLIT_MAX_M;
   const uint64_t kb = fp8 ? (uint64_t)K : (uint64_t)K / 2;
   const int nslot4 = K / V / 4;
   const uint32_t aps = fp8 ? 1u : (V == 16 ? 4u : 2u);
@@ -181,10 +180,7 @@ int run_gemm_small(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_
   std::memset(&p, 0, sizeof(p));
   p.M = M; p.N = N; p.K = K; p.K_L = K_L;
   p.S = pl.S; p.n_tiles = pl.n_tiles; p.num_sms = ds->sms;
-  // a grid that leaves at least half the SMs free lets the next launch's CTAs start early:
-  // they prefetch their weights into L2 while this one runs
-  p.prefetch = pl.n_tiles * pl.S <= ds->sms / 2 ? 1 : 0;
-  p.Y = Y; p.Yf32 = Yf32; p.partial = pl.S > 1 ? workspace : nullptr;
+  p.Y = Y; p.Yf32 = Yf32; p.partial = workspace;
   p.status = ds->status;
   const int units = pl.n_tiles * pl.S;
   const int grid = units < ds->sms ? units : ds->sms;
@@ -204,10 +200,13 @@ int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
   int bn = g_tile_n.load();
   int cg = g_pair.load();
   const bool grouped = mblock_expert != nullptr;
-  // few token rows: the transposed product whose tensor work scales with the real row count,
-  // unless a tile shape was forced (the tests use that to reach the general kernel at small M)
-  if (!grouped && M <= 128 && bn == 0 && cg < 0)
-    return run_gemm_small(kind, QX, SX, B, QW, SW, WL, M, N, K, K_L, Y, Yf32, workspace, workspace_bytes, ds, stream);
+  // few token rows with a workspace for split partials: the transposed split product, unless
+  // a tile shape was forced (the tests use that to reach the general kernel there)
+  if (!grouped && workspace != nullptr && M <= osc::SPLIT_MAX_M && bn == 0 && cg < 0) {
+    const SmallPlan pl = small_plan(kind, M, N, K, K_L, ds->sms);
+    if (pl.S > 1 && workspace_bytes >= pl.partial_bytes)
+      return run_gemm_small(kind, QX, SX, B, QW, SW, WL, M, N, K, K_L, Y, Yf32, workspace, pl, ds, stream);
+  }
   if (bn == 0) bn = (N >= 256 && (long long)((M + 127) / 128) * ((N + 255) / 256) >= ds->sms) ? 256 : 128;
   // the CTA pair needs 256-wide tiles, whole 256-row tiles of work and a per-128-row expert map
   // it cannot honour, so grouped calls stay on single CTAs
@@ -489,10 +488,11 @@ int osc_linear(const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const ui
 }
 
 size_t osc_linear_workspace_bytes(int M, int N, int K, int K_L) {
-  if (M <= 0 || M > 128 || N <= 0 || K <= 0 || K_L < 0 || K % 256 != 0 || N % 16 != 0 || K_L % 16 != 0) return 0;
+  if (M <= 0 || M > osc::SPLIT_MAX_M || N <= 0 || K <= 0 || K_L < 0 || K % 256 != 0 || N % 16 != 0 || K_L % 16 != 0)
+    return 0;
   DeviceState* ds = nullptr;
   if (device_state(&ds) != OSC_OK) return 0;
-  return small_plan(osc::KIND_MXF4_B32, M, N, K, K_L, ds->sms, true).partial_bytes;
+  return small_plan(osc::KIND_MXF4_B32, M, N, K, K_L, ds->sms).partial_bytes;
 }
 
 int osc_linear_splitk(const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const uint8_t* QW, const uint8_t* SW,
@@ -686,7 +686,7 @@ extern "C" int osc_linear_splitk_noalloc(const uint8_t* QX, const uint8_t* SX, c
   DeviceState* ds = nullptr;
   if ((rc = device_state(&ds)) != OSC_OK) return rc;
   const int kind = G == 16 ? osc::KIND_MXF4_B16 : osc::KIND_MXF4_B32;
-  if (M <= 128 && small_plan(kind, M, N, K, K_L, ds->sms, true).partial_bytes > (size_t)OSC_NOALLOC_SCRATCH_BYTES)
+  if (small_plan(kind, M, N, K, K_L, ds->sms).partial_bytes > (size_t)OSC_NOALLOC_SCRATCH_BYTES)
     return OSC_ERR_SCRATCH;
   float* scratch = nullptr;
   if ((rc = noalloc_scratch(&scratch)) != OSC_OK) return rc;

@@ -128,7 +128,6 @@ cudaError_t launch_gemm(int kind, int bn, int cg, const GemmMaps& maps, const Ge
 struct SmallParams {
   int M, N, K, K_L;
   int S, n_tiles, num_sms;
-  int prefetch;          // 1: prefetch each unit's weights into L2 before the dependency wait
   uint16_t* Y;
   float* Yf32;
   float* partial;
@@ -137,7 +136,10 @@ struct SmallParams {
 struct SmallMaps {
   CUtensorMap w, x, sw, sx, wl, b;
 };
-int small_token_tile(int M);   // MMA N for M token rows: 16, 32, 64 or 128
+// The split few-row product serves osc_linear_splitk up to this many token rows (one 16-wide
+// token tile). Measured on the B200 at the QKV weights (K = 4096, N = 6144, cold): 8.8 / 9.4 us
+// at M = 1 / 16 against 10.1 us for the general kernel, which is as fast or faster from M = 32.
+constexpr int SPLIT_MAX_M = 16;
 // Scale atoms (512 bytes: 128 rows x 4 slots) one scale chunk of the few-row product holds
 // per operand: the host encodes the scale maps with boxes of this many atoms.
 constexpr int SMALL_CHUNK_ATOMS = 16;

@@ -1,21 +1,20 @@
-// OSC dual-path linear for few token rows (M <= 128), the weight-bound regime of decoding:
+// Split-K OSC dual-path linear for few token rows (M <= 16), the weight-bound regime of
+// decoding:
 //
 //   Y = (Q_X (x) Q_W) * S  +  B * W_L          (the OSC page, §3.2)
 //
 // computed transposed, Y^T = Q_W (x) Q_X^T + W_L * B^T: the weight tile is the MMA's 128-row
-// operand and the token rows its N (16, 32, 64 or 128), so the tensor-core work scales with the
-// real token count instead of a 128-row tile that is mostly padding (a 128 x 16 block-scaled
-// MMA costs an eighth of a 128 x 128 one). What remains is streaming the weights: Q_W, S_W and
-// W_L are read once, and their boxes are prefetched into L2 before the kernel waits for the
-// previous kernel of the stream (weights are not produced by it; a prefetch changes no value
-// any later load returns), so the weight stream overlaps the previous kernel's tail.
+// operand and the token rows its N = 16, so the tensor-core work scales with the real token
+// count instead of a 128-row tile that is mostly padding (a 128 x 16 block-scaled MMA costs an
+// eighth of a 128 x 128 one). What remains is streaming the weights: Q_W, S_W and W_L are read
+// once.
 //
-// Split K: a work unit is (128-row weight tile, part s of S). The k-stages of a tile (the FP4
+// A work unit is (128-row weight tile, part s of S), S >= 2. The k-stages of a tile (the FP4
 // stages, then the compensation stages of B * W_L) are dealt out in S equal runs, so S x tiles
-// CTAs stream weights at once instead of one per tile. With S > 1 each unit writes its fp32
-// partial (M x 128) to a caller-provided workspace and a second kernel, chained by programmatic
-// dependent launch, adds the S partials in the order s = 0 .. S-1 and rounds to bf16; with
-// S = 1 the unit writes Y itself. Either way the result does not depend on timing.
+// CTAs stream weights at once instead of one per tile. Each unit writes its fp32 partial
+// (M x 128) to a caller-provided workspace and a second kernel, chained by programmatic
+// dependent launch, adds the S partials in the order s = 0 .. S-1 and rounds to bf16, so the
+// result does not depend on timing.
 //
 // Roles (256 threads): warp 0 lane 0 TMA producer; warp 1 lane 0 MMA issuer; warp 2 TMEM
 // allocator; warp 3 lane 0 scale copier; warps 4..7 epilogue, warp w reading TMEM lanes
@@ -51,7 +50,7 @@ struct SmallCfg {
   static_assert(SF_COL + CHUNKS * CHUNK_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(STAGES >= 3, "smem budget");
   static_assert(SC >= 1 && SC * APS == SMALL_CHUNK_ATOMS, "chunk of whole stages");
-  static_assert(NT == 16 || NT == 32 || NT == 64 || NT == 128, "token tile");
+  static_assert(NT == 16, "token tile: one 16-row MMA N");
 };
 
 // Stage range [i0, i1) of unit (tile, s) among T = FP4 stages + compensation stages.
@@ -114,20 +113,6 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) grid_dep_launch();   // the split's reduction may be scheduled now
-  if (warp == 0 && lane == 0 && p.prefetch) {
-    // When the grid leaves SMs free, this CTA may start while the previous kernel still runs:
-    // the weights of its first two units go to L2 now. They are not that kernel's output, and
-    // a prefetch changes no value a later load returns.
-    for (int u = blockIdx.x, r = 0; u < units && r < 2; u += gridDim.x, ++r) {
-      const int tile = u / p.S, s = u % p.S, n0 = tile * 128;
-      int i0, i1;
-      unit_range(s, p.S, T, i0, i1);
-      for (int i = i0; i < i1; ++i) {
-        if (i < n_k) tma_prefetch_l2_2d(&tmW, i * 128, n0);
-        else tma_prefetch_l2_2d(&tmWL, (i - n_k) * 64, n0);
-      }
-    }
-  }
   grid_dep_wait();                           // Q_X, S_X and B of the previous kernel are visible
 
   if (warp == 0 && lane == 0) {
@@ -287,35 +272,13 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
       const int n = tile * 128 + 32 * q + lane;               // this thread's weight row = output column
       const bool col_ok = n < p.N;
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + acc * C::ACC_COLS;
+      uint32_t r[NT];
+      tmem_ld16(tbase, r);                                     // the NT = 16 token columns
+      tmem_ld_wait();
+      if (col_ok) {
 #pragma unroll
-      for (int c0 = 0; c0 < NT; c0 += (NT < 32 ? NT : 32)) {
-        constexpr int W = NT < 32 ? NT : 32;
-        uint32_t r[32];
-        if constexpr (W == 16) {
-          uint32_t r16[16];
-          tmem_ld16(tbase + c0, r16);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) r[i] = r16[i];
-        } else {
-          tmem_ld32(tbase + c0, r);
-          tmem_ld_wait();
-        }
-        if (col_ok) {
-#pragma unroll
-          for (int i = 0; i < W; ++i) {
-            const int m = c0 + i;
-            if (m < p.M) {
-              const float v = __uint_as_float(r[i]);
-              if (p.S == 1) {
-                p.Y[(size_t)m * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-                if (p.Yf32 != nullptr) p.Yf32[(size_t)m * p.N + n] = v;
-              } else {
-                p.partial[((size_t)s * p.M + m) * p.N + n] = v;
-              }
-            }
-          }
-        }
+        for (int m = 0; m < NT; ++m)
+          if (m < p.M) p.partial[((size_t)s * p.M + m) * p.N + n] = __uint_as_float(r[m]);
       }
       tc_fence_before();
       __syncwarp();
@@ -375,28 +338,14 @@ static cudaError_t launch_small_one(const SmallMaps& m, const SmallParams& p, in
   return cudaLaunchKernelEx(&cfg, gemm_small_kernel<NT, KIND>, m.w, m.x, m.sw, m.sx, m.wl, m.b, p);
 }
 
-template <int KIND>
-static cudaError_t launch_small_kind(int nt, const SmallMaps& m, const SmallParams& p, int grid, cudaStream_t s) {
-  switch (nt) {
-    case 16: return launch_small_one<16, KIND>(m, p, grid, s);
-    case 32: return launch_small_one<32, KIND>(m, p, grid, s);
-    case 64: return launch_small_one<64, KIND>(m, p, grid, s);
-    case 128: return launch_small_one<128, KIND>(m, p, grid, s);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-int small_token_tile(int M) { return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128)); }
-
 cudaError_t launch_gemm_small(int kind, const SmallMaps& maps, const SmallParams& p, int grid, cudaStream_t s) {
-  if (p.M < 1 || p.M > 128 || p.S < 1 || (p.S > 1 && p.partial == nullptr)) return cudaErrorInvalidValue;
-  const int nt = small_token_tile(p.M);
+  if (p.M < 1 || p.M > SPLIT_MAX_M || p.S < 2 || p.partial == nullptr) return cudaErrorInvalidValue;
   cudaError_t e;
-  if (kind == KIND_MXF4_B32) e = launch_small_kind<KIND_MXF4_B32>(nt, maps, p, grid, s);
-  else if (kind == KIND_MXF4_B16) e = launch_small_kind<KIND_MXF4_B16>(nt, maps, p, grid, s);
-  else if (kind == KIND_MXF8_B32) e = launch_small_kind<KIND_MXF8_B32>(nt, maps, p, grid, s);
+  if (kind == KIND_MXF4_B32) e = launch_small_one<SPLIT_MAX_M, KIND_MXF4_B32>(maps, p, grid, s);
+  else if (kind == KIND_MXF4_B16) e = launch_small_one<SPLIT_MAX_M, KIND_MXF4_B16>(maps, p, grid, s);
+  else if (kind == KIND_MXF8_B32) e = launch_small_one<SPLIT_MAX_M, KIND_MXF8_B32>(maps, p, grid, s);
   else return cudaErrorInvalidValue;
-  if (e != cudaSuccess || p.S == 1) return e;
+  if (e != cudaSuccess) return e;
   // the reduction: a grid of at most 2 x SMs CTAs, chained to the product by programmatic
   // dependent launch so that it is scheduled while the product runs
   const size_t quads = (size_t)p.M * p.N / 4;
