@@ -85,6 +85,23 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Bounded wait for the same phase parity on two barriers. The two try_waits go out back to
+// back, so when both phases are already complete (the common case in a k-loop that runs ahead
+// of its data) the caller pays one round trip to the barrier unit instead of two.
+__device__ __forceinline__ bool mbar_wait2(uint32_t bar_a, uint32_t bar_b, uint32_t parity, volatile int* abort,
+                                           int* status) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred pa, pb;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 pa, [%1], %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 pb, [%2], %3;\n\t"
+      "and.pred pa, pa, pb;\n\t"
+      "selp.u32 %0, 1, 0, pa;\n\t}"
+      : "=r"(ok) : "r"(bar_a), "r"(bar_b), "r"(parity) : "memory");
+  if (ok) return true;
+  return mbar_wait(bar_a, parity, abort, status) && mbar_wait(bar_b, parity, abort, status);
+}
+
 // ---- programmatic dependent launch -----------------------------------------------------------
 // The library's kernels are launched with programmatic stream serialization: a kernel may start
 // while the previous kernel of the stream is still running, so every thread runs

@@ -226,8 +226,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       tc_fence_after();
       const uint32_t d = tmem + acc * BN;
       for (int ks = 0; ks < n_k; ++ks) {
-        if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, p.status))) break;
-        if (!(ok = mbar_wait(sfready_bar(stage), phase, abort_flag, p.status))) break;   // scales in TMEM
+        // the stage's operands landed and its scales are in TMEM
+        if (!(ok = mbar_wait2(full_bar(stage), sfready_bar(stage), phase, abort_flag, p.status))) break;
         tc_fence_after();
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
         const uint32_t sfo = tmem + stage * C::SF_SET;      // this stage's scale set
@@ -253,8 +253,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       }
       const int n_c = (ti.kl + 63) / 64;
       for (int c = 0; c < n_c && ok; ++c) {
-        if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, p.status))) break;
-        if (!(ok = mbar_wait(sfready_bar(stage), phase, abort_flag, p.status))) break;   // keeps phases aligned
+        // (the compensation stages' scale barrier carries no scales; waiting on it keeps phases aligned)
+        if (!(ok = mbar_wait2(full_bar(stage), sfready_bar(stage), phase, abort_flag, p.status))) break;
         tc_fence_after();
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
         const int nm = min(4, (ti.kl - 64 * c) / 16);
