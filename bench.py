@@ -3,7 +3,8 @@
 Workload (default): the Qwen3-8B-shaped fused QKV projection, M=2048 tokens, K=4096,
 N=6144, G=32, table from Algorithm 1 (alpha=5) on 3x512 calibration tokens; synthetic seeded
 inputs with the outlier structure of the OSC page (its Qwen3 activations are not available).
-One step = osc_quantize(X) + osc_linear over one batch with the weights prepared offline.
+One step = osc_quantize_linear (osc_quantize of X, then osc_linear, issued by one C-ABI call)
+over one batch with the weights prepared offline.
 The metric counts the useful 2*M*N*K flops per step (the compensation flops are reported
 apart). The K timed steps run as one CUDA graph and rotate over 8 input sets (each with its
 own copy of the prepared weights, ~490 MB in all), so no step finds its inputs in L2;
@@ -211,8 +212,9 @@ def run_osc(args):
         osc.osc_linear(c["QX"], c["SX"], c["B"], c["QW"], c["SW"], c["WL"], M_, N_, K_, G_, K_L, c["Y"])
 
     def step(i):
-        quant(i)
-        lin(i)
+        c = sets[i % R]
+        osc.osc_quantize_linear(c["Xd"], G_, wl["Ld"], K_L, c["QX"], c["SX"], c["B"], c["QW"], c["SW"], c["WL"],
+                                N_, c["Y"])
 
     # K steps are captured once as one CUDA graph (the kernels are the ones the C-ABI calls
     # launch; no host launch overhead between them) and replayed as the timed region; the
@@ -297,8 +299,8 @@ def run_osc(args):
                 s_cmp.wait_event(ev_in[b])
                 if i >= 2:
                     s_cmp.wait_event(ev_out[b])                # step i-2's Y has left dY[b]
-                osc.osc_quantize(dX[b], G_, wl["Ld"], K_L, wl["QX"], wl["SX"], wl["B"])
-                osc.osc_linear(wl["QX"], wl["SX"], wl["B"], wl["QW"], wl["SW"], wl["WL"], M_, N_, K_, G_, K_L, dY[b])
+                osc.osc_quantize_linear(dX[b], G_, wl["Ld"], K_L, wl["QX"], wl["SX"], wl["B"], wl["QW"], wl["SW"],
+                                        wl["WL"], N_, dY[b])
                 ev_cmp[b].record(s_cmp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_cmp[b])
@@ -355,7 +357,7 @@ def run_osc(args):
             "e2e": {"value": round(weak_scaling_tflops(ws, flops, e2e_ms), 2), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": M_ * K_ * 2, "d2h_bytes_per_step": M_ * N_ * 2,
                     "ms_per_step": round(e2e_ms, 4),
-                    "how": "pinned host X in and Y out every step through osc_quantize + osc_linear; the input "
+                    "how": "pinned host X in and Y out every step through osc_quantize_linear; the input "
                            "copy of step i+1 and the output copy of step i-1 overlap step i's kernels on "
                            "separate streams (double-buffered device X and Y)"},
             "weight_bound": {
@@ -527,8 +529,8 @@ def _osc_dense_row(name, X, W, calib, G, steps, R, peaks):
         osc.osc_linear(c["QX"], c["SX"], c["B"], c["QW"], c["SW"], c["WL"], M, N, K, G, K_L, c["Y"])
 
     def step(i):
-        quant(i)
-        lin(i)
+        c = sets[i % R]
+        osc.osc_quantize_linear(c["X"], G, Ld, K_L, c["QX"], c["SX"], c["B"], c["QW"], c["SW"], c["WL"], N, c["Y"])
 
     for i in range(max(3, R)):
         step(i)
@@ -780,7 +782,7 @@ def scope_rows(steps: int):
             tiers[f"{mod}_choice"] = {"G": g, "tier": osc.TIERS[t],
                                       "path": "MXFP8 fallback" if g == 0 else f"OSC W4A4 G={g}"}
     out["tiers"] = tiers
-    out["how"] = ("per row: K steps (quantize + linear) as one CUDA graph between events, R rotating input sets "
+    out["how"] = ("per row: K steps (osc_quantize_linear: quantize + linear) as one CUDA graph between events, R rotating input sets "
                   "(each with its own weight copy) so that inputs exceed L2; linear_frac = useful flops against the "
                   "FP4 peak (bf16 burst x 4), or the FP8 peak (x 2) for MXFP8; linear_roofline_frac = the longer of "
                   "(MMA flops / tensor peak) and (linear_bytes / HBM) over the measured time, linear_bound names it; "

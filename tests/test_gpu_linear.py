@@ -70,6 +70,38 @@ def test_qkv(oracle, osc, M):
     _run_osc(oracle, osc, c.X, c.W, 32, L)
 
 
+@pytest.mark.parametrize("M, G, table", [(2048, 32, True), (2048, 16, True), (130, 64, True), (16, 32, True),
+                                          (300, 32, False)])
+def test_quantize_linear_matches_the_two_calls(oracle, osc, M, G, table):
+    """osc_quantize_linear (one call; the product starts reading its weights before the quantize
+    ends) against osc_quantize then osc_linear on the same inputs: Q_X, S_X, B, Y and the fp32
+    accumulator bit for bit, in the CTA-pair (M = 2048), single-CTA and ragged configurations,
+    with and without a table; the two-call Y is checked against the oracle elsewhere."""
+    c = I.qkv_case(M)
+    K, N = c.K, c.N
+    L = oracle.build_table(c.calib, G) if table else None
+    K_L = I.pad16(oracle.table_count(L)) if table else 0
+    Ld = to_dev(L) if table else None
+    QW, SW, WL = osc.prepare_weight(to_dev(c.W), G, Ld, K_L)
+    Xd = to_dev(c.X)
+    QX, SX, B = osc.quantize(Xd, G, Ld, K_L)
+    Y, Yf = osc.linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, want_f32=True)
+    QX2, SX2, B2 = osc.alloc_quantize_outputs(M, K, G, K_L, "cuda")
+    Y2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    Yf2 = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    Y3 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    osc.osc_quantize_linear(Xd, G, Ld, K_L, QX2, SX2, B2, QW, SW, WL, N, Y2, Yf2)
+    osc.osc_quantize_linear(Xd, G, Ld, K_L, QX2, SX2, B2, QW, SW, WL, N, Y3)
+    torch.cuda.synchronize()
+    assert osc.osc_status() == (0, 0)
+    assert torch.equal(QX2, QX) and torch.equal(SX2, SX)
+    if K_L:
+        assert torch.equal(B2, B)
+    assert torch.equal(Y2.view(torch.int16), Y.view(torch.int16))
+    assert torch.equal(Y3.view(torch.int16), Y.view(torch.int16))
+    assert torch.equal(Yf2, Yf)
+
+
 @pytest.mark.parametrize("G", [16, 64])
 def test_qkv_group_sizes_full_size(oracle, osc, G):
     """The QKV shape at G = 16 and 64 in the launch configuration the bench times (automatic

@@ -112,6 +112,9 @@ struct GemmParams {
   int num_groups;
   const int* mblock_expert;      // m_tiles entries (device)
   const int* group_kl;           // per-expert compensation width (device) or nullptr = K_L
+  // 1 (dense calls only): the kernel issued just before on the stream writes no weight operand,
+  // so the weight parts of the first tile's stages may be loaded before the dependency wait
+  int preload;
 };
 
 struct GemmMaps {

@@ -148,13 +148,36 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   if constexpr (CG == 2) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  grid_dep_wait();                       // the previous kernel's writes (Q_X, S_X, B) are visible
-  if (threadIdx.x == 0) grid_dep_launch();
-
   const int num_tiles = p.m_tiles * p.n_tiles;
   const int n_k = p.K / C::ELEMS;
   const int n_rb = (p.N + 127) / 128;
   const int unit = blockIdx.x / CG, nunits = gridDim.x / CG;
+  // With p.preload the producer issues the weight parts (B and its scales) of its first tile's
+  // first stages before the dependency wait, so they stream in while the previous kernel (the
+  // library's own quantize of X, which writes no weights) finishes; the activation parts follow
+  // after the wait. A stage's full barrier counts both parts.
+  int pre = 0;
+  if (warp == 0 && lane == 0 && p.preload && p.num_groups == 0 && unit < num_tiles) {
+    const TileInfo ti = tile_info<CG>(unit, p, BN, rank);   // dense: no device memory read
+    const int brow = ti.n0 + rank * C::BROWS;
+    pre = min(C::STAGES, n_k);
+    for (int ks = 0; ks < pre; ++ks) {
+      const uint32_t st = sbase + ks * C::STAGE_BYTES;
+      if constexpr (CG == 1) {
+        const uint32_t fb = full_bar(ks);
+        mbar_arrive_expect_tx(fb, C::MAIN_TX);
+        tma_load_3d(st + C::A_BYTES, &tmB, ks * 128, brow, 0, fb);
+        tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, 0, ks * C::APS, ti.n0 / 128, fb);
+      } else {
+        const uint32_t fb = mapa_shared(full_bar(ks), 0);
+        if (leader) mbar_arrive_expect_tx(full_bar(ks), 2 * C::MAIN_TX);
+        tma_load_3d_pair(st + C::A_BYTES, &tmB, ks * 128, brow, 0, fb);
+        tma_load_3d_pair(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, 0, ks * C::APS, ti.n0 / 128, fb);
+      }
+    }
+  }
+  grid_dep_wait();                       // the previous kernel's writes (Q_X, S_X, B) are visible
+  if (threadIdx.x == 0) grid_dep_launch();
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -167,22 +190,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       for (int ks = 0; ks < n_k && ok; ++ks) {
         if (!(ok = mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, p.status))) break;
         const uint32_t st = sbase + stage * C::STAGE_BYTES;
+        const bool w_issued = t == unit && ks < pre;            // weight parts issued before the wait
         if constexpr (CG == 1) {
           const uint32_t fb = full_bar(stage);
-          mbar_arrive_expect_tx(fb, C::MAIN_TX);
+          if (!w_issued) mbar_arrive_expect_tx(fb, C::MAIN_TX);
           tma_load_2d(st, &tmA, ks * 128, ti.m0, fb);
-          tma_load_3d(st + C::A_BYTES, &tmB, ks * 128, brow, ti.e, fb);
+          if (!w_issued) tma_load_3d(st + C::A_BYTES, &tmB, ks * 128, brow, ti.e, fb);
           tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFA, 0, ks * C::APS, ti.m0 / 128, fb);
-          tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, 0, ks * C::APS,
-                      ti.e * n_rb + ti.n0 / 128, fb);
+          if (!w_issued)
+            tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, 0, ks * C::APS,
+                        ti.e * n_rb + ti.n0 / 128, fb);
         } else {
           const uint32_t fb = mapa_shared(full_bar(stage), 0);     // the leader counts both CTAs' bytes
-          if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * C::MAIN_TX);
+          if (leader && !w_issued) mbar_arrive_expect_tx(full_bar(stage), 2 * C::MAIN_TX);
           tma_load_2d_pair(st, &tmA, ks * 128, ti.m0, fb);
-          tma_load_3d_pair(st + C::A_BYTES, &tmB, ks * 128, brow, ti.e, fb);
+          if (!w_issued) tma_load_3d_pair(st + C::A_BYTES, &tmB, ks * 128, brow, ti.e, fb);
           tma_load_3d_pair(st + C::A_BYTES + C::B_BYTES, &tmSFA, 0, ks * C::APS, ti.m0 / 128, fb);
-          tma_load_3d_pair(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, 0, ks * C::APS,
-                           ti.e * n_rb + ti.n0 / 128, fb);
+          if (!w_issued)
+            tma_load_3d_pair(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFB, 0, ks * C::APS,
+                             ti.e * n_rb + ti.n0 / 128, fb);
         }
         ++fills;
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
