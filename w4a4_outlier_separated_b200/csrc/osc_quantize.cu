@@ -562,8 +562,14 @@ __global__ void __launch_bounds__(NQ_THREADS, 1) rmsnorm_quantize_kernel(const _
     for (int i = 0; i < iters; ++i) {
       const int blk = lane + 32 * i;
       const bool valid = blk < nb;
+      const bool here = loaded && valid;                      // the lane holds a block of a real row
+      // the normalized block goes back over its x in the row buffer (same swizzle), so the
+      // table channels move out by address, as in the dense kernel, rather than by a select
+      // over the block's registers (fused quantize 11.85 -> 11.2 us at QKV M = 2048)
+      uint8_t* item = const_cast<uint8_t*>(buf) + blk * 64;
+      const int swz = (blk >> 1) & 3;
       uint32_t w[16];
-      if (loaded && valid) {
+      if (here) {
         uint32_t x[16], g[16];
         load_block_smem(buf, blk, x);
         load_block_smem(gam, blk, g);
@@ -573,13 +579,24 @@ __global__ void __launch_bounds__(NQ_THREADS, 1) rmsnorm_quantize_kernel(const _
           const float yhi = __fmul_rn(__fmul_rn(hi_f(x[j]), inv), hi_f(g[j]));
           w[j] = pack_bf16x2(ylo, yhi);
         }
-      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(item + ((c ^ swz) * 16)) = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+      }
+      if constexpr (TABLE) {
+        if (valid) {
+          const BlockTable t = block_table_packed<G>(blk, s_tab, p.R);
+          extract_from_item<G>(item, swz, t, here, here, p.B + (size_t)row * p.K_L);
+        }
+        if (loaded && blk == 0)                               // B's pad columns of a real row
+          for (int c = count; c < p.K_L; ++c) p.B[(size_t)row * p.K_L + c] = 0;
+      }
+      if (here) load_block_smem(buf, blk, w);
+      else {
 #pragma unroll
         for (int j = 0; j < 16; ++j) w[j] = 0u;
       }
-      BlockTable t = no_table();
-      if constexpr (TABLE) t = block_table_packed<G>(valid ? blk : 0, s_tab, p.R);
-      quant_block<G, false, TABLE>(w, (int)row, blk, loaded, t, count, p.K, p.K_L, p.B, p.Q, p.S, valid);
+      quant_block<G, false, false>(w, (int)row, blk, loaded, no_table(), count, p.K, p.K_L, p.B, p.Q, p.S, valid);
     }
     __syncwarp();                                             // every lane is done with this buffer
     const uint32_t nxt = row + (uint32_t)nslots * NQ_WARPS;
