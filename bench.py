@@ -585,8 +585,9 @@ def _rmsnorm_fused_row(name, X, W, calib, G, steps, R, peaks):
         osc.osc_linear(c["QX"], c["SX"], c["B"], c["QW"], c["SW"], c["WL"], M, N, K, G, K_L, c["Y"])
 
     def step(i):
-        fused(i)
-        lin(i)
+        c = sets[i % R]
+        osc.osc_rmsnorm_quantize_linear(c["X"], gbits, eps, G, Ld, K_L, c["QX"], c["SX"], c["B"], c["QW"], c["SW"],
+                                        c["WL"], N, c["Y"])
 
     for i in range(max(3, R)):
         step(i)
@@ -601,7 +602,7 @@ def _rmsnorm_fused_row(name, X, W, calib, G, steps, R, peaks):
             "fused_quantize_hbm_frac": round(qb / (f_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
             "unfused_norm_then_quantize_ms": round(u_ms, 5),
             "bytes_saved_per_step": 2 * M * K * 2,
-            "how": "fused = osc_rmsnorm_quantize; unfused = torch rms_norm (bf16 out, library kernel) then "
+            "how": "step = osc_rmsnorm_quantize_linear; fused = osc_rmsnorm_quantize; unfused = torch rms_norm (bf16 out, library kernel) then "
                    "osc_quantize; the fused kernel neither writes nor re-reads the normalized rows"}
 
 

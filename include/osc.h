@@ -197,6 +197,14 @@ OSC_API int osc_quantize_linear(const uint16_t* X, int M, int K, int G, const in
                                 uint8_t* QX, uint8_t* SX, uint16_t* B, const uint8_t* QW, const uint8_t* SW,
                                 const uint16_t* WL, int N, uint16_t* Y, float* Yf32, osc_stream_t stream);
 
+/* The same with the RMSNorm-fused quantize: osc_rmsnorm_quantize(X, gamma, eps, ...) then
+ * osc_linear on the same stream, in one call, with the arguments, outputs and errors of the two
+ * calls (K at most 6144); the product may start reading QW, SW and WL before the quantize ends. */
+OSC_API int osc_rmsnorm_quantize_linear(const uint16_t* X, const uint16_t* gamma, float eps, int M, int K, int G,
+                                        const int8_t* L, int R, int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B,
+                                        const uint8_t* QW, const uint8_t* SW, const uint16_t* WL, int N,
+                                        uint16_t* Y, float* Yf32, osc_stream_t stream);
+
 /* The product of osc_linear for few token rows, with the weight stream split over more SMs.
  * For M <= 16 (decoding) the product is weight-bound: every call reads all of QW, SW and W_L,
  * and osc_linear gives each 128-row weight tile one SM. osc_linear_splitk computes the product

@@ -198,6 +198,14 @@ def test_argument_limits_of_every_entry_point(lib):
     assert ql(p16, 4, 256, 32, p16, 1, 16, p16, p16, p16, p16, p16, None, 128, p16, None, None) == -1   # W_L missing
     assert ql(p16, 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 100, p16, None, None) == -2  # N % 16
     assert ql(V(p16.value + 2), 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, None) == -2
+    rl = lib.osc_rmsnorm_quantize_linear
+    rl.argtypes = [V, V, ctypes.c_float, I, I, I, V, I, I, V, V, V, V, V, V, I, V, V, V]
+    assert rl(None, None, 1e-6, 0, 256, 32, None, 1, 0, None, None, None, None, None, None, 128, None, None, None) == 0
+    assert rl(p16, p16, -1.0, 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, None) == -1
+    assert rl(p16, None, 1e-6, 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, None) == -1
+    assert rl(p16, p16, 1e-6, 4, 8192, 32, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, None) == -1
+    assert rl(p16, p16, 1e-6, 4, 256, 24, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, None) == -3
+    assert rl(p16, p16, 1e-6, 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 100, p16, None, None) == -2
     wb = lib.osc_linear_workspace_bytes
     wb.argtypes = [I, I, I, I]
     wb.restype = ctypes.c_size_t

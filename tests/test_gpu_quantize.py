@@ -283,6 +283,31 @@ def test_rmsnorm_quantize_qkv(oracle, osc, M):
     _check_rmsnorm_quant(oracle, osc, c.X, gamma, 1e-6, 32, L, K_L)
 
 
+@pytest.mark.parametrize("M, G", [(2048, 32), (130, 64)])
+def test_rmsnorm_quantize_linear_matches_the_two_calls(oracle, osc, M, G):
+    """osc_rmsnorm_quantize_linear (one call; the product may read its weights before the fused
+    quantize ends) against osc_rmsnorm_quantize then osc_linear: Q_X, S_X, B, Y and the fp32
+    accumulator bit for bit (the two-call outputs are checked against the oracle elsewhere)."""
+    c = I.qkv_case(M)
+    K, N = c.K, c.N
+    gamma = _gamma(K, G)
+    L = oracle.build_table(oracle.rmsnorm(c.calib[:512], gamma, 1e-6)[0], G)
+    K_L = I.pad16(oracle.table_count(L))
+    Ld, gd, Xd = to_dev(L), to_dev(gamma), to_dev(c.X)
+    QW, SW, WL = osc.prepare_weight(to_dev(c.W), G, Ld, K_L)
+    QX, SX, B = osc.rmsnorm_quantize(Xd, gd, 1e-6, G, Ld, K_L)
+    Y, Yf = osc.linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, want_f32=True)
+    QX2, SX2, B2 = osc.alloc_quantize_outputs(M, K, G, K_L, "cuda")
+    Y2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    Yf2 = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    osc.osc_rmsnorm_quantize_linear(Xd, gd, 1e-6, G, Ld, K_L, QX2, SX2, B2, QW, SW, WL, N, Y2, Yf2)
+    torch.cuda.synchronize()
+    assert osc.osc_status() == (0, 0)
+    assert torch.equal(QX2, QX) and torch.equal(SX2, SX) and torch.equal(B2, B)
+    assert torch.equal(Y2.view(torch.int16), Y.view(torch.int16))
+    assert torch.equal(Yf2, Yf)
+
+
 @pytest.mark.parametrize("G", [16, 64])
 def test_rmsnorm_quantize_group_sizes(oracle, osc, G):
     c = I.qkv_case(256)

@@ -515,6 +515,36 @@ int osc_quantize_linear(const uint16_t* X, int M, int K, int G, const int8_t* L,
                   nullptr, 0, true);
 }
 
+int osc_rmsnorm_quantize_linear(const uint16_t* X, const uint16_t* gamma, float eps, int M, int K, int G,
+                                const int8_t* L, int R, int K_L, uint8_t* QX, uint8_t* SX, uint16_t* B,
+                                const uint8_t* QW, const uint8_t* SW, const uint16_t* WL, int N, uint16_t* Y,
+                                float* Yf32, osc_stream_t stream) {
+  if (!valid_g(G)) return OSC_ERR_G;
+  if (R < 1 || R > osc::MAX_R) return OSC_ERR_ARG;
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return OSC_ERR_ARG;
+  if (M == 0 && N > 0 && K > 0 && K_L >= 0) return OSC_OK;  // nothing to read or write
+  // every argument of both steps is checked before anything is launched
+  if (!X || !gamma || M < 0 || K_L < 0) return OSC_ERR_ARG;
+  if (K > osc::NQ_MAX_K) return OSC_ERR_ARG;
+  if ((long long)(M + 127) * (K / 32) >= (1LL << 31)) return OSC_ERR_ARG;
+  if (L == nullptr && K_L != 0) return OSC_ERR_ARG;
+  if (K_L > 0 && (!B || !WL)) return OSC_ERR_ARG;
+  if (K_L > 32767) return OSC_ERR_ARG;
+  int rc = check_linear_common(QX, SX, QW, SW, M, N, K, Y, Yf32);
+  if (rc != OSC_OK) return rc;
+  if (!a16(X) || !a16(gamma) || (B && !a16(B)) || (WL && !a16(WL))) return OSC_ERR_ALIGN;
+  if (K_L % 16 != 0) return OSC_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(&ds)) != OSC_OK) return rc;
+  osc::NormQuantParams qp{X, gamma, eps, M, K, G, K / G, L, R, K_L, QX, SX, B, ds->status};
+  CUtensorMap tm;
+  if ((rc = make_row_map(&tm, X, M, K))) return rc;
+  if ((rc = launch_result(osc::launch_rmsnorm_quantize(tm, qp, ds->sms, (cudaStream_t)stream))) != OSC_OK) return rc;
+  const int kind = G == 16 ? osc::KIND_MXF4_B16 : osc::KIND_MXF4_B32;
+  return run_gemm(kind, QX, SX, B, QW, SW, WL, M, N, K, K_L, 1, nullptr, nullptr, Y, Yf32, (cudaStream_t)stream,
+                  nullptr, 0, true);
+}
+
 size_t osc_linear_workspace_bytes(int M, int N, int K, int K_L) {
   if (M <= 0 || M > osc::SPLIT_MAX_M || N <= 0 || K <= 0 || K_L < 0 || K % 256 != 0 || N % 16 != 0 || K_L % 16 != 0)
     return 0;

@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
             "osc_prepare_weight": ([P, i32, i32, i32, P, i32, i32, P, P, P, P], i32),
             "osc_linear": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P], i32),
             "osc_quantize_linear": ([P, i32, i32, i32, P, i32, i32, P, P, P, P, P, P, i32, P, P, P], i32),
+            "osc_rmsnorm_quantize_linear": ([P, P, f32, i32, i32, i32, P, i32, i32, P, P, P, P, P, P, i32, P, P, P],
+                                            i32),
             "osc_linear_workspace_bytes": ([i32, i32, i32, i32], ctypes.c_size_t),
             "osc_linear_splitk": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P, ctypes.c_size_t, P], i32),
             "osc_linear_splitk_noalloc": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P], i32),
@@ -213,6 +215,16 @@ def osc_quantize_linear(X, G: int, L, K_L: int, QX, SX, B, QW, SW, WL, N: int, Y
     _check("osc_quantize_linear", lib().osc_quantize_linear(
         _ptr(X), M, K, G, _ptr(L), _slots(L, K // G), K_L, _ptr(QX), _ptr(SX), _ptr(B) if K_L else None,
         _ptr(QW), _ptr(SW), _ptr(WL) if K_L else None, N, _ptr(Y), _ptr(Yf32), _stream(stream)))
+
+
+def osc_rmsnorm_quantize_linear(X, gamma, eps: float, G: int, L, K_L: int, QX, SX, B, QW, SW, WL, N: int, Y,
+                                Yf32=None, stream=None):
+    """osc_rmsnorm_quantize then osc_linear in one call; same outputs as the two calls."""
+    M, K = X.shape
+    _check("osc_rmsnorm_quantize_linear", lib().osc_rmsnorm_quantize_linear(
+        _ptr(X), _ptr(gamma), eps, M, K, G, _ptr(L), _slots(L, K // G), K_L, _ptr(QX), _ptr(SX),
+        _ptr(B) if K_L else None, _ptr(QW), _ptr(SW), _ptr(WL) if K_L else None, N, _ptr(Y), _ptr(Yf32),
+        _stream(stream)))
 
 
 def osc_linear_workspace_bytes(M: int, N: int, K: int, K_L: int) -> int:
