@@ -365,12 +365,15 @@ def run_osc(args):
                         "Q_X, S_X, B and Y per launch over its duration, for osc_linear_splitk (K split over "
                         "several SMs, fp32 partials in a workspace, chained reduction; 'us') and osc_linear "
                         "(one part per weight tile; 'us_one_part'); launches rotate over 10 weight copies "
-                        "(~146 MB > L2)",
+                        "(~146 MB > L2). The decoding step with its quantize: osc_quantize + osc_linear_splitk "
+                        "('step_two_calls_us') and osc_quantize_linear with the same workspace ('step_one_call_us')",
                 "unit": "GB/s", "peak": peaks["hbm_gbs"],
                 "lines": [{"M": d["M"], "us": round(d["us"], 2), "GBps": round(d["bytes"] / (d["us"] * 1e-6) / 1e9, 1),
                            "frac": round(d["bytes"] / (d["us"] * 1e-6) / 1e9 / peaks["hbm_gbs"], 3),
                            "us_one_part": round(d["us_one_part"], 2),
-                           "frac_one_part": round(d["bytes"] / (d["us_one_part"] * 1e-6) / 1e9 / peaks["hbm_gbs"], 3)}
+                           "frac_one_part": round(d["bytes"] / (d["us_one_part"] * 1e-6) / 1e9 / peaks["hbm_gbs"], 3),
+                           "step_two_calls_us": round(d["step_two_calls_us"], 2),
+                           "step_one_call_us": round(d["step_one_call_us"], 2)}
                           for d in wb]},
             "gpu_launches": 2 * args.steps,
             "clocks": clk.summary(),
@@ -406,16 +409,30 @@ def weight_bound(wl, steps: int):
             QW, SW, WL = wsets[i % R]
             osc.osc_linear_splitk(QX, SX, B, QW, SW, WL, M, N_, K_, G_, K_L, Y, ws)
 
+        Xm = wl["Xd"][:M].contiguous()
+
+        def step_two(i):                       # decoding step as two calls: quantize, split product
+            QW, SW, WL = wsets[i % R]
+            osc.osc_quantize(Xm, G_, wl["Ld"], K_L, QX, SX, B)
+            osc.osc_linear_splitk(QX, SX, B, QW, SW, WL, M, N_, K_, G_, K_L, Y, ws)
+
+        def step_one(i):                       # the same step as one call
+            QW, SW, WL = wsets[i % R]
+            osc.osc_quantize_linear(Xm, G_, wl["Ld"], K_L, QX, SX, B, QW, SW, WL, N_, Y, workspace=ws)
+
         for i in range(R):
             lin(i)
             lin_split(i)
+            step_two(i)
+            step_one(i)
         torch.cuda.synchronize()
-        us_plain, us_split = (t * 1e3 for t in _timed_graphs([lin, lin_split], steps))
+        us_plain, us_split, us_two, us_one = (t * 1e3 for t in _timed_graphs([lin, lin_split, step_two, step_one],
+                                                                             steps))
         _status_ok()
         nbytes = (wl["QW"].numel() + wl["SW"].numel() + wl["WL"].numel() * 2 + QX.numel() + SX.numel()
                   + (B.numel() * 2 if B is not None else 0) + Y.numel() * 2)
         out.append({"M": M, "us": us_split, "us_one_part": us_plain, "bytes": nbytes,
-                    "workspace_bytes": ws.numel() * 4})
+                    "workspace_bytes": ws.numel() * 4, "step_two_calls_us": us_two, "step_one_call_us": us_one})
     return out
 
 
@@ -916,8 +933,10 @@ def tail_order(res: dict) -> dict:
         wb = res["weight_bound"]
         out["weight_bound"] = {"unit": wb["unit"], "peak": wb["peak"],
                                "lines": [[d["M"], d["us"], d["GBps"], d["frac"], d.get("us_one_part"),
-                                          d.get("frac_one_part")] for d in wb["lines"]],
-                               "columns": ["M", "us", "GB/s", "frac", "us_one_part", "frac_one_part"],
+                                          d.get("frac_one_part"), d.get("step_two_calls_us"),
+                                          d.get("step_one_call_us")] for d in wb["lines"]],
+                               "columns": ["M", "us", "GB/s", "frac", "us_one_part", "frac_one_part",
+                                           "step_two_calls_us", "step_one_call_us"],
                                "what": wb["what"]}
     return out
 

@@ -187,15 +187,18 @@ OSC_API int osc_linear(const uint8_t* QX, const uint8_t* SX, const uint16_t* B,
                osc_stream_t stream);
 
 /* Figure 2 and the §3.2 equation in one call: osc_quantize(X, M, K, G, L, R, K_L, QX, SX, B)
- * then osc_linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y, Yf32) on the same stream, with the
- * same arguments, outputs and errors as the two calls (every argument is checked before either
- * kernel is launched; QX, SX and B are written as by osc_quantize). The results are identical
- * to the two calls. Because the library issues both kernels back to back, the product may start
- * reading QW, SW and WL (which the quantize does not write) before the quantize has finished.
- * As for any call, the weight operands must be complete before the call is issued. */
+ * then the product on the same stream: osc_linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y,
+ * Yf32) when workspace is NULL, else osc_linear_splitk(..., Y, Yf32, workspace,
+ * workspace_bytes) (see below: the split applies at M <= 16). Same arguments, outputs and errors
+ * as the two calls (every argument is checked before either kernel is launched; QX, SX and B
+ * are written as by osc_quantize), and results identical to them. Because the library issues
+ * both kernels back to back, the product may start reading QW, SW and WL (which the quantize
+ * does not write) before the quantize has finished. As for any call, the weight operands must
+ * be complete before the call is issued. */
 OSC_API int osc_quantize_linear(const uint16_t* X, int M, int K, int G, const int8_t* L, int R, int K_L,
                                 uint8_t* QX, uint8_t* SX, uint16_t* B, const uint8_t* QW, const uint8_t* SW,
-                                const uint16_t* WL, int N, uint16_t* Y, float* Yf32, osc_stream_t stream);
+                                const uint16_t* WL, int N, uint16_t* Y, float* Yf32, float* workspace,
+                                size_t workspace_bytes, osc_stream_t stream);
 
 /* The same with the RMSNorm-fused quantize: osc_rmsnorm_quantize(X, gamma, eps, ...) then
  * osc_linear on the same stream, in one call, with the arguments, outputs and errors of the two

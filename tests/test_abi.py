@@ -188,16 +188,16 @@ def test_argument_limits_of_every_entry_point(lib):
     assert sk(p16, p16, None, p16, p16, None, 4, 100, 256, 32, 0, p16, None, p16, 64, None) == -2    # N % 16
     assert sk(None, None, None, None, None, None, 0, 128, 256, 32, 0, None, None, None, 0, None) == 0  # M = 0
     ql = lib.osc_quantize_linear
-    ql.argtypes = [V, I, I, I, V, I, I, V, V, V, V, V, V, I, V, V, V]
-    assert ql(None, 0, 256, 32, None, 1, 0, None, None, None, None, None, None, 128, None, None, None) == 0  # M = 0
-    assert ql(p16, 4, 256, 24, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, None) == -3  # G
-    assert ql(p16, 4, 256, 32, p16, 4, 0, p16, p16, None, p16, p16, None, 128, p16, None, None) == -1   # R > 3
-    assert ql(None, 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, None) == -1  # X
-    assert ql(p16, 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 128, None, None, None) == -1  # Y
-    assert ql(p16, 4, 256, 32, None, 1, 16, p16, p16, p16, p16, p16, p16, 128, p16, None, None) == -1   # K_L, no table
-    assert ql(p16, 4, 256, 32, p16, 1, 16, p16, p16, p16, p16, p16, None, 128, p16, None, None) == -1   # W_L missing
-    assert ql(p16, 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 100, p16, None, None) == -2  # N % 16
-    assert ql(V(p16.value + 2), 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, None) == -2
+    ql.argtypes = [V, I, I, I, V, I, I, V, V, V, V, V, V, I, V, V, V, ctypes.c_size_t, V]
+    assert ql(None, 0, 256, 32, None, 1, 0, None, None, None, None, None, None, 128, None, None, None, 0, None) == 0  # M = 0
+    assert ql(p16, 4, 256, 24, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, None, 0, None) == -3  # G
+    assert ql(p16, 4, 256, 32, p16, 4, 0, p16, p16, None, p16, p16, None, 128, p16, None, None, 0, None) == -1   # R > 3
+    assert ql(None, 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, None, 0, None) == -1  # X
+    assert ql(p16, 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 128, None, None, None, 0, None) == -1  # Y
+    assert ql(p16, 4, 256, 32, None, 1, 16, p16, p16, p16, p16, p16, p16, 128, p16, None, None, 0, None) == -1   # K_L, no table
+    assert ql(p16, 4, 256, 32, p16, 1, 16, p16, p16, p16, p16, p16, None, 128, p16, None, None, 0, None) == -1   # W_L missing
+    assert ql(p16, 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 100, p16, None, None, 0, None) == -2  # N % 16
+    assert ql(V(p16.value + 2), 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, None, 0, None) == -2
     rl = lib.osc_rmsnorm_quantize_linear
     rl.argtypes = [V, V, ctypes.c_float, I, I, I, V, I, I, V, V, V, V, V, V, I, V, V, V]
     assert rl(None, None, 1e-6, 0, 256, 32, None, 1, 0, None, None, None, None, None, None, 128, None, None, None) == 0
@@ -206,6 +206,9 @@ def test_argument_limits_of_every_entry_point(lib):
     assert rl(p16, p16, 1e-6, 4, 8192, 32, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, None) == -1
     assert rl(p16, p16, 1e-6, 4, 256, 24, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, None) == -3
     assert rl(p16, p16, 1e-6, 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 100, p16, None, None) == -2
+    assert ql(p16, 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, None, 64, None) == -1  # bytes, no buffer
+    assert ql(p16, 4, 256, 32, None, 1, 0, p16, p16, None, p16, p16, None, 128, p16, None, V(p16.value + 4), 64,
+              None) == -2                                                                 # workspace alignment
     wb = lib.osc_linear_workspace_bytes
     wb.argtypes = [I, I, I, I]
     wb.restype = ctypes.c_size_t

@@ -70,13 +70,15 @@ def test_qkv(oracle, osc, M):
     _run_osc(oracle, osc, c.X, c.W, 32, L)
 
 
-@pytest.mark.parametrize("M, G, table", [(2048, 32, True), (2048, 16, True), (130, 64, True), (16, 32, True),
-                                          (300, 32, False)])
-def test_quantize_linear_matches_the_two_calls(oracle, osc, M, G, table):
+@pytest.mark.parametrize("M, G, table, split", [(2048, 32, True, False), (2048, 16, True, False),
+                                                 (130, 64, True, False), (16, 32, True, False),
+                                                 (300, 32, False, False), (16, 32, True, True), (5, 16, True, True)])
+def test_quantize_linear_matches_the_two_calls(oracle, osc, M, G, table, split):
     """osc_quantize_linear (one call; the product starts reading its weights before the quantize
-    ends) against osc_quantize then osc_linear on the same inputs: Q_X, S_X, B, Y and the fp32
-    accumulator bit for bit, in the CTA-pair (M = 2048), single-CTA and ragged configurations,
-    with and without a table; the two-call Y is checked against the oracle elsewhere."""
+    ends) against osc_quantize then osc_linear (or, with a workspace, osc_linear_splitk) on the
+    same inputs: Q_X, S_X, B, Y and the fp32 accumulator bit for bit, in the CTA-pair (M = 2048),
+    single-CTA, ragged and split (M <= 16) configurations, with and without a table; the
+    two-call outputs are checked against the oracle elsewhere."""
     c = I.qkv_case(M)
     K, N = c.K, c.N
     L = oracle.build_table(c.calib, G) if table else None
@@ -84,14 +86,24 @@ def test_quantize_linear_matches_the_two_calls(oracle, osc, M, G, table):
     Ld = to_dev(L) if table else None
     QW, SW, WL = osc.prepare_weight(to_dev(c.W), G, Ld, K_L)
     Xd = to_dev(c.X)
+    ws = None
+    if split:
+        nbytes = osc.osc_linear_workspace_bytes(M, N, K, K_L)
+        assert nbytes > 0
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
     QX, SX, B = osc.quantize(Xd, G, Ld, K_L)
-    Y, Yf = osc.linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, want_f32=True)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    Yf = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    if split:
+        osc.osc_linear_splitk(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y, ws, Yf)
+    else:
+        osc.osc_linear(QX, SX, B, QW, SW, WL, M, N, K, G, K_L, Y, Yf)
     QX2, SX2, B2 = osc.alloc_quantize_outputs(M, K, G, K_L, "cuda")
     Y2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     Yf2 = torch.empty((M, N), dtype=torch.float32, device="cuda")
     Y3 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    osc.osc_quantize_linear(Xd, G, Ld, K_L, QX2, SX2, B2, QW, SW, WL, N, Y2, Yf2)
-    osc.osc_quantize_linear(Xd, G, Ld, K_L, QX2, SX2, B2, QW, SW, WL, N, Y3)
+    osc.osc_quantize_linear(Xd, G, Ld, K_L, QX2, SX2, B2, QW, SW, WL, N, Y2, Yf2, workspace=ws)
+    osc.osc_quantize_linear(Xd, G, Ld, K_L, QX2, SX2, B2, QW, SW, WL, N, Y3, workspace=ws)
     torch.cuda.synchronize()
     assert osc.osc_status() == (0, 0)
     assert torch.equal(QX2, QX) and torch.equal(SX2, SX)

@@ -141,7 +141,7 @@ SmallPlan small_plan(int kind, int M, int N, int K, int K_L, int sms) {
 // partials): see osc_linear_small.cu.
 int run_gemm_small(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const uint8_t* QW,
                    const uint8_t* SW, const uint16_t* WL, int M, int N, int K, int K_L, uint16_t* Y, float* Yf32,
-                   float* workspace, const SmallPlan& pl, const DeviceState* ds, cudaStream_t stream) {
+                   float* workspace, const SmallPlan& pl, bool preload, const DeviceState* ds, cudaStream_t stream) {
   const bool fp8 = kind == osc::KIND_MXF8_B32;
   const int V = kind == osc::KIND_MXF4_B16 ? 16 : 32;
   const int nt = osc::SPLIT_MAX_M;
@@ -180,6 +180,7 @@ int run_gemm_small(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_
   std::memset(&p, 0, sizeof(p));
   p.M = M; p.N = N; p.K = K; p.K_L = K_L;
   p.S = pl.S; p.n_tiles = pl.n_tiles; p.num_sms = ds->sms;
+  p.preload = preload ? 1 : 0;
   p.Y = Y; p.Yf32 = Yf32; p.partial = workspace;
   p.status = ds->status;
   const int units = pl.n_tiles * pl.S;
@@ -205,7 +206,7 @@ int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
   if (!grouped && workspace != nullptr && M <= osc::SPLIT_MAX_M && bn == 0 && cg < 0) {
     const SmallPlan pl = small_plan(kind, M, N, K, K_L, ds->sms);
     if (pl.S > 1 && workspace_bytes >= pl.partial_bytes)
-      return run_gemm_small(kind, QX, SX, B, QW, SW, WL, M, N, K, K_L, Y, Yf32, workspace, pl, ds, stream);
+      return run_gemm_small(kind, QX, SX, B, QW, SW, WL, M, N, K, K_L, Y, Yf32, workspace, pl, preload, ds, stream);
   }
   if (bn == 0) bn = (N >= 256 && (long long)((M + 127) / 128) * ((N + 255) / 256) >= ds->sms) ? 256 : 128;
   // the CTA pair needs 256-wide tiles, whole 256-row tiles of work and a per-128-row expert map
@@ -490,7 +491,7 @@ int osc_linear(const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const ui
 
 int osc_quantize_linear(const uint16_t* X, int M, int K, int G, const int8_t* L, int R, int K_L, uint8_t* QX,
                         uint8_t* SX, uint16_t* B, const uint8_t* QW, const uint8_t* SW, const uint16_t* WL, int N,
-                        uint16_t* Y, float* Yf32, osc_stream_t stream) {
+                        uint16_t* Y, float* Yf32, float* workspace, size_t workspace_bytes, osc_stream_t stream) {
   if (!valid_g(G)) return OSC_ERR_G;
   if (R < 1 || R > osc::MAX_R) return OSC_ERR_ARG;
   if (M == 0 && N > 0 && K > 0 && K_L >= 0) return OSC_OK;  // nothing to read or write
@@ -504,6 +505,8 @@ int osc_quantize_linear(const uint16_t* X, int M, int K, int G, const int8_t* L,
   if (rc != OSC_OK) return rc;
   if (!a16(X) || (B && !a16(B)) || (WL && !a16(WL))) return OSC_ERR_ALIGN;
   if (K_L % 16 != 0) return OSC_ERR_ALIGN;
+  if (workspace_bytes > 0 && !workspace) return OSC_ERR_ARG;
+  if (workspace && !a16(workspace)) return OSC_ERR_ALIGN;
   DeviceState* ds = nullptr;
   if ((rc = device_state(&ds)) != OSC_OK) return rc;
   osc::QuantParams qp{X, M, K, G, K / G, L, R, K_L, QX, SX, B, ds->status};
@@ -512,7 +515,7 @@ int osc_quantize_linear(const uint16_t* X, int M, int K, int G, const int8_t* L,
   if ((rc = launch_result(osc::launch_quantize(tm, qp, false, ds->sms, (cudaStream_t)stream))) != OSC_OK) return rc;
   const int kind = G == 16 ? osc::KIND_MXF4_B16 : osc::KIND_MXF4_B32;
   return run_gemm(kind, QX, SX, B, QW, SW, WL, M, N, K, K_L, 1, nullptr, nullptr, Y, Yf32, (cudaStream_t)stream,
-                  nullptr, 0, true);
+                  workspace, workspace_bytes, true);
 }
 
 int osc_rmsnorm_quantize_linear(const uint16_t* X, const uint16_t* gamma, float eps, int M, int K, int G,

@@ -54,7 +54,8 @@ def lib() -> ctypes.CDLL:
             "osc_rmsnorm_quantize": ([P, P, f32, i32, i32, i32, P, i32, i32, P, P, P, P], i32),
             "osc_prepare_weight": ([P, i32, i32, i32, P, i32, i32, P, P, P, P], i32),
             "osc_linear": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P], i32),
-            "osc_quantize_linear": ([P, i32, i32, i32, P, i32, i32, P, P, P, P, P, P, i32, P, P, P], i32),
+            "osc_quantize_linear": ([P, i32, i32, i32, P, i32, i32, P, P, P, P, P, P, i32, P, P, P, ctypes.c_size_t, P],
+                                    i32),
             "osc_rmsnorm_quantize_linear": ([P, P, f32, i32, i32, i32, P, i32, i32, P, P, P, P, P, P, i32, P, P, P],
                                             i32),
             "osc_linear_workspace_bytes": ([i32, i32, i32, i32], ctypes.c_size_t),
@@ -208,13 +209,17 @@ def osc_linear(QX, SX, B, QW, SW, WL, M: int, N: int, K: int, G: int, K_L: int, 
                                           _stream(stream)))
 
 
-def osc_quantize_linear(X, G: int, L, K_L: int, QX, SX, B, QW, SW, WL, N: int, Y, Yf32=None, stream=None):
-    """osc_quantize then osc_linear in one call (the product may stream its weights while the
-    quantize finishes); same outputs as the two calls."""
+def osc_quantize_linear(X, G: int, L, K_L: int, QX, SX, B, QW, SW, WL, N: int, Y, Yf32=None, workspace=None,
+                        stream=None):
+    """osc_quantize then osc_linear (or, with a workspace, osc_linear_splitk) in one call: the
+    product may stream its weights while the quantize finishes; same outputs as the two calls.
+    `workspace`: a CUDA tensor (any dtype) for the split's fp32 partials, or None."""
     M, K = X.shape
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("osc_quantize_linear", lib().osc_quantize_linear(
         _ptr(X), M, K, G, _ptr(L), _slots(L, K // G), K_L, _ptr(QX), _ptr(SX), _ptr(B) if K_L else None,
-        _ptr(QW), _ptr(SW), _ptr(WL) if K_L else None, N, _ptr(Y), _ptr(Yf32), _stream(stream)))
+        _ptr(QW), _ptr(SW), _ptr(WL) if K_L else None, N, _ptr(Y), _ptr(Yf32), _ptr(workspace), nbytes,
+        _stream(stream)))
 
 
 def osc_rmsnorm_quantize_linear(X, gamma, eps: float, G: int, L, K_L: int, QX, SX, B, QW, SW, WL, N: int, Y,
