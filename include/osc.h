@@ -192,9 +192,9 @@ OSC_API int osc_linear(const uint8_t* QX, const uint8_t* SX, const uint16_t* B,
  * workspace_bytes) (see below: the split applies at M <= 16). Same arguments, outputs and errors
  * as the two calls (every argument is checked before either kernel is launched; QX, SX and B
  * are written as by osc_quantize), and results identical to them. Because the library issues
- * both kernels back to back, the product may start reading QW, SW and WL (which the quantize
- * does not write) before the quantize has finished. As for any call, the weight operands must
- * be complete before the call is issued. */
+ * both kernels back to back, the general product may start reading QW, SW and WL (which the
+ * quantize does not write) before the quantize has finished. As for any call, the weight
+ * operands must be complete before the call is issued. */
 OSC_API int osc_quantize_linear(const uint16_t* X, int M, int K, int G, const int8_t* L, int R, int K_L,
                                 uint8_t* QX, uint8_t* SX, uint16_t* B, const uint8_t* QW, const uint8_t* SW,
                                 const uint16_t* WL, int N, uint16_t* Y, float* Yf32, float* workspace,

@@ -141,7 +141,7 @@ SmallPlan small_plan(int kind, int M, int N, int K, int K_L, int sms) {
 // partials): see osc_linear_small.cu.
 int run_gemm_small(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, const uint8_t* QW,
                    const uint8_t* SW, const uint16_t* WL, int M, int N, int K, int K_L, uint16_t* Y, float* Yf32,
-                   float* workspace, const SmallPlan& pl, bool preload, const DeviceState* ds, cudaStream_t stream) {
+                   float* workspace, const SmallPlan& pl, const DeviceState* ds, cudaStream_t stream) {
   const bool fp8 = kind == osc::KIND_MXF8_B32;
   const int V = kind == osc::KIND_MXF4_B16 ? 16 : 32;
   const int nt = osc::SPLIT_MAX_M;
@@ -180,7 +180,6 @@ int run_gemm_small(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_
   std::memset(&p, 0, sizeof(p));
   p.M = M; p.N = N; p.K = K; p.K_L = K_L;
   p.S = pl.S; p.n_tiles = pl.n_tiles; p.num_sms = ds->sms;
-  p.preload = preload ? 1 : 0;
   p.Y = Y; p.Yf32 = Yf32; p.partial = workspace;
   p.status = ds->status;
   const int units = pl.n_tiles * pl.S;
@@ -206,7 +205,7 @@ int run_gemm(int kind, const uint8_t* QX, const uint8_t* SX, const uint16_t* B, 
   if (!grouped && workspace != nullptr && M <= osc::SPLIT_MAX_M && bn == 0 && cg < 0) {
     const SmallPlan pl = small_plan(kind, M, N, K, K_L, ds->sms);
     if (pl.S > 1 && workspace_bytes >= pl.partial_bytes)
-      return run_gemm_small(kind, QX, SX, B, QW, SW, WL, M, N, K, K_L, Y, Yf32, workspace, pl, preload, ds, stream);
+      return run_gemm_small(kind, QX, SX, B, QW, SW, WL, M, N, K, K_L, Y, Yf32, workspace, pl, ds, stream);
   }
   if (bn == 0) bn = (N >= 256 && (long long)((M + 127) / 128) * ((N + 255) / 256) >= ds->sms) ? 256 : 128;
   // the CTA pair needs 256-wide tiles, whole 256-row tiles of work and a per-128-row expert map

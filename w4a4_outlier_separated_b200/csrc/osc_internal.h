@@ -131,7 +131,6 @@ cudaError_t launch_gemm(int kind, int bn, int cg, const GemmMaps& maps, const Ge
 struct SmallParams {
   int M, N, K, K_L;
   int S, n_tiles, num_sms;
-  int preload;           // 1: weight parts of the first unit issued before the dependency wait
   uint16_t* Y;
   float* Yf32;
   float* partial;

@@ -114,30 +114,6 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) grid_dep_launch();   // the split's reduction may be scheduled now
-  // With p.preload (the kernel before this one is the library's own quantize, which writes no
-  // weight operand), the producer issues the weight parts of its first unit's first stages and
-  // scale chunks before the dependency wait, so they stream in while the quantize runs; the
-  // token parts follow after the wait, and each barrier counts both parts.
-  int pre = 0;
-  if (warp == 0 && lane == 0 && p.preload && (int)blockIdx.x < units) {
-    const int u = blockIdx.x, tile = u / p.S, s = u % p.S, n0 = tile * 128;
-    int i0, i1;
-    unit_range(s, p.S, T, i0, i1);
-    pre = min(C::STAGES, i1 - i0);
-    if (pre > C::CHUNKS * C::SC && i0 + C::CHUNKS * C::SC < n_k) pre = C::CHUNKS * C::SC;   // chunks fit the buffers
-    int c = 0;
-    for (int j = 0; j < pre; ++j) {
-      const int i = i0 + j;
-      if (i < n_k && j % C::SC == 0) {
-        mbar_arrive_expect_tx(cfull_bar(c), C::CHUNK_BYTES);
-        tma_load_3d(schunk0 + c * C::CHUNK_BYTES, &tmSW, 0, i * C::APS, n0 / 128, cfull_bar(c));
-        ++c;
-      }
-      mbar_arrive_expect_tx(full_bar(j), C::DATA_TX);
-      if (i < n_k) tma_load_2d(sbase + j * C::STAGE_BYTES, &tmW, i * 128, n0, full_bar(j));
-      else tma_load_2d(sbase + j * C::STAGE_BYTES, &tmWL, (i - n_k) * 64, n0, full_bar(j));
-    }
-  }
   grid_dep_wait();                           // Q_X, S_X and B of the previous kernel are visible
 
   if (warp == 0 && lane == 0) {
@@ -146,29 +122,11 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
     int cb = 0; uint32_t cphase = 0;
     long long fills = 0, cfills = 0;
     bool ok = true;
-    if (pre > 0) {
-      // the token parts of the stages and chunks armed before the wait
-      int i0, i1;
-      unit_range((int)blockIdx.x % p.S, p.S, T, i0, i1);
-      for (int j = 0; j < pre; ++j) {
-        const int i = i0 + j;
-        if (i < n_k && j % C::SC == 0) {
-          tma_load_3d(schunk0 + cb * C::CHUNK_BYTES + C::CHUNK_OP_BYTES, &tmSX, 0, i * C::APS, 0, cfull_bar(cb));
-          ++cfills;
-          if (++cb == C::CHUNKS) { cb = 0; cphase ^= 1; }
-        }
-        const uint32_t st = sbase + stage * C::STAGE_BYTES;
-        if (i < n_k) tma_load_2d(st + C::A_BYTES, &tmX, i * 128, 0, full_bar(stage));
-        else tma_load_2d(st + C::A_BYTES, &tmB, (i - n_k) * 64, 0, full_bar(stage));
-        ++fills;
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
-      }
-    }
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       const int tile = u / p.S, s = u % p.S, n0 = tile * 128;
       int i0, i1;
       unit_range(s, p.S, T, i0, i1);
-      for (int i = (u == (int)blockIdx.x ? i0 + pre : i0); i < i1; ++i) {
+      for (int i = i0; i < i1; ++i) {
         if (i < n_k && (i - i0) % C::SC == 0) {
           // the scale chunk of stages i .. i + SC - 1 (atoms past the unit's range are unused)
           if (!(ok = mbar_wait(cempty_bar(cb), cphase ^ 1, abort_flag, p.status))) break;
