@@ -159,7 +159,8 @@ def test_line_ends_with_the_kernel_figures():
     res = {"metric": "m", "value": 1.0, "kernels": {"osc_quantize_GBps": 2950.0, "osc_quantize_hbm_frac": 0.46},
            "weight_bound": {"unit": "GB/s", "peak": 6450.0, "what": "w",
                             "lines": [{"M": m, "us": 9.9, "GBps": 1490.0, "frac": 0.23, "us_one_part": 12.0,
-                                       "frac_one_part": 0.19} for m in (1, 16, 128)]},
+                                       "frac_one_part": 0.19, "step_two_calls_us": 11.5,
+                                       "step_one_call_us": 11.0} for m in (1, 16, 128)]},
            "roofline": {"frac": 0.5},
            "scope_rows": {f"row{i}": dict(row) for i in range(12)} | {"table2_osc_speedup_over_w8a8": {"G32": 1.35}},
            "cpu_baseline": {"value": 0.0035}}
@@ -168,5 +169,5 @@ def test_line_ends_with_the_kernel_figures():
     assert out["rows_brief"]["row3"] == [37.3, 0.54, 0.46] and out["rows_brief"]["table2"] == {"G32": 1.35}
     line = json.dumps(out)
     tail = line[-1500:]
-    assert '"osc_quantize_GBps": 2950.0' in tail and "[16, 9.9, 1490.0, 0.23, 12.0, 0.19]" in tail and '"row11"' in tail
+    assert '"osc_quantize_GBps": 2950.0' in tail and "[16, 9.9, 1490.0, 0.23, 12.0, 0.19, 11.5, 11.0]" in tail and '"row11"' in tail
     assert {"metric", "value", "roofline", "scope_rows", "cpu_baseline"} <= set(out)
