@@ -19,8 +19,11 @@
 //                       that stage's own TMEM scale set; copies issued by threads other than
 //                       the MMA issuer overlap the MMAs instead of queueing in front of them
 //   warps 4..11         epilogue, two warps per TMEM lane quadrant (warp % 4), each owning half
-//                       of the accumulator columns: tcgen05.ld all of them in one round trip,
+//                       of the accumulator columns: tcgen05.ld them 64 columns per round trip,
 //                       release the accumulator, then bf16 -> smem -> TMA store
+// With GemmParams::preload (set only when the kernel before it on the stream is the library's
+// own quantize) the producer issues the weight halves of its first tile's first stages before
+// griddepcontrol.wait.
 // CG = 2 runs the CTA pair of a 2-CTA cluster as one M = 256 tile: each CTA loads its 128
 // rows of A and half of the BN rows of B, the leader issues cta_group::2 MMAs over both
 // CTAs' shared memory, and each CTA's TMEM holds its 128 rows of the accumulator. Per SM this
