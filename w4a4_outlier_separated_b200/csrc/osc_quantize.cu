@@ -409,29 +409,38 @@ __global__ void __launch_bounds__(256) quantize_tma_kernel(const __grid_constant
     int rowa = (int)(it0 / (uint32_t)nblk);
     int blka = (int)(it0 - (uint32_t)rowa * nblk) + lane;
     while (blka >= nblk) { blka -= nblk; ++rowa; }
+    // the lane's items in three passes (extraction, loads, quantization), so that the
+    // quantization of its items is independent work the scheduler can interleave (QKV quantize
+    // 8.52 -> 8.39 us against one item after the other)
+    constexpr int NH = QSTEP / 32;
+    int rows[NH], blks[NH];
+    bool lives[NH];
 #pragma unroll
-    for (int h = 0; h < QSTEP / 32; ++h) {
+    for (int h = 0; h < NH; ++h) {
       const int r = lane + 32 * h;                            // item within the box
       int row = rowa, blk = blka + 32 * h;
       while (blk >= nblk) { blk -= nblk; ++row; }
-      const bool live = row < p.M;
-      uint8_t* item = box + r * 64;
-      const int swz = (r >> 1) & 3;
+      rows[h] = row; blks[h] = blk; lives[h] = row < p.M;
       if constexpr (TABLE) {
         // move the table channels out of the box (in table order), then clear B's pad columns
         const BlockTable t = block_table_packed<G>(blk, s_tab, p.R);
-        extract_from_item<G>(item, swz, t, loaded, live, p.B + (size_t)row * p.K_L);
-        if (live && blk == 0)
+        extract_from_item<G>(box + r * 64, (r >> 1) & 3, t, loaded, lives[h], p.B + (size_t)row * p.K_L);
+        if (lives[h] && blk == 0)
           for (int i = count; i < p.K_L; ++i) p.B[(size_t)row * p.K_L + i] = 0;
       }
-      uint32_t w[16];
-      if (loaded) load_block_smem(box, r, w);                 // rows past M arrive zero-filled
+    }
+    uint32_t w[NH][16];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      if (loaded) load_block_smem(box, lane + 32 * h, w[h]);  // rows past M arrive zero-filled
       else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) w[j] = 0u;
+        for (int j = 0; j < 16; ++j) w[h][j] = 0u;
       }
-      quant_block<G, FP8, false>(w, row, blk, live, no_table(), count, p.K, p.K_L, p.B, p.Q, p.S);
     }
+#pragma unroll
+    for (int h = 0; h < NH; ++h)
+      quant_block<G, FP8, false>(w[h], rows[h], blks[h], lives[h], no_table(), count, p.K, p.K_L, p.B, p.Q, p.S);
     __syncwarp();                                             // every lane is done with this slot
     if (step + 2 * wstride < cta_end) { fence_proxy_async_smem(); issue(step + 2 * wstride, slot); }
   }
