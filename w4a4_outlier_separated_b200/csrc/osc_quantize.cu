@@ -745,8 +745,12 @@ __global__ void __launch_bounds__(256) quantize_grouped_tma_kernel(const __grid_
     int blka = (int)(it0 - (uint32_t)ta * nblk) + lane;
     while (blka >= nblk) { blka -= nblk; ++ta; }
     int e_row = -1, e = 0, dest0 = 0;                         // expert lookup cached per dense row
+    // three passes over the lane's items (extraction, loads, quantization), as in the dense kernel
+    constexpr int NH = QSTEP / 32;
+    int rows[NH], blks[NH];
+    bool lives[NH];
 #pragma unroll
-    for (int h = 0; h < QSTEP / 32; ++h) {
+    for (int h = 0; h < NH; ++h) {
       const int r = lane + 32 * h;
       int t = ta, blk = blka + 32 * h;
       while (blk >= nblk) { blk -= nblk; ++t; }
@@ -757,16 +761,19 @@ __global__ void __launch_bounds__(256) quantize_grouped_tma_kernel(const __grid_
         e_row = t;
       }
       const int row = live ? dest0 + t : 0;
-      uint8_t* item = box + r * 64;
-      const int swz = (r >> 1) & 3;
+      rows[h] = row; blks[h] = blk; lives[h] = live;
       const BlockTable tb = live ? block_table_packed<G>(blk, s_tab + e * nt, p.R) : no_table();
-      extract_from_item<G>(item, swz, tb, true, live, p.B + (size_t)row * p.K_L);
+      extract_from_item<G>(box + r * 64, (r >> 1) & 3, tb, true, live, p.B + (size_t)row * p.K_L);
       if (live && blk == 0)
         for (int i = s_cnt[e]; i < p.K_L; ++i) p.B[(size_t)row * p.K_L + i] = 0;
-      uint32_t w[16];
-      load_block_smem(box, r, w);
-      quant_block<G, false, false>(w, row, blk, live, no_table(), 0, p.K, p.K_L, p.B, p.Q, p.S, live);
     }
+    uint32_t w[NH][16];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) load_block_smem(box, lane + 32 * h, w[h]);
+#pragma unroll
+    for (int h = 0; h < NH; ++h)
+      quant_block<G, false, false>(w[h], rows[h], blks[h], lives[h], no_table(), 0, p.K, p.K_L, p.B, p.Q, p.S,
+                                   lives[h]);
     __syncwarp();
     if (step + 2 * wstride < cta_end) { fence_proxy_async_smem(); issue(step + 2 * wstride, slot); }
   }
